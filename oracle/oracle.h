@@ -1,0 +1,136 @@
+/*
+ * oracle.h -- plain, slow CPU reference of the hybrid Mamba-2 / attention
+ * backbone frame step (TEST INFRASTRUCTURE ONLY).
+ *
+ * Only the test-suite, the smoke check and the benchmark's CPU-baseline leg
+ * may load this library.  It shares no code, header or table with the CUDA
+ * library; its inputs come from the seeded generator package (synth/) or from
+ * its own quantizer.
+ *
+ * Sources of the arithmetic (page titles and sections):
+ *  - "NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM, MLX": the LLM inside is
+ *    Nemotron-Nano-9B-v2, a 56-layer hybrid of Mamba-2 and attention,
+ *    GPTQ-quantized at group size 64; its per-frame step is bandwidth bound.
+ *  - "NemotronLabs VoiceChat" (SGLang-Omni cookbook): the thinker emits one
+ *    text and one function token per 80 ms frame, always greedy; backbone and
+ *    KV cache in bf16.
+ *  - The pages name the layer kinds but print no equations.  The plainest
+ *    reading is used: the Mamba-2 layer of Dao & Gu, "Transformers are SSMs"
+ *    (arXiv:2405.21060): causal depthwise conv1d over a ring of past inputs,
+ *    dt = softplus(dt_raw + dt_bias), decay a = exp(A*dt) with A = -exp(A_log),
+ *    state update h = a*h + dt*(x outer B), readout y = C.h + D*x, output
+ *    gate y*silu(z) followed by a grouped RMSNorm; GQA attention with no
+ *    positional encoding; a squared-ReLU MLP; pre-RMSNorm residual blocks.
+ *    The chunked prefill follows that paper's block decomposition of the
+ *    semiseparable matrix (its "SSD algorithm": diagonal blocks, chunk
+ *    states, state passing, off-diagonal outputs).
+ *
+ * Precision: all arithmetic in double.  Two modes:
+ *   OR_EXACT  -- no rounding at all (used for the invariant self-checks);
+ *   OR_MIRROR -- rounds to bf16 at the points where the GPU path stores a
+ *                bf16 tensor (listed in oracle.c, "storage points").
+ */
+#ifndef VC_ORACLE_H
+#define VC_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { OR_BF16 = 0, OR_W8 = 1, OR_W4 = 2, OR_W3 = 3 };
+enum { OR_EXACT = 0, OR_MIRROR = 1 };
+
+/* A linear weight W[N][K] (y = W u).
+ *   OR_BF16: q = uint16 bf16 bits, row-major [N][K]; scales/zeros unused.
+ *   OR_W8  : q = int8 two's complement, 4 per uint32 little-endian, row-major
+ *            [N][ceil(K/4)]; scales fp16 bits [N][ceil(K/group)]; symmetric.
+ *   OR_W4/OR_W3: q = b-bit unsigned codes as a little-endian bit stream along K,
+ *            [N][ceil(K*b/32)] uint32; scales fp16 [N][ng]; zeros b-bit stream
+ *            [N][ceil(ng*b/32)], ng = ceil(K/group); w = s*(q - z).          */
+typedef struct {
+    int fmt, group, N, K;
+    const void* q;
+    const uint16_t* scales;
+    const uint32_t* zeros;
+} or_mat;
+
+typedef struct {
+    int d_model;
+    const char* pattern;  /* one char per layer: 'M' Mamba-2, '*' attention, '-' MLP */
+    int ssm_heads, ssm_head_dim, ssm_state, ssm_groups, conv_width, norm_groups;
+    int attn_q_heads, attn_kv_heads, attn_head_dim;
+    int mlp_hidden, vocab_text, vocab_func;
+    double eps;
+} or_config;
+
+typedef struct {
+    const float* norm;                     /* [d] pre-RMSNorm gamma */
+    or_mat in_proj, out_proj;              /* Mamba-2: [E+Cx+H][d], [d][E] */
+    const float *conv_w, *conv_b;          /* [Cx][W] (k = W-1 multiplies the newest row), [Cx] */
+    const float *A_log, *D, *dt_bias;      /* [H] */
+    const float* gnorm;                    /* [E] gated-RMSNorm gamma */
+    or_mat qkv, o;                         /* attention: [(Hq+2Hk)Dh][d], [d][Hq*Dh] */
+    or_mat up, down;                       /* MLP: [F][d], [d][F] */
+} or_layer;
+
+typedef struct {
+    const or_layer* layers;                /* indexed by layer */
+    const float* final_norm;               /* [d] */
+    or_mat head_text, head_func;
+} or_weights;
+
+/* Session state, oracle's own logical layout (all double):
+ *   ssm  [n_mamba][n_slots][H][P][N]
+ *   conv [n_mamba][n_slots][W-1][Cx]   last W-1 pre-conv xBC rows, oldest first
+ *   k, v [n_attn][n_slots][Hk][cap][Dh]
+ *   ctx_len [n_slots] frames cached so far                                   */
+typedef struct {
+    int n_slots, kv_capacity;
+    double *ssm, *conv, *k, *v;
+    int32_t* ctx_len;
+} or_state;
+
+/* RTN group quantizer into the canonical packed format above; decisions in
+ * fp32 exactly as documented in oracle.c.  w is fp32 [N][K]. */
+void or_quantize(int fmt, int group, int N, int K, const float* w, uint32_t* q, uint16_t* scales,
+                 uint32_t* zeros);
+/* unpacked integer codes [N][K] (int32), zeros [N][ng] (0 for W8) and scales as
+ * double [N][ng] */
+void or_codes(const or_mat* W, int32_t* codes, int32_t* zeros, double* scales);
+/* dequantized W as double [N][K] (exact: s*(q-z) with s an fp16 value) */
+void or_dequant(const or_mat* W, double* out);
+/* y[N] = W u, u[K] (double) */
+void or_matvec(const or_mat* W, const double* u, double* y);
+
+/* One decode step for B sessions.  x: bf16 bits [B][d]; slots: [B] or NULL (=0..B-1).
+ * Outputs: tok_text/tok_func [B]; optional taps: hidden [n_layers+1][B][d]
+ * (residual stream after each layer, entry 0 = input), logits [2][B][V]
+ * (text then function), final_act [B][d] (normed input of the heads).
+ * Returns 0, or 1 if a session's cache is full (that session is skipped). */
+int or_step(const or_config* cfg, const or_weights* w, or_state* st, int B, const uint16_t* x,
+            const int32_t* slots, int mode, int32_t* tok_text, int32_t* tok_func, double* hidden,
+            double* logits);
+
+/* Prefill of T frames into one zero-initialised slot, layer by layer.
+ * ssd_chunk = 0: Mamba-2 layers use the sequential recurrence;
+ * ssd_chunk = Q > 0: they use the chunked SSD algorithm with chunk length Q.
+ * hidden (optional): [n_layers+1][T][d].  Sets ctx_len[slot] = T. */
+int or_prefill(const or_config* cfg, const or_weights* w, or_state* st, int slot, int T,
+               const uint16_t* x, int mode, int ssd_chunk, double* hidden);
+
+/* Isolated Mamba-2 mixer over T frames for one session (used by the kernel-level
+ * checks): input zxbcdt [T][E+Cx+H] (double), state in/out ssm [H][P][N] and
+ * conv history [W-1][Cx]; outputs the gated-norm input v [T][E] (= y*silu(z))
+ * and ysum [T][E] (= y before gating).  ssd_chunk as in or_prefill. */
+void or_mamba_mixer(const or_config* cfg, const or_layer* L, int T, const double* zxbcdt, double* ssm,
+                    double* conv, int ssd_chunk, double* y_out, double* v_out);
+
+/* Rounding helpers exposed for tests: RNE to bf16 / fp16 value, in double. */
+double or_round_bf16(double v);
+double or_round_fp16(double v);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,380 @@
+"""Pins of the CPU oracle against things other than itself (no GPU).
+
+  1. T decode steps == direct full-sequence evaluation (semiseparable SSM matrix,
+     full causal conv, masked softmax attention) on tiny inputs.
+  2. decode attention == full softmax attention (an attention-only stack).
+  3. dequantization: code round-trip against an independent numpy bit packer,
+     constructed weights s*(q-z) survive quantize -> dequantize bit-exactly,
+     quantized matvec == dense matvec on the dequantized matrix, and a
+     hand-worked quantizer example (tests/golden/quant_example.txt).
+  4. chunked SSD == sequential recurrence for several chunk lengths, ragged T
+     and a non-zero initial state.
+  5. closed forms: memoryless limit, pure decay with x = 0 and softplus(0) = ln 2,
+     relu^2 of negative pre-activations, argmax ties, the hand-worked scalar
+     SSM recurrence in tests/golden/ssm_scalar.txt.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.bruteforce import full_sequence
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def small_cfg(**kw):
+    base = dict(name="pin", d_model=64, pattern="M*-M", ssm_heads=4, ssm_head_dim=8, ssm_state=8, ssm_groups=2,
+                conv_width=4, norm_groups=2, attn_q_heads=6, attn_kv_heads=2, attn_head_dim=16, mlp_hidden=96,
+                vocab_text=80, vocab_func=48, wfmt=oracle.BF16, head_fmt=oracle.BF16, group_size=64,
+                kv_capacity=64, steps=20)
+    base.update(kw)
+    return synth.Config(**base)
+
+
+def run_steps(model, T, mode=oracle.EXACT, seed=0):
+    cfg = model.cfg
+    st = model.new_state(1, cfg.kv_capacity)
+    hid, lt, lf, xs = [], [], [], []
+    for t in range(T):
+        x = synth.frame_inputs(cfg, seed, t, 1)
+        xs.append(synth.bf16_to_f32(x)[0].astype(np.float64))
+        r = model.step(st, x, mode, taps=True)
+        hid.append(r["hidden"][:, 0, :])
+        lt.append(r["logits"][0, 0, :cfg.vocab_text])
+        lf.append(r["logits"][1, 0, :cfg.vocab_func])
+    return np.stack(xs), np.stack(hid, axis=1), np.stack(lt), np.stack(lf), st
+
+
+def rel_err(a, b):
+    return np.max(np.abs(a - b)) / max(np.sqrt(np.mean(b * b)), 1e-300)
+
+
+@pytest.mark.parametrize("cfg", [
+    small_cfg(),
+    small_cfg(wfmt=oracle.W8, head_fmt=oracle.W8, pattern="M-*-"),
+    small_cfg(wfmt=oracle.W4, pattern="*MM-"),
+    small_cfg(wfmt=oracle.W3, pattern="-M*", ssm_groups=1, norm_groups=1),
+    synth.tiny_config(),
+], ids=["bf16", "w8", "w4", "w3", "tiny"])
+def test_steps_equal_full_sequence(cfg):
+    model = oracle.Model(cfg, seed=3)
+    T = 20
+    X, hid, lt, lf, st = run_steps(model, T)
+    bh, blt, blf = full_sequence(model, X)
+    assert rel_err(hid, bh) < 1e-10
+    assert rel_err(lt, blt) < 1e-10
+    assert rel_err(lf, blf) < 1e-10
+    assert int(st.ctx_len[0]) == T
+
+
+def test_decode_attention_equals_full_softmax():
+    cfg = small_cfg(pattern="*", attn_q_heads=10, attn_kv_heads=2, attn_head_dim=32)
+    model = oracle.Model(cfg, seed=5)
+    X, hid, lt, lf, st = run_steps(model, 33)
+    bh, _, _ = full_sequence(model, X)
+    assert rel_err(hid[1], bh[1]) < 1e-10
+    # first frame: softmax over a single key, so the output is v itself
+    assert rel_err(hid[1][0], bh[1][0]) < 1e-12
+
+
+def test_first_frame_attention_is_value():
+    """ctx = 0: one key, weight 1, so o == v exactly; the layer output is r + W_o v."""
+    cfg = small_cfg(pattern="*")
+    model = oracle.Model(cfg, seed=11)
+    st = model.new_state(1, cfg.kv_capacity)
+    x = synth.frame_inputs(cfg, 11, 0, 1)
+    r = model.step(st, x, oracle.EXACT, taps=True)
+    u = synth.bf16_to_f32(x)[0].astype(np.float64)
+    g = model.small[0]["norm"].astype(np.float64)
+    un = u * g / np.sqrt(np.mean(u * u) + cfg.eps)
+    qkv = model.mats[(0, synth.K_QKV)].dequant() @ un
+    Dh, Hq, Hk = cfg.attn_head_dim, cfg.attn_q_heads, cfg.attn_kv_heads
+    v = qkv[(Hq + Hk) * Dh:].reshape(Hk, Dh)
+    o = np.concatenate([v[i * Hk // Hq] for i in range(Hq)])
+    expect = u + model.mats[(0, synth.K_O)].dequant() @ o
+    assert np.max(np.abs(r["hidden"][1, 0] - expect)) < 1e-12
+
+
+# ------------------------------------------------------------------------------------------------
+# quantization pins
+# ------------------------------------------------------------------------------------------------
+
+def np_pack(codes, bits):
+    """independent bit packer: element k occupies bits [k*b, k*b+b) of a little-endian stream"""
+    N, K = codes.shape
+    words = (K * bits + 31) // 32
+    out = np.zeros((N, words), np.uint64)
+    for k in range(K):
+        o = k * bits
+        w, sh = o // 32, o % 32
+        c = codes[:, k].astype(np.uint64) & np.uint64((1 << bits) - 1)
+        out[:, w] |= (c << np.uint64(sh)) & np.uint64(0xFFFFFFFF)
+        if sh + bits > 32:
+            out[:, w + 1] |= c >> np.uint64(32 - sh)
+    return out.astype(np.uint32)
+
+
+@pytest.mark.parametrize("fmt", [oracle.W8, oracle.W4, oracle.W3])
+@pytest.mark.parametrize("K", [64, 100, 192])
+def test_codes_roundtrip(fmt, K):
+    bits = oracle.BITS[fmt]
+    N, G = 7, 64
+    ng = (K + G - 1) // G
+    if fmt == oracle.W8:
+        codes = synth.uniform_i32(9, K, (N, K), -127, 127)
+        zeros = np.zeros((N, ng), np.int32)
+        zw = None
+    else:
+        codes = synth.uniform_i32(9, K, (N, K), 0, (1 << bits) - 1)
+        zeros = synth.uniform_i32(10, K, (N, ng), 0, (1 << bits) - 1)
+        zw = np_pack(zeros, bits)
+    scales = synth.uniform_f32(11, K, (N, ng), 0.001, 0.1).astype(np.float16).view(np.uint16)
+    m = oracle.Mat(fmt, G, N, K, np_pack(codes, bits), scales, zw)
+    c2, z2, s2 = m.codes()
+    assert np.array_equal(c2, codes)
+    assert np.array_equal(z2, zeros)
+    assert np.array_equal(s2, scales.view(np.float16).astype(np.float64))
+    deq = m.dequant()
+    gidx = np.arange(K) // G
+    expect = s2[:, gidx] * (codes - zeros[:, gidx])
+    assert np.array_equal(deq, expect)
+
+
+@pytest.mark.parametrize("fmt", [oracle.W8, oracle.W4, oracle.W3])
+def test_constructed_weights_survive_quantization(fmt):
+    """w = s*(q - z) with each group spanning the full code range quantizes back to
+    exactly (q, s, z), so dequantize(quantize(w)) == w bit-exactly."""
+    bits = oracle.BITS[fmt]
+    Q = (1 << bits) - 1
+    N, K, G = 9, 256, 64
+    ng = K // G
+    s = synth.uniform_f32(1, 1, (N, ng), 0.002, 0.05).astype(np.float16).astype(np.float32)
+    if fmt == oracle.W8:
+        q = synth.uniform_i32(1, 2, (N, K), -127, 127)
+        q[:, ::G] = 127                       # amax hits the code limit in every group
+        z = np.zeros((N, ng), np.int32)
+    else:
+        q = synth.uniform_i32(1, 2, (N, K), 0, Q)
+        q[:, ::G] = 0
+        q[:, 1::G] = Q                        # max - min = s * Q in every group
+        z = synth.uniform_i32(1, 3, (N, ng), 0, Q)
+    gidx = np.arange(K) // G
+    w = (s[:, gidx] * (q - z[:, gidx]).astype(np.float32)).astype(np.float32)
+    m = oracle.quantize(fmt, G, w)
+    c2, z2, s2 = m.codes()
+    assert np.array_equal(c2, q)
+    assert np.array_equal(z2, z)
+    assert np.array_equal(s2.astype(np.float32), s)
+    assert np.array_equal(m.dequant(), w.astype(np.float64))
+
+
+@pytest.mark.parametrize("fmt", [oracle.BF16, oracle.W8, oracle.W4, oracle.W3])
+def test_quantized_matvec_equals_dense(fmt):
+    N, K = 37, 320
+    w = synth.normal_f32(4, 4, (N, K), 0.0, 0.02)
+    m = oracle.bf16_mat(synth.f32_to_bf16(w)) if fmt == oracle.BF16 else oracle.quantize(fmt, 64, w)
+    u = synth.normal_f32(4, 5, (K,)).astype(np.float64)
+    assert np.allclose(m.matvec(u), m.dequant() @ u, rtol=1e-13, atol=1e-13)
+    # RTN error: half a step inside the grid; the fp16 scale and the rounded zero point can
+    # push a group's extreme one step further (clamped), never more
+    if fmt != oracle.BF16:
+        _, _, s = m.codes()
+        err = np.abs(m.dequant() - w)
+        step = np.repeat(s, 64, axis=1)[:, :K]
+        assert np.all(err <= step * (1 + 1e-6))
+        assert np.mean(err <= 0.5 * step * (1 + 1e-6)) > 0.95
+
+
+def read_golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            k, v = line.split("=", 1)
+            vals[k.strip()] = [float(t) for t in v.split()]
+    return vals
+
+
+def test_quantizer_hand_example():
+    g = read_golden("quant_example.txt")
+    w = np.array([g["w"]], np.float32)
+    m = oracle.quantize(oracle.W4, 8, w)
+    c, z, s = m.codes()
+    assert s[0, 0] == g["scale_w4"][0]
+    assert z[0, 0] == g["zero_w4"][0]
+    assert list(c[0]) == [int(v) for v in g["codes_w4"]]
+    m8 = oracle.quantize(oracle.W8, 8, w)
+    c8, _, s8 = m8.codes()
+    assert s8[0, 0] == g["scale_w8"][0]
+    assert list(c8[0]) == [int(v) for v in g["codes_w8"]]
+
+
+def test_rounding_helpers():
+    assert oracle.round_bf16(1.0 + 2 ** -8) == 1.0          # tie -> even
+    assert oracle.round_bf16(1.0 + 3 * 2 ** -8) == 1.0 + 2 ** -6
+    assert oracle.round_fp16(1.0 + 2 ** -11) == 1.0
+    assert oracle.round_fp16(2 ** -24 * 1.5) == 2 ** -23      # subnormal tie -> even
+    assert oracle.round_fp16(0.1) == float(np.float16(0.1))
+
+
+# ------------------------------------------------------------------------------------------------
+# SSD chunked == sequential
+# ------------------------------------------------------------------------------------------------
+
+def mixer_inputs(cfg, model, T, seed):
+    R = cfg.in_proj_rows
+    zx = synth.normal_f32(seed, 77, (T, R), 0.0, 1.0).astype(np.float64)
+    ssm0 = synth.normal_f32(seed, 78, (cfg.ssm_heads, cfg.ssm_head_dim, cfg.ssm_state)).astype(np.float64)
+    conv0 = synth.normal_f32(seed, 79, (cfg.conv_width - 1, cfg.conv_dim)).astype(np.float64)
+    return zx, ssm0, conv0
+
+
+@pytest.mark.parametrize("Q", [1, 3, 16, 64, 256, 70])
+@pytest.mark.parametrize("T", [70, 37])
+def test_ssd_chunked_equals_sequential(Q, T):
+    cfg = small_cfg(pattern="M")
+    model = oracle.Model(cfg, seed=2)
+    zx, ssm0, conv0 = mixer_inputs(cfg, model, T, 2)
+    s1, c1 = ssm0.copy(), conv0.copy()
+    y1, v1 = model.mamba_mixer(0, zx, s1, c1, 0)
+    s2, c2 = ssm0.copy(), conv0.copy()
+    y2, v2 = model.mamba_mixer(0, zx, s2, c2, Q)
+    assert rel_err(y2, y1) < 1e-10
+    assert rel_err(s2, s1) < 1e-10
+    assert np.array_equal(c1, c2)
+
+
+def test_prefill_chunked_equals_steps():
+    cfg = small_cfg(pattern="M*-M", kv_capacity=80)
+    model = oracle.Model(cfg, seed=8)
+    T = 45
+    xb = synth.prefill_inputs(cfg, 8, T)
+    st1 = model.new_state(1, cfg.kv_capacity)
+    for t in range(T):
+        model.step(st1, xb[t:t + 1], oracle.EXACT)
+    st2 = model.new_state(1, cfg.kv_capacity)
+    model.prefill(st2, 0, xb, oracle.EXACT, ssd_chunk=16)
+    assert rel_err(st2.ssm, st1.ssm) < 1e-10
+    assert rel_err(st2.conv, st1.conv) < 1e-12
+    assert rel_err(st2.k[:, :, :, :T], st1.k[:, :, :, :T]) < 1e-10
+    assert rel_err(st2.v[:, :, :, :T], st1.v[:, :, :, :T]) < 1e-10
+    assert st2.ctx_len[0] == st1.ctx_len[0] == T
+
+
+# ------------------------------------------------------------------------------------------------
+# closed forms
+# ------------------------------------------------------------------------------------------------
+
+def test_memoryless_limit():
+    """A_log large => a = exp(A dt) underflows to 0: y = (C.B) dt x + D x per frame."""
+    cfg = small_cfg(pattern="M")
+    model = oracle.Model(cfg, seed=4)
+    model.small[0]["A_log"][:] = 8.0            # A = -2981, a = exp(-2981 dt) == 0
+    T = 6
+    zx, ssm0, conv0 = mixer_inputs(cfg, model, T, 4)
+    y, _ = model.mamba_mixer(0, zx, ssm0.copy(), conv0.copy(), 0)
+    # conv output recomputed directly
+    E, Cx, G, N, H, P = cfg.d_inner, cfg.conv_dim, cfg.ssm_groups, cfg.ssm_state, cfg.ssm_heads, cfg.ssm_head_dim
+    sp = model.small[0]
+    seq = np.vstack([conv0, zx[:, E:E + Cx]])
+    for t in range(T):
+        pre = sp["conv_b"] + np.sum(sp["conv_w"].T * seq[t:t + 4], axis=0)
+        xc = pre / (1 + np.exp(-pre))
+        dt = np.logaddexp(0, zx[t, E + Cx:] + sp["dt_bias"])
+        for h in range(H):
+            g = h * G // H
+            cb = xc[E + G * N + g * N:E + G * N + (g + 1) * N] @ xc[E + g * N:E + (g + 1) * N]
+            xh = xc[h * P:(h + 1) * P]
+            assert np.allclose(y[t, h * P:(h + 1) * P], cb * dt[h] * xh + sp["D"][h] * xh, rtol=1e-12, atol=1e-12)
+
+
+def test_pure_decay_and_softplus_zero():
+    """x = 0 (conv weights and bias 0 on the x channels => silu(0) = 0) and dt_raw = -dt_bias
+    (dt = softplus(0) = ln 2): S_T = prod_t exp(A ln 2) S_0 = 2^(A T) S_0, y = C.S."""
+    cfg = small_cfg(pattern="M")
+    model = oracle.Model(cfg, seed=6)
+    sp = model.small[0]
+    E, Cx, H = cfg.d_inner, cfg.conv_dim, cfg.ssm_heads
+    sp["conv_w"][:E] = 0.0
+    sp["conv_b"][:E] = 0.0
+    T = 5
+    zx, ssm0, conv0 = mixer_inputs(cfg, model, T, 6)
+    zx[:, E + Cx:] = -sp["dt_bias"].astype(np.float64)[None, :]
+    s = ssm0.copy()
+    model.mamba_mixer(0, zx, s, conv0.copy(), 0)
+    A = -np.exp(sp["A_log"].astype(np.float64))
+    expect = ssm0 * (2.0 ** (A * T))[:, None, None]
+    assert np.allclose(s, expect, rtol=1e-13, atol=1e-300)
+    assert math.isclose(math.log1p(math.exp(0.0)), math.log(2.0))
+
+
+def test_relu2_kills_negative_preactivations():
+    """MLP with W_up rows = -|.|-ish so every pre-activation of a positive input is < 0:
+    relu(.)^2 = 0 and the layer leaves the residual unchanged."""
+    cfg = small_cfg(pattern="-")
+    model = oracle.Model(cfg, seed=7)
+    up = model.mats[(0, synth.K_UP)]
+    wneg = -np.abs(synth.bf16_to_f32(up.q)).astype(np.float32) - 0.01
+    model.mats[(0, synth.K_UP)] = oracle.bf16_mat(synth.f32_to_bf16(wneg))
+    model.layers[0].up = model.mats[(0, synth.K_UP)].c()
+    model.small[0]["norm"][:] = 1.0
+    st = model.new_state(1, cfg.kv_capacity)
+    x = synth.f32_to_bf16(np.abs(synth.normal_f32(7, 7, (1, cfg.d_model))) + 0.5)
+    r = model.step(st, x, oracle.EXACT, taps=True)
+    assert np.array_equal(r["hidden"][1], r["hidden"][0])
+
+
+def test_argmax_lowest_index_on_ties():
+    cfg = small_cfg(pattern="-", vocab_text=40, vocab_func=40)
+    model = oracle.Model(cfg, seed=9)
+    wt = np.full((40, cfg.d_model), 0.0, np.float32)
+    wt[17] = 0.05
+    wt[4] = 0.05                                 # same row twice: tied maximum at 4 and 17
+    wt[30] = -0.05
+    model.head_text = oracle.bf16_mat(synth.f32_to_bf16(wt))
+    model.head_func = oracle.bf16_mat(synth.f32_to_bf16(np.zeros((40, cfg.d_model), np.float32)))
+    model.weights.head_text = model.head_text.c()
+    model.weights.head_func = model.head_func.c()
+    st = model.new_state(1, cfg.kv_capacity)
+    x = synth.f32_to_bf16(np.abs(synth.normal_f32(9, 9, (1, cfg.d_model))) + 0.5)
+    model.final_norm[:] = 1.0
+    r = model.step(st, x, oracle.EXACT)
+    # all logits of the function head are 0: ties everywhere -> index 0
+    assert r["tok_func"][0] == 0
+    # text: rows 4 and 17 identical; the residual stays positive only if the MLP adds little,
+    # so compare with the explicit argmax of the returned logits instead of assuming a sign.
+    rr = model.step(model.new_state(1, cfg.kv_capacity), x, oracle.EXACT, taps=True)
+    lt = rr["logits"][0, 0, :40]
+    assert lt[4] == lt[17]
+    best = int(np.flatnonzero(lt == lt.max())[0])
+    assert rr["tok_text"][0] == best
+
+
+def test_scalar_ssm_hand_example():
+    """One head, P = N = 1, G = 1: the hand-worked recurrence in tests/golden/ssm_scalar.txt."""
+    g = read_golden("ssm_scalar.txt")
+    cfg = small_cfg(pattern="M", d_model=8, ssm_heads=1, ssm_head_dim=1, ssm_state=1, ssm_groups=1, norm_groups=1,
+                    conv_width=2)
+    model = oracle.Model(cfg, seed=1)
+    sp = model.small[0]
+    # conv: width 2, weights (0, 1) and bias 0 on every channel => xc = silu(current input)
+    sp["conv_w"][:] = np.array([0.0, 1.0], np.float32)
+    sp["conv_b"][:] = 0.0
+    sp["A_log"][:] = 0.0          # A = -1
+    sp["dt_bias"][:] = 0.0
+    sp["D"][:] = g["D"][0]
+    xs, bs, cs, dts = g["x_pre"], g["b_pre"], g["c_pre"], g["dt_raw"]
+    T = len(xs)
+    zx = np.zeros((T, cfg.in_proj_rows))
+    # layout [z(E=1) | x(1) B(1) C(1) | dt(1)]
+    zx[:, 1], zx[:, 2], zx[:, 3], zx[:, 4] = xs, bs, cs, dts
+    s = np.array([[[g["S0"][0]]]], np.float64)
+    y, _ = model.mamba_mixer(0, zx, s, np.zeros((1, cfg.conv_dim)), 0)
+    assert np.allclose(y[:, 0], g["y"], rtol=0, atol=5e-12)
+    assert abs(s[0, 0, 0] - g["S_final"][0]) < 5e-12
