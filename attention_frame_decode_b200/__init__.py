@@ -1,0 +1,267 @@
+"""Python binding of libvc (include/vc.h): argument marshalling only.
+
+Every computation runs in the CUDA kernels of libvc.so; PyTorch provides device memory and
+streams.  Importing this package fails loudly if libvc.so has not been built
+(``python attention_frame_decode_b200/build.py``).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvc.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libvc.so not found at {LIB_PATH}; build it with `python attention_frame_decode_b200/build.py`")
+
+_lib = C.CDLL(LIB_PATH)
+
+VC_OK, VC_ERR_INVALID_ARG, VC_ERR_UNSUPPORTED, VC_ERR_CUDA, VC_ERR_CAPACITY, VC_ERR_STATE = range(6)
+VC_DEV_CAPACITY, VC_DEV_NONFINITE, VC_DEV_TIMEOUT = 1, 2, 4
+W_BF16, W_INT8_SYM, W_INT4_ASYM, W_INT3_ASYM = 0, 1, 2, 3
+OPT_GRAPH, OPT_PDL = 1, 2
+
+
+class VcConfig(C.Structure):
+    _fields_ = [("d_model", C.c_int), ("pattern", C.c_char_p), ("ssm_heads", C.c_int), ("ssm_head_dim", C.c_int),
+                ("ssm_state", C.c_int), ("ssm_groups", C.c_int), ("conv_width", C.c_int), ("norm_groups", C.c_int),
+                ("attn_q_heads", C.c_int), ("attn_kv_heads", C.c_int), ("attn_head_dim", C.c_int),
+                ("mlp_hidden", C.c_int), ("vocab_text", C.c_int), ("vocab_func", C.c_int), ("eps", C.c_float),
+                ("wfmt", C.c_int), ("group_size", C.c_int), ("head_fmt", C.c_int), ("max_batch", C.c_int),
+                ("kv_capacity", C.c_int), ("n_slots", C.c_int)]
+
+
+class VcQmat(C.Structure):
+    _fields_ = [("data", C.c_void_p), ("fmt", C.c_int), ("group", C.c_int), ("N", C.c_int), ("K", C.c_int)]
+
+
+class VcLayerWeights(C.Structure):
+    _fields_ = [("norm", C.c_void_p), ("in_proj", VcQmat), ("out_proj", VcQmat), ("conv_w", C.c_void_p),
+                ("conv_b", C.c_void_p), ("A_log", C.c_void_p), ("D", C.c_void_p), ("dt_bias", C.c_void_p),
+                ("gnorm", C.c_void_p), ("qkv", VcQmat), ("o", VcQmat), ("up", VcQmat), ("down", VcQmat)]
+
+
+class VcWeights(C.Structure):
+    _fields_ = [("layers", C.POINTER(VcLayerWeights)), ("final_norm", C.c_void_p), ("head_text", VcQmat),
+                ("head_func", VcQmat)]
+
+
+class VcState(C.Structure):
+    _fields_ = [("ssm", C.c_void_p), ("conv", C.c_void_p), ("k", C.c_void_p), ("v", C.c_void_p),
+                ("ctx_len", C.c_void_p), ("status", C.c_void_p)]
+
+
+_p = C.c_void_p
+_i = C.c_int
+_lib.vc_weight_bytes.argtypes = [_i, _i, _i, _i]
+_lib.vc_weight_bytes.restype = C.c_size_t
+_lib.vc_quantize_weight.argtypes = [_i, _i, _i, _i, _p, _p, _p]
+_lib.vc_pack_bf16_weight.argtypes = [_i, _i, _p, _p, _p]
+_lib.vc_pack_weight.argtypes = [_i, _i, _i, _i, _p, _p, _p, _p, _p]
+_lib.vc_debug_dequant.argtypes = [C.POINTER(VcQmat), _p, _p]
+_lib.vc_workspace_bytes.argtypes = [C.POINTER(VcConfig)]
+_lib.vc_workspace_bytes.restype = C.c_size_t
+_lib.vc_backbone_create.argtypes = [C.POINTER(VcConfig), C.POINTER(VcWeights), _p, C.c_size_t, _p, C.POINTER(_p)]
+_lib.vc_set_option.argtypes = [_p, _i, _i]
+_lib.vc_step.argtypes = [_p, _p, _i, _p, C.POINTER(VcState), _p, _p, _p]
+_lib.vc_step_host.argtypes = [_p, _p, _i, _p, C.POINTER(VcState), _p, _p, _p]
+_lib.vc_prefill.argtypes = [_p, _p, _i, _i, C.POINTER(VcState), _p]
+_lib.vc_debug_set_taps.argtypes = [_p, _p, _p]
+_lib.vc_debug_mamba_step.argtypes = [C.POINTER(VcConfig), C.POINTER(VcLayerWeights), _p, _i, _p, _p, _p, _p, _p, _p,
+                                      _p, _p]
+_lib.vc_destroy.argtypes = [_p]
+_lib.vc_destroy.restype = None
+_lib.vc_status_string.argtypes = [_i]
+_lib.vc_status_string.restype = C.c_char_p
+_lib.vc_last_cuda_error.argtypes = []
+_lib.vc_last_cuda_error.restype = C.c_char_p
+for _f in ("vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant", "vc_backbone_create",
+           "vc_set_option", "vc_step", "vc_step_host", "vc_prefill", "vc_debug_set_taps", "vc_debug_mamba_step"):
+    getattr(_lib, _f).restype = _i
+
+EXPORTS = ("vc_weight_bytes", "vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant",
+           "vc_workspace_bytes", "vc_backbone_create", "vc_set_option", "vc_step", "vc_step_host", "vc_prefill",
+           "vc_debug_set_taps", "vc_debug_mamba_step", "vc_destroy", "vc_status_string", "vc_last_cuda_error")
+
+
+class VcError(RuntimeError):
+    def __init__(self, code, where):
+        msg = _lib.vc_status_string(code).decode()
+        if code == VC_ERR_CUDA:
+            msg += ": " + _lib.vc_last_cuda_error().decode()
+        super().__init__(f"{where}: {msg}")
+        self.code = code
+
+
+def _check(code, where):
+    if code != VC_OK:
+        raise VcError(code, where)
+
+
+def lib():
+    return _lib
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+# ------------------------------------------------------------------------------------------------
+# weight preparation
+# ------------------------------------------------------------------------------------------------
+
+def weight_bytes(fmt: int, group: int, N: int, K: int) -> int:
+    return int(_lib.vc_weight_bytes(fmt, group, N, K))
+
+
+def qmat(buf, fmt, group, N, K) -> VcQmat:
+    return VcQmat(buf.data_ptr(), fmt, group, N, K)
+
+
+def quantize_weight(w, fmt: int, group: int, out=None, stream=None):
+    """w: fp32 CUDA tensor [N][K] -> uint8 CUDA tensor in the device layout."""
+    import torch
+    N, K = w.shape
+    assert w.dtype == torch.float32 and w.is_cuda and w.is_contiguous()
+    if out is None:
+        out = torch.empty(weight_bytes(fmt, group, N, K), dtype=torch.uint8, device=w.device)
+    _check(_lib.vc_quantize_weight(fmt, group, N, K, _ptr(w), _ptr(out), _stream(stream)), "vc_quantize_weight")
+    return out
+
+
+def pack_bf16_weight(w, out=None, stream=None):
+    """w: bf16 CUDA tensor [N][K] -> device layout."""
+    import torch
+    N, K = w.shape
+    assert w.dtype == torch.bfloat16 and w.is_cuda and w.is_contiguous()
+    if out is None:
+        out = torch.empty(weight_bytes(W_BF16, 64, N, K), dtype=torch.uint8, device=w.device)
+    _check(_lib.vc_pack_bf16_weight(N, K, _ptr(w), _ptr(out), _stream(stream)), "vc_pack_bf16_weight")
+    return out
+
+
+def pack_weight(fmt, group, N, K, q, scales, zeros=None, out=None, stream=None):
+    """GPTQ-style packed codes (CUDA int32 tensors) -> device layout."""
+    import torch
+    if out is None:
+        out = torch.empty(weight_bytes(fmt, group, N, K), dtype=torch.uint8, device=q.device)
+    _check(_lib.vc_pack_weight(fmt, group, N, K, _ptr(q), _ptr(scales), _ptr(zeros), _ptr(out), _stream(stream)),
+           "vc_pack_weight")
+    return out
+
+
+def debug_dequant(buf, fmt, group, N, K, stream=None):
+    import torch
+    out = torch.empty((N, K), dtype=torch.float32, device=buf.device)
+    m = qmat(buf, fmt, group, N, K)
+    _check(_lib.vc_debug_dequant(C.byref(m), _ptr(out), _stream(stream)), "vc_debug_dequant")
+    return out
+
+
+# ------------------------------------------------------------------------------------------------
+# backbone
+# ------------------------------------------------------------------------------------------------
+
+def make_config(cfg, max_batch: int, kv_capacity: int, n_slots: int) -> VcConfig:
+    """cfg: any object with the vc_config field names (e.g. synth.Config)."""
+    c = VcConfig()
+    c._pattern = cfg.pattern.encode()
+    c.pattern = c._pattern
+    for f in ("d_model", "ssm_heads", "ssm_head_dim", "ssm_state", "ssm_groups", "conv_width", "norm_groups",
+              "attn_q_heads", "attn_kv_heads", "attn_head_dim", "mlp_hidden", "vocab_text", "vocab_func",
+              "wfmt", "group_size", "head_fmt"):
+        setattr(c, f, int(getattr(cfg, f)))
+    c.eps = float(cfg.eps)
+    c.max_batch, c.kv_capacity, c.n_slots = max_batch, kv_capacity, n_slots
+    return c
+
+
+def workspace_bytes(c: VcConfig) -> int:
+    return int(_lib.vc_workspace_bytes(C.byref(c)))
+
+
+def debug_mamba_step(cfg_c: VcConfig, layer: VcLayerWeights, zx, slots, ssm, conv, ctx_len, act, parts, status,
+                     stream=None):
+    B = zx.shape[0]
+    _check(_lib.vc_debug_mamba_step(C.byref(cfg_c), C.byref(layer), _ptr(zx), B, _ptr(slots), _ptr(ssm), _ptr(conv),
+                                    _ptr(ctx_len), _ptr(act), _ptr(parts), _ptr(status), _stream(stream)),
+           "vc_debug_mamba_step")
+
+
+class State:
+    """Session state tensors (see vc_state in vc.h)."""
+
+    def __init__(self, cfg, n_slots: int, kv_capacity: int, device="cuda"):
+        import torch
+        nm, na = max(cfg.pattern.count("M"), 1), max(cfg.pattern.count("*"), 1)
+        H, P, N = cfg.ssm_heads, cfg.ssm_head_dim, cfg.ssm_state
+        Cx = H * P + 2 * cfg.ssm_groups * N
+        self.ssm = torch.zeros((nm, n_slots, H, P, N), dtype=torch.float32, device=device)
+        self.conv = torch.zeros((nm, n_slots, cfg.conv_width, Cx), dtype=torch.bfloat16, device=device)
+        self.k = torch.zeros((na, n_slots, cfg.attn_kv_heads, kv_capacity, cfg.attn_head_dim), dtype=torch.bfloat16,
+                             device=device)
+        self.v = torch.zeros_like(self.k)
+        self.ctx_len = torch.zeros((n_slots,), dtype=torch.int32, device=device)
+        self.status = torch.zeros((1,), dtype=torch.int32, device=device)
+        self.c = VcState(self.ssm.data_ptr(), self.conv.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                         self.ctx_len.data_ptr(), self.status.data_ptr())
+
+
+class Backbone:
+    """Handle over vc_backbone_create / vc_step / vc_prefill / vc_destroy."""
+
+    def __init__(self, cfg, weights: VcWeights, max_batch: int, kv_capacity: int, n_slots: int, device="cuda",
+                 keepalive=None, stream=None):
+        import torch
+        self.cfg = cfg
+        self.c = make_config(cfg, max_batch, kv_capacity, n_slots)
+        nbytes = workspace_bytes(self.c)
+        if nbytes == 0:
+            raise VcError(VC_ERR_INVALID_ARG, "vc_workspace_bytes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.weights = weights
+        self.keepalive = keepalive
+        h = C.c_void_p()
+        _check(_lib.vc_backbone_create(C.byref(self.c), C.byref(weights), _ptr(self.workspace), nbytes,
+                                       _stream(stream), C.byref(h)), "vc_backbone_create")
+        self.h = h
+        self.max_batch, self.kv_capacity, self.n_slots = max_batch, kv_capacity, n_slots
+
+    def set_option(self, option: int, value: int):
+        _check(_lib.vc_set_option(self.h, option, value), "vc_set_option")
+
+    def set_taps(self, hidden=None, logits=None):
+        self._taps = (hidden, logits)
+        _check(_lib.vc_debug_set_taps(self.h, _ptr(hidden), _ptr(logits)), "vc_debug_set_taps")
+
+    def step(self, x, state: State, tok_text, tok_func, slots=None, stream=None):
+        B = x.shape[0]
+        _check(_lib.vc_step(self.h, _ptr(x), B, _ptr(slots), C.byref(state.c), _ptr(tok_text), _ptr(tok_func),
+                            _stream(stream)), "vc_step")
+
+    def step_host(self, x_host, state: State, tok_text_host, tok_func_host, slots=None, stream=None):
+        B = x_host.shape[0]
+        _check(_lib.vc_step_host(self.h, _ptr(x_host), B, _ptr(slots), C.byref(state.c), _ptr(tok_text_host),
+                                 _ptr(tok_func_host), _stream(stream)), "vc_step_host")
+
+    def prefill(self, x, slot: int, state: State, stream=None):
+        T = x.shape[0]
+        _check(_lib.vc_prefill(self.h, _ptr(x), T, slot, C.byref(state.c), _stream(stream)), "vc_prefill")
+
+    def close(self):
+        if getattr(self, "h", None):
+            _lib.vc_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,279 @@
+"""GPU parity of the decode path against the CPU oracle (same seeded inputs).
+
+Tolerances (stated once, used everywhere):
+  * quantized-weight unpacking: bit-exact (fp32 s*(q-z) on both sides);
+  * greedy tokens: identical wherever the oracle's top-2 logit margin exceeds 1e-3;
+  * bf16-path hidden states and logits: max |gpu - oracle| <= 2e-2 * RMS(oracle);
+  * fp32 SSM state of an isolated mixer step on identical bf16 inputs:
+    max |gpu - oracle| <= 1e-4 * RMS(oracle).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+HID_TOL = 2e-2
+SSM_TOL = 1e-4
+MARGIN = 1e-3
+
+pytestmark = pytest.mark.gpu
+
+
+def rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.max(np.abs(a - b)) / max(np.sqrt(np.mean(b * b)), 1e-30))
+
+
+def tokens_agree(gpu_tok, logits, tok_oracle):
+    """compare only where the oracle's top-2 margin > MARGIN; returns (#compared, #mismatch)"""
+    top2 = np.sort(logits)[-2:]
+    if top2[1] - top2[0] <= MARGIN:
+        return 0, 0
+    return 1, int(gpu_tok != tok_oracle)
+
+
+# ------------------------------------------------------------------------------------------------
+# weight unpacking: bit-exact
+# ------------------------------------------------------------------------------------------------
+
+FMTS = [(oracle.W8, 64), (oracle.W8, 128), (oracle.W4, 64), (oracle.W4, 128), (oracle.W3, 64), (oracle.W3, 128)]
+
+
+@pytest.mark.parametrize("fmt,group", FMTS)
+@pytest.mark.parametrize("N,K", [(200, 448), (64, 15680), (37, 192)])
+def test_quantize_matches_oracle_bit_exact(cuda, fmt, group, N, K):
+    import torch
+    import attention_frame_decode_b200 as vc
+    w = synth.normal_f32(21, N * 7 + K, (N, K), 0.0, 0.02)
+    w[0, :group] = 0.0                                    # an all-zero group (scale 1 rule)
+    w[1, :] = 0.0125                                       # constant row
+    buf = vc.quantize_weight(torch.from_numpy(w).to(cuda), fmt, group)
+    deq = vc.debug_dequant(buf, fmt, group, N, K).cpu().numpy()
+    ref = oracle.quantize(fmt, group, w).dequant()
+    assert np.array_equal(deq.astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("fmt,group", FMTS)
+def test_pack_canonical_matches_oracle_bit_exact(cuda, fmt, group):
+    """GPTQ-style canonical codes (random, from the generator) -> device layout -> dequant."""
+    import torch
+    import attention_frame_decode_b200 as vc
+    from tests.test_oracle import np_pack
+    N, K = 100, 320
+    bits = oracle.BITS[fmt]
+    ng = (K + group - 1) // group
+    if fmt == oracle.W8:
+        codes = synth.uniform_i32(5, 1, (N, K), -127, 127)
+        zw = None
+    else:
+        codes = synth.uniform_i32(5, 1, (N, K), 0, (1 << bits) - 1)
+        zw = np_pack(synth.uniform_i32(5, 2, (N, ng), 0, (1 << bits) - 1), bits)
+    q = np_pack(codes, bits)
+    sc = synth.uniform_f32(5, 3, (N, ng), 0.001, 0.05).astype(np.float16).view(np.uint16)
+    m = oracle.Mat(fmt, group, N, K, q, sc, zw)
+    tq = torch.from_numpy(q.view(np.int32)).to(cuda)
+    ts = torch.from_numpy(sc.view(np.int16)).to(cuda)
+    tz = None if zw is None else torch.from_numpy(zw.view(np.int32)).to(cuda)
+    buf = vc.pack_weight(fmt, group, N, K, tq, ts, tz)
+    deq = vc.debug_dequant(buf, fmt, group, N, K).cpu().numpy()
+    assert np.array_equal(deq.astype(np.float64), m.dequant())
+
+
+# ------------------------------------------------------------------------------------------------
+# end to end: the tiny hybrid stack, 64 frames from zero state
+# ------------------------------------------------------------------------------------------------
+
+class Run:
+    """a GPU backbone and the oracle on the same synthetic model"""
+
+    def __init__(self, cfg, seed, B, cap, ctx_lens=None, taps=True):
+        import torch
+        from attention_frame_decode_b200.synthetic import build_model, fill_state
+        self.cfg, self.seed, self.B, self.cap = cfg, seed, B, cap
+        self.dm = build_model(cfg, seed)
+        self.bb = self.dm.backbone(B, cap, B)
+        self.st = self.dm.new_state(B, cap)
+        self.om = oracle.Model(cfg, seed)
+        self.ost = self.om.new_state(B, cap)
+        if ctx_lens is not None:
+            fill_state(self.st, cfg, seed, ctx_lens, cap)
+            self.ost.fill_random(seed, ctx_lens)
+        V = max(cfg.vocab_text, cfg.vocab_func)
+        self.hid = torch.zeros((cfg.n_layers + 1, B, cfg.d_model), dtype=torch.float32, device="cuda") if taps else None
+        self.lg = torch.zeros((2, B, V), dtype=torch.float32, device="cuda") if taps else None
+        if taps:
+            self.bb.set_taps(self.hid, self.lg)
+        self.tt = torch.zeros((B,), dtype=torch.int32, device="cuda")
+        self.tf = torch.zeros((B,), dtype=torch.int32, device="cuda")
+
+    def step(self, t, slots=None):
+        import torch
+        x = synth.frame_inputs(self.cfg, self.seed, t, self.B)
+        xd = torch.from_numpy(x).cuda().view(torch.bfloat16)
+        sl = None if slots is None else torch.from_numpy(np.asarray(slots, np.int32)).cuda()
+        self.bb.step(xd, self.st, self.tt, self.tf, slots=sl)
+        torch.cuda.synchronize()
+        ro = self.om.step(self.ost, x, oracle.MIRROR, slots=slots, taps=True)
+        return ro
+
+
+def check_step(run, ro, hid_tol=HID_TOL):
+    cfg = run.cfg
+    hid = run.hid.cpu().numpy()
+    lg = run.lg.cpu().numpy()
+    errs = [rel(hid[l], ro["hidden"][l]) for l in range(cfg.n_layers + 1)]
+    assert max(errs) < hid_tol, errs
+    cmp = mis = 0
+    for b in range(run.B):
+        for hsel, (tg, to, V) in enumerate(((run.tt, ro["tok_text"], cfg.vocab_text),
+                                            (run.tf, ro["tok_func"], cfg.vocab_func))):
+            lo = ro["logits"][hsel, b, :V]
+            assert rel(lg[hsel, b, :V], lo) < hid_tol
+            c, m = tokens_agree(int(tg.cpu().numpy()[b]), lo, int(to[b]))
+            cmp += c
+            mis += m
+    assert mis == 0
+    return max(errs), cmp
+
+
+def test_tiny_stack_64_frames(cuda):
+    cfg = synth.tiny_config()
+    run = Run(cfg, 0, 1, cfg.kv_capacity)
+    worst, compared = 0.0, 0
+    for t in range(64):
+        ro = run.step(t)
+        e, c = check_step(run, ro)
+        worst, compared = max(worst, e), compared + c
+    assert compared >= 100
+    assert int(run.st.ctx_len.cpu()[0]) == 64
+    assert int(run.st.status.cpu()[0]) == 0
+    # state after 64 frames (end to end: bf16 flips upstream make 1e-4 a kernel-level bound only)
+    ssm = run.st.ssm.cpu().numpy()[0, 0]
+    assert rel(ssm, run.ost.ssm[0, 0]) < 1e-2
+    kv = run.st.k.float().cpu().numpy()[0, 0, :, :64]
+    assert rel(kv, run.ost.k[0, 0, :, :64]) < HID_TOL
+
+
+@pytest.mark.parametrize("graph", [0, 1])
+def test_tiny_direct_launch_equals_graph(cuda, graph):
+    import attention_frame_decode_b200 as vc
+    cfg = synth.tiny_config()
+    run = Run(cfg, 1, 1, cfg.kv_capacity)
+    run.bb.set_option(vc.OPT_GRAPH, graph)
+    run.bb.set_taps(run.hid, run.lg)
+    for t in range(6):
+        ro = run.step(t)
+        check_step(run, ro)
+
+
+# ------------------------------------------------------------------------------------------------
+# single layers at the Nano-9B-v2 widths
+# ------------------------------------------------------------------------------------------------
+
+def nano_layer_cfg(pattern, wfmt=synth.FMT_BF16, group=64, **kw):
+    return synth.nano_config(name="layer", pattern=pattern, wfmt=wfmt, group_size=group, vocab_text=4096,
+                             vocab_func=2048, **kw)
+
+
+@pytest.mark.parametrize("pattern", ["-", "M", "*"])
+@pytest.mark.parametrize("wfmt,group", [(synth.FMT_BF16, 64), (synth.FMT_W4, 64), (synth.FMT_W8, 128),
+                                        (synth.FMT_W3, 64)])
+def test_nano_layer(cuda, pattern, wfmt, group):
+    cfg = nano_layer_cfg(pattern, wfmt, group)
+    ctx = np.array([2000], np.int32)
+    run = Run(cfg, 2, 1, 2048, ctx_lens=ctx)
+    for t in range(2):
+        ro = run.step(t)
+        check_step(run, ro)
+    if pattern == "M":
+        assert rel(run.st.ssm.cpu().numpy()[0, 0], run.ost.ssm[0, 0]) < 1e-2
+    assert int(run.st.ctx_len.cpu()[0]) == 2002
+
+
+@pytest.mark.parametrize("B", [3, 16])
+def test_nano_batch_ragged_contexts(cuda, B):
+    cfg = nano_layer_cfg("M*-", synth.FMT_W8, 128)
+    ctx = synth.uniform_i32(7, 0, (B,), 0, 300)
+    ctx[0] = 0
+    ctx[-1] = 63
+    run = Run(cfg, 4, B, 512, ctx_lens=ctx)
+    for t in range(2):
+        ro = run.step(t)
+        check_step(run, ro)
+    assert np.array_equal(run.st.ctx_len.cpu().numpy()[:B], ctx + 2)
+
+
+def test_slots_map_batch_rows(cuda):
+    import torch
+    cfg = nano_layer_cfg("*-", synth.FMT_W4, 64)
+    B = 2
+    ctx = np.array([70, 5], np.int32)
+    run = Run(cfg, 6, B, 256, ctx_lens=ctx)
+    ro = run.step(0, slots=[1, 0])
+    check_step(run, ro)
+    assert np.array_equal(run.st.ctx_len.cpu().numpy(), ctx + 1)
+
+
+def test_full_cache_sets_status_and_skips(cuda):
+    cfg = nano_layer_cfg("M*", synth.FMT_W4, 64)
+    ctx = np.array([64, 10], np.int32)
+    run = Run(cfg, 8, 2, 64, ctx_lens=ctx)
+    import torch
+    ssm_before = run.st.ssm[0, 0].clone()
+    run.step(0)
+    assert int(run.st.status.cpu()[0]) & 1
+    tt = run.tt.cpu().numpy()
+    assert tt[0] == -1 and tt[1] >= 0
+    assert torch.equal(run.st.ssm[0, 0], ssm_before)
+    assert np.array_equal(run.st.ctx_len.cpu().numpy(), [64, 11])
+
+
+# ------------------------------------------------------------------------------------------------
+# kernel level: the Mamba-2 step on identical bf16 inputs (fp32 state within 1e-4 of RMS)
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [1, 64])
+def test_mamba_step_kernel_state(cuda, T):
+    import torch
+    import attention_frame_decode_b200 as vc
+    cfg = nano_layer_cfg("M")
+    dm_small = synth.small_params(cfg, 3, 0)
+    from attention_frame_decode_b200.model import DeviceModel
+    dm = DeviceModel(cfg)
+    for k, v in dm_small.items():
+        dm.set_small(0, k, v)
+    c = vc.make_config(cfg, 1, 64, 1)
+    R = cfg.in_proj_rows
+    zx_all = synth.normal_bf16(3, 500, (T, R), 0.0, 1.0)
+    ssm0 = synth.ssm_state(cfg, 3, 0, 1)
+    hist0 = synth.conv_history(cfg, 3, 0, 1)
+    ssm = torch.from_numpy(ssm0).cuda().contiguous()
+    W = cfg.conv_width
+    t0 = 10
+    ring = np.zeros((1, W, cfg.conv_dim), np.uint16)
+    for i in range(W - 1):
+        ring[0, (t0 - (W - 1) + i) % W] = hist0[0, i]
+    conv = torch.from_numpy(ring).cuda().view(torch.bfloat16).contiguous()
+    ctx = torch.tensor([t0], dtype=torch.int32, device="cuda")
+    act = torch.zeros((1, cfg.d_inner), dtype=torch.bfloat16, device="cuda")
+    parts = torch.zeros((1, 2 * cfg.ssm_heads), dtype=torch.float32, device="cuda")
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    om = oracle.Model(cfg.replace(vocab_text=16, vocab_func=16), 3)
+    S = ssm0[0].astype(np.float64).copy()
+    hist = synth.bf16_to_f32(hist0[0]).astype(np.float64).copy()
+    for t in range(T):
+        zx = torch.from_numpy(zx_all[t:t + 1]).cuda().view(torch.bfloat16)
+        vc.debug_mamba_step(c, dm.layers[0], zx, None, ssm, conv, ctx, act, parts, status)
+        ctx += 1
+        y, v = om.mamba_mixer(0, synth.bf16_to_f32(zx_all[t:t + 1]).astype(np.float64), S, hist, 0)
+    torch.cuda.synchronize()
+    assert rel(ssm.cpu().numpy()[0], S) < SSM_TOL
+    gam = dm_small["gnorm"].astype(np.float64)
+    # act is a bf16 storage point: compare with the oracle's value rounded the same way
+    ref_act = synth.bf16_to_f32(synth.f32_to_bf16((v[0] * gam).astype(np.float32)))
+    assert rel(act.float().cpu().numpy()[0], ref_act) < HID_TOL
+    ss = (v[0].reshape(cfg.ssm_heads * 2, -1) ** 2).sum(axis=1)
+    assert rel(parts.cpu().numpy()[0], ss) < 1e-4
+    assert int(status.cpu()[0]) == 0
