@@ -70,6 +70,9 @@ _lib.vc_prefill.argtypes = [_p, _p, _i, _i, C.POINTER(VcState), _p]
 _lib.vc_debug_set_taps.argtypes = [_p, _p, _p]
 _lib.vc_debug_mamba_step.argtypes = [C.POINTER(VcConfig), C.POINTER(VcLayerWeights), _p, _i, _p, _p, _p, _p, _p, _p,
                                       _p, _p]
+_lib.vc_gemv_scratch_bytes.argtypes = []
+_lib.vc_gemv_scratch_bytes.restype = C.c_size_t
+_lib.vc_debug_gemv.argtypes = [C.POINTER(VcQmat), _p, _i, _i, _p, _p, _p]
 _lib.vc_destroy.argtypes = [_p]
 _lib.vc_destroy.restype = None
 _lib.vc_status_string.argtypes = [_i]
@@ -77,12 +80,14 @@ _lib.vc_status_string.restype = C.c_char_p
 _lib.vc_last_cuda_error.argtypes = []
 _lib.vc_last_cuda_error.restype = C.c_char_p
 for _f in ("vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant", "vc_backbone_create",
-           "vc_set_option", "vc_step", "vc_step_host", "vc_prefill", "vc_debug_set_taps", "vc_debug_mamba_step"):
+           "vc_set_option", "vc_step", "vc_step_host", "vc_prefill", "vc_debug_set_taps", "vc_debug_mamba_step",
+           "vc_debug_gemv"):
     getattr(_lib, _f).restype = _i
 
 EXPORTS = ("vc_weight_bytes", "vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant",
            "vc_workspace_bytes", "vc_backbone_create", "vc_set_option", "vc_step", "vc_step_host", "vc_prefill",
-           "vc_debug_set_taps", "vc_debug_mamba_step", "vc_destroy", "vc_status_string", "vc_last_cuda_error")
+           "vc_debug_set_taps", "vc_debug_mamba_step", "vc_gemv_scratch_bytes", "vc_debug_gemv", "vc_destroy",
+           "vc_status_string", "vc_last_cuda_error")
 
 
 class VcError(RuntimeError):
@@ -185,6 +190,23 @@ def make_config(cfg, max_batch: int, kv_capacity: int, n_slots: int) -> VcConfig
 
 def workspace_bytes(c: VcConfig) -> int:
     return int(_lib.vc_workspace_bytes(C.byref(c)))
+
+
+def gemv_scratch(device="cuda"):
+    import torch
+    return torch.zeros(int(_lib.vc_gemv_scratch_bytes()), dtype=torch.uint8, device=device)
+
+
+def debug_gemv(wbuf, fmt, group, N, K, act, scratch, out=None, stream=None):
+    """y[B][N] = W act^T with the step's GEMV kernel; act: 16-bit CUDA tensor [B][act_ld]"""
+    import torch
+    B, act_ld = act.shape
+    if out is None:
+        out = torch.empty((B, N), dtype=torch.float32, device=act.device)
+    m = qmat(wbuf, fmt, group, N, K)
+    _check(_lib.vc_debug_gemv(C.byref(m), _ptr(act), act_ld, B, _ptr(out), _ptr(scratch), _stream(stream)),
+           "vc_debug_gemv")
+    return out
 
 
 def debug_mamba_step(cfg_c: VcConfig, layer: VcLayerWeights, zx, slots, ssm, conv, ctx_len, act, parts, status,

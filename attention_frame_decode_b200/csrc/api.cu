@@ -579,6 +579,38 @@ extern "C" vc_status vc_debug_mamba_step(const vc_config* cfg, const vc_layer_we
     return VC_OK;
 }
 
+extern "C" size_t vc_gemv_scratch_bytes(void) {
+    return align_up(gemv_partials_bytes(256), 256) + gemv_counter_ints() * 4;
+}
+
+extern "C" vc_status vc_debug_gemv(const vc_qmat* w, const void* act, int act_ld, int B, float* out, void* scratch,
+                                   vc_stream_t stream) {
+    if (!w || !w->data || !act || !out || !scratch || !aligned16(act) || !aligned16(scratch)) return VC_ERR_INVALID_ARG;
+    if (!fmt_ok(w->fmt, w->group) || w->N <= 0 || w->K <= 0 || B < 1 || B > 16) return VC_ERR_INVALID_ARG;
+    if (act_ld % 128 || act_ld < round_up(w->K, 128)) return VC_ERR_INVALID_ARG;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    GemvArgs a{};
+    a.nmat = 1;
+    a.mat[0] = gm(*w);
+    a.act = (const uint16_t*)act;
+    a.act_ld = act_ld;
+    a.B = B;
+    a.tap = out;
+    a.tap_ld = w->N;
+    a.partials = (float*)scratch;
+    a.counters = (int*)((uint8_t*)scratch + align_up(gemv_partials_bytes(256), 256));
+    GemvLaunch L{};
+    L.fmt = w->fmt;
+    L.group = w->fmt == VC_W_BF16 ? 64 : w->group;
+    L.epi = EPI_STORE;
+    L.num_sms = sms > 256 ? 256 : sms;
+    L.pdl = 0;
+    CK(launch_gemv(L, a, (cudaStream_t)stream));
+    return VC_OK;
+}
+
 extern "C" void vc_destroy(vc_backbone* h) {
     if (!h) return;
     clear_graphs(h);

@@ -17,7 +17,7 @@
 // device status bits VC_DEV_* (OR-ed into the caller's status word) come from vc.h
 #include "../../include/vc.h"
 
-static constexpr long long kWaitLimit = 1ll << 24;   // try_wait polls before giving up
+static constexpr long long kWaitLimit = 1ll << 22;   // try_wait polls before giving up
 
 // ------------------------------------------------------------------------------------------
 // programmatic dependent launch

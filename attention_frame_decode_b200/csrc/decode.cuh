@@ -54,7 +54,7 @@ struct AttnArgs {
     int* status;
 };
 
-static constexpr int kAttnSplit = 64;   // keys per split
+static constexpr int kAttnSplit = 128;  // keys per split
 
 cudaError_t launch_input(const InputArgs& a, cudaStream_t s);
 cudaError_t launch_mamba_step(const MambaStepArgs& a, int pdl, cudaStream_t s);

@@ -22,9 +22,12 @@
 
 namespace vc {
 
-static constexpr int kWarps = 8;
-static constexpr int kThreads = kWarps * 32;
+static constexpr int kWarps = 16;   // upper bound of warps per CTA
+// warps per CTA: 16 for up to 8 batch rows (<= 128 registers each), 8 for 9..16 rows
+__host__ __device__ constexpr int warps_for(int NT) { return NT == 1 ? 16 : 8; }
 static constexpr int kMaxB = 16;
+static constexpr int kMaxSlots = 8;          // ring slots per warp (upper bound)
+static constexpr int kRingBudget = 210 * 1024; // dynamic shared memory for the rings of one CTA
 
 // ------------------------------------------------------------------------------------------
 // partition helpers (worker w of W owns flat blocks [w*T/W, (w+1)*T/W))
@@ -128,16 +131,19 @@ __device__ __forceinline__ void mma_step(float (&d)[4], const uint32_t (&a)[4], 
 // ------------------------------------------------------------------------------------------
 struct RingGeom {
     int slots;        // ring slots per warp
-    int slot_bytes;   // weights (bps blocks) + activation rows
+    int slot_bytes;   // weights (bps blocks) [+ activation rows when act_smem == 0]
     int act_row;      // bytes per staged activation row (KS*2 + 16)
+    int act_smem;     // 1: the whole activation [B][act_ld] is copied to shared memory once per CTA
+    int act_stride;   // bytes per activation row in shared memory (act_ld*2 + 16)
 };
 
 template <int FMT, int GRP, int NT, int EPI>
-__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, const RingGeom rg) {
+__global__ void __launch_bounds__(warps_for(NT) * 32, 1) gemv_kernel(const GemvArgs args, const RingGeom rg) {
+    constexpr int WARPS = warps_for(NT);
     constexpr LayoutInfo L = layout_info(FMT, GRP);
     constexpr int R = L.R, SUB = L.SUB, KS = L.KS;
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t bars[kWarps][4];
+    __shared__ uint64_t bars[WARPS][kMaxSlots];
     __shared__ float insc_tab[kMaxB * 16];
 
     pdl_trigger();
@@ -147,8 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, 
     const int B = args.B;
 
     // ---- worker range -------------------------------------------------------------------
-    const long long Wall = (long long)gridDim.x * kWarps;
-    const long long wid = (long long)blockIdx.x * kWarps + warp;
+    const long long Wall = (long long)gridDim.x * WARPS;
+    const long long wid = (long long)blockIdx.x * WARPS + warp;
     int m = 0;
     long long Wm = Wall, wl = wid, wbase = 0;
     if (args.nmat == 2) {
@@ -162,66 +168,77 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, 
     // worker between the first and last contributor of a unit is a contributor
     if (Wm > T) Wm = T;
     const bool idle = wl >= Wm;
-    const long long f0 = idle ? 0 : part_begin(wl, T, Wm), f1 = idle ? 0 : part_begin(wl + 1, T, Wm);
+    // block indices fit in 32 bits (at most a few 10^5 blocks per matrix); positions advance
+    // incrementally so the hot loop has no integer division
+    const int f0 = idle ? 0 : (int)part_begin(wl, T, Wm), f1 = idle ? 0 : (int)part_begin(wl + 1, T, Wm);
     const int bps = L.bps;
-    const long long nstages = (f1 - f0 + bps - 1) / bps;
+    const int nstages = (f1 - f0 + bps - 1) / bps;
+    const int KT = M.KT;
 
     uint8_t* ring = smem + (size_t)warp * rg.slots * rg.slot_bytes;
     uint64_t* bar = bars[warp];
     const int act_rows = B;
 
-    auto issue_weights = [&](long long i) {
-        const int slot = (int)(i % rg.slots);
-        const long long fb = f0 + i * bps;
-        const int nb = (int)(int)llmin((long long)bps, f1 - fb);
+    // stage i covers blocks [f0 + i*bps, min(f0 + (i+1)*bps, f1)) and lives in ring slot i mod slots
+    auto issue_weights = [&](int i, int slot) {
+        const int fb = f0 + i * bps;
+        const int nb = min(bps, f1 - fb);
         const uint32_t wbytes = nb * L.block_bytes;
-        const uint32_t abytes = nb * act_rows * KS * 2;
+        const uint32_t abytes = rg.act_smem ? 0u : (uint32_t)(nb * act_rows * KS * 2);
         mbar_arrive_expect_tx(&bar[slot], wbytes + abytes);
-        bulk_g2s(ring + (size_t)slot * rg.slot_bytes, M.w + fb * L.block_bytes, wbytes, &bar[slot]);
+        bulk_g2s(ring + (size_t)slot * rg.slot_bytes, M.w + (size_t)fb * L.block_bytes, wbytes, &bar[slot]);
     };
-    auto issue_act = [&](long long i) {
-        const int slot = (int)(i % rg.slots);
-        const long long fb = f0 + i * bps;
-        const int nb = (int)(int)llmin((long long)bps, f1 - fb);
+    int act_kt = f0 % KT;   // k-step of the next block whose activation slice is issued
+    auto issue_act = [&](int i, int slot) {
+        const int nb = min(bps, f1 - (f0 + i * bps));
         uint8_t* abase = ring + (size_t)slot * rg.slot_bytes + bps * L.block_bytes;
         for (int j = 0; j < nb; ++j) {
-            const int kt = (int)((fb + j) % M.KT);
             for (int b = 0; b < act_rows; ++b)
-                bulk_g2s(abase + (j * act_rows + b) * rg.act_row, args.act + (size_t)b * args.act_ld + (size_t)kt * KS,
-                         KS * 2, &bar[slot]);
+                bulk_g2s(abase + (j * act_rows + b) * rg.act_row,
+                         args.act + (size_t)b * args.act_ld + (size_t)act_kt * KS, KS * 2, &bar[slot]);
+            if (++act_kt == KT) act_kt = 0;
         }
     };
 
     if (lane == 0) {
         for (int s = 0; s < rg.slots; ++s) mbar_init(&bar[s], 1);
         fence_mbar_init();
-        for (long long i = 0; i < nstages && i < rg.slots; ++i) issue_weights(i);
+        for (int i = 0; i < nstages && i < rg.slots; ++i) issue_weights(i, i);
     }
     __syncwarp();
 
     pdl_wait();
 
-    // ---- input-scale table (per CTA) ------------------------------------------------------
+    // ---- input-scale table (per CTA): one warp per (row b, norm group q) --------------------
     const int ng = args.insc.parts ? args.insc.n_groups : 1;
-    for (int idx = threadIdx.x; idx < B * ng; idx += kThreads) {
+    for (int idx = warp; idx < B * ng; idx += WARPS) {
         float v = 1.0f;
         if (args.insc.parts) {
             const int b = idx / ng, q = idx % ng;
             const float* p = args.insc.parts + ((size_t)b * ng + q) * args.insc.per_group;
             float s = 0.0f;
-            for (int i = 0; i < args.insc.per_group; ++i) s += p[i];
+            for (int i = lane; i < args.insc.per_group; i += 32) s += p[i];
+            s = warp_sum(s);
             v = rsqrtf(s * args.insc.inv_width + args.insc.eps);
         }
-        insc_tab[idx] = v;
+        if (lane == 0) insc_tab[idx] = v;
+    }
+    uint8_t* act_s = smem + (size_t)WARPS * rg.slots * rg.slot_bytes;
+    if (rg.act_smem) {
+        const int row16 = args.act_ld / 8;   // 16-byte chunks per row
+        for (int idx = threadIdx.x; idx < B * row16; idx += WARPS * 32) {
+            const int b = idx / row16, c = idx % row16;
+            *reinterpret_cast<uint4*>(act_s + (size_t)b * rg.act_stride + c * 16) =
+                *reinterpret_cast<const uint4*>(args.act + (size_t)b * args.act_ld + (size_t)c * 8);
+        }
     }
     __syncthreads();
 
-    if (lane == 0)
-        for (long long i = 0; i < nstages && i < rg.slots; ++i) issue_act(i);
+    if (lane == 0 && !rg.act_smem)
+        for (int i = 0; i < nstages && i < rg.slots; ++i) issue_act(i, i);
 
     // ---- accumulation state ---------------------------------------------------------------
     float acc[R][NT][4];
-    long long cur_u = -1;
     unsigned long long best[NT][2];
 #pragma unroll
     for (int j = 0; j < NT; ++j) best[j][0] = best[j][1] = 0ull;
@@ -236,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, 
     };
 
     // epilogue of a finished unit (values in v)
-    auto epilogue = [&](long long u, float (&v)[R][NT][4]) {
+    auto epilogue = [&](int u, float (&v)[R][NT][4]) {
         const int row0 = (int)(u * 16 * R);
         if constexpr (EPI == EPI_ARGMAX) {
 #pragma unroll
@@ -320,7 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, 
                                 cache[(((size_t)slot * args.Hk + jj) * args.cap + pos) * args.Dh + d] = act_bits<false>(x);
                             }
                         } else {
-                            args.out[(size_t)b * args.out_ld + row] = args.out_f16 ? act_bits<true>(x) : act_bits<false>(x);
+                            if (args.out)
+                                args.out[(size_t)b * args.out_ld + row] = args.out_f16 ? act_bits<true>(x) : act_bits<false>(x);
                             if (args.tap) args.tap[(size_t)b * args.tap_ld + row] = x;
                         }
                     }
@@ -328,8 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, 
     };
 
     // a unit leaves this worker: finish it here or hand a partial to the last contributor
-    auto flush = [&](long long u) {
-        const long long lo = part_owner(u * M.KT, T, Wm), hi = part_owner((u + 1) * M.KT - 1, T, Wm);
+    auto flush = [&](int u) {
+        const long long lo = part_owner((long long)u * M.KT, T, Wm), hi = part_owner((long long)(u + 1) * M.KT - 1, T, Wm);
         if (lo == hi) {
             epilogue(u, acc);
             return;
@@ -357,16 +375,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, 
             for (int j = 0; j < NT; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) tot[r][j][e] = 0.0f;
-        for (long long w2 = lo; w2 <= hi; ++w2) {
-            const long long fu = part_begin(w2, T, Wm) / M.KT;
-            const float* p = args.partials + ((size_t)(wbase + w2) * 2 + (u == fu ? 0 : 1)) * (R * NT * 128);
+        for (long long w0 = lo; w0 <= hi; w0 += 4) {
+            float4 x[4][R * NT];
 #pragma unroll
-            for (int r = 0; r < R; ++r)
+            for (int q = 0; q < 4; ++q) {
+                const long long w2 = w0 + q;
+                if (w2 > hi) break;
+                const long long fu = part_begin(w2, T, Wm) / M.KT;
+                const float* p = args.partials + ((size_t)(wbase + w2) * 2 + (u == fu ? 0 : 1)) * (R * NT * 128);
 #pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    float4 x = __ldcg(reinterpret_cast<const float4*>(p + ((r * NT + j) * 32 + lane) * 4));
-                    tot[r][j][0] += x.x; tot[r][j][1] += x.y; tot[r][j][2] += x.z; tot[r][j][3] += x.w;
-                }
+                for (int rj = 0; rj < R * NT; ++rj) x[q][rj] = __ldcg(reinterpret_cast<const float4*>(p + (rj * 32 + lane) * 4));
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (w0 + q > hi) break;
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int j = 0; j < NT; ++j) {
+                        const float4 v = x[q][r * NT + j];
+                        tot[r][j][0] += v.x; tot[r][j][1] += v.y; tot[r][j][2] += v.z; tot[r][j][3] += v.w;
+                    }
+            }
         }
         if (lane == 0) *cnt = 0;
         epilogue(u, tot);
@@ -374,32 +404,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, 
 
     zero_acc();
     bool alive = true;
-    for (long long i = 0; i < nstages && alive; ++i) {
-        const int slot = (int)(i % rg.slots);
-        if (!mbar_wait(&bar[slot], (uint32_t)((i / rg.slots) & 1), args.status)) { alive = false; break; }
+    int cur_u = f0 / KT, kt = f0 % KT;   // unit and k-step of the next block to consume
+    bool pending = false;                 // acc holds contributions of cur_u not yet flushed
+    int slot = 0;
+    uint32_t phase = 0;
+    float sc[NT][2];
+    int sc_next = kt;   // first k-step at which sc must be (re)loaded
+    for (int i = 0; i < nstages; ++i) {
+        if (!mbar_wait(&bar[slot], phase, args.status)) { alive = false; break; }
         const uint8_t* base = ring + (size_t)slot * rg.slot_bytes;
-        const long long fb = f0 + i * bps;
-        const int nb = (int)(int)llmin((long long)bps, f1 - fb);
+        const int nb = min(bps, f1 - (f0 + i * bps));
         for (int jb = 0; jb < nb; ++jb) {
-            const long long f = fb + jb;
-            const long long u = f / M.KT;
-            const int kt = (int)(f % M.KT);
-            if (u != cur_u) {
-                if (cur_u >= 0) { flush(cur_u); zero_acc(); }
-                cur_u = u;
-            }
             const uint8_t* blk = base + jb * L.block_bytes;
             const uint8_t* arow = base + bps * L.block_bytes + (size_t)jb * act_rows * rg.act_row;
-            // input scales of this k-step for the lane's two batch columns per n-tile
-            const int qg = ng > 1 ? (kt * KS) / args.insc.group_cols : 0;
-            float sc[NT][2];
+            // input scales of this k-step (norm group qg) for the lane's batch columns
+            if (kt == sc_next) {
+                const int qg = ng > 1 ? (kt * KS) / args.insc.group_cols : 0;
+                sc_next = ng > 1 ? min(KT, ((qg + 1) * args.insc.group_cols) / KS) : KT;
 #pragma unroll
-            for (int j = 0; j < NT; ++j)
+                for (int j = 0; j < NT; ++j)
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int b = 8 * j + 2 * t + e;
-                    sc[j][e] = b < B ? insc_tab[b * ng + qg] : 0.0f;
-                }
+                    for (int e = 0; e < 2; ++e) {
+                        const int b = 8 * j + 2 * t + e;
+                        sc[j][e] = b < B ? insc_tab[b * ng + qg] : 0.0f;
+                    }
+            }
             // activation B-fragments
             uint32_t bf[SUB][NT][4][2];
 #pragma unroll
@@ -409,7 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, 
                     const int b = 8 * j + g;
                     uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
                     if (b < B) {
-                        const uint8_t* p = arow + b * rg.act_row + (64 * st + 16 * t) * 2;
+                        const uint8_t* p = rg.act_smem
+                            ? act_s + (size_t)b * rg.act_stride + ((size_t)kt * KS + 64 * st + 16 * t) * 2
+                            : arow + b * rg.act_row + (64 * st + 16 * t) * 2;
                         v0 = *reinterpret_cast<const uint4*>(p);
                         v1 = *reinterpret_cast<const uint4*>(p + 16);
                     }
@@ -460,15 +491,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs args, 
                     acc[r][j][3] = fmaf(s_hi * sc[j][1], c[j][3], acc[r][j][3]);
                 }
             }
+            pending = true;
+            if (++kt == KT) {   // the unit's last k-step: finish it (or hand over the partial)
+                flush(cur_u);
+                zero_acc();
+                pending = false;
+                kt = 0;
+                ++cur_u;
+                if (ng > 1) sc_next = 0;
+            }
         }
         __syncwarp();
         if (lane == 0 && i + rg.slots < nstages) {
             fence_proxy_async();
-            issue_weights(i + rg.slots);
-            issue_act(i + rg.slots);
+            issue_weights(i + rg.slots, slot);
+            if (!rg.act_smem) issue_act(i + rg.slots, slot);
         }
+        if (++slot == rg.slots) { slot = 0; phase ^= 1u; }
     }
-    if (alive && cur_u >= 0) flush(cur_u);
+    if (alive && pending) flush(cur_u);
 
     if constexpr (EPI == EPI_ARGMAX) {
         // publish this worker's best keys, then the last worker of the launch emits the tokens
@@ -508,18 +549,25 @@ cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
     constexpr LayoutInfo L = layout_info(FMT, GRP);
     RingGeom rg{};
     rg.act_row = L.KS * 2 + 16;
+    rg.act_stride = a.act_ld * 2 + 16;
+    const int act_total = a.B * rg.act_stride;
+    rg.act_smem = act_total <= 32 * 1024;
     const int wbytes = L.bps * L.block_bytes;
-    rg.slot_bytes = round_up(wbytes + L.bps * a.B * rg.act_row, 128);
-    rg.slots = kWarps * 3 * rg.slot_bytes <= 100 * 1024 ? 3 : 2;
-    if (rg.slots > 4) rg.slots = 4;
-    const size_t smem = (size_t)kWarps * rg.slots * rg.slot_bytes;
-    if (smem > 200 * 1024) return cudaErrorInvalidValue;
+    rg.slot_bytes = round_up(wbytes + (rg.act_smem ? 0 : L.bps * a.B * rg.act_row), 128);
+    // as many 4 KB-class slots per warp as the budget allows: the bytes in flight per SM
+    // (warps x (slots - 1) x slot) must cover HBM latency x per-SM bandwidth (~60-100 KB)
+    constexpr int WARPS = warps_for(NT);
+    rg.slots = (kRingBudget - (rg.act_smem ? act_total : 0)) / (WARPS * rg.slot_bytes);
+    if (rg.slots > kMaxSlots) rg.slots = kMaxSlots;
+    if (rg.slots < 2) rg.slots = 2;
+    const size_t smem = (size_t)WARPS * rg.slots * rg.slot_bytes + (rg.act_smem ? act_total : 0);
+    if (smem > 220 * 1024) return cudaErrorInvalidValue;
     auto kern = gemv_kernel<FMT, GRP, NT, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(Lh.num_sms);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(WARPS * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

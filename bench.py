@@ -1,0 +1,343 @@
+"""Benchmark of the per-frame decode step (and the reference arm: the CPU oracle).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl vc|reference]
+
+Default workload: the Nemotron-Nano-9B-v2-shaped backbone with bf16 weights, batch 1, steady
+state decode at a context of 2000 frames (KV cache and SSM state pre-filled from N(0,1)),
+synthetic seeded weights N(0, 0.02) and inputs N(0, 1).  One "step" is one frame through all
+56 layers and both vocabulary heads.  Other workloads: --config nano_w4 | nano_w3 |
+nano_w8_b16 | tiny_w8 (see synth.CONFIGS).
+
+With N > 1 (torchrun) every rank serves its own independent sessions with a full replica of
+the weights (no collective on the data path); the reported value is the sum over ranks of
+frames / max-over-ranks time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "backbone frame-steps/s & ms/frame at batch 1 and 16; achieved HBM GB/s vs 8 TB/s"
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic bytes (layout independent: what the method must read per frame)
+# ------------------------------------------------------------------------------------------------
+
+def weight_bits(fmt):
+    return {synth.FMT_BF16: 16, synth.FMT_W8: 8, synth.FMT_W4: 4, synth.FMT_W3: 3}[fmt]
+
+
+def matrix_bytes(fmt, group, N, K):
+    if fmt == synth.FMT_BF16:
+        return N * K * 2
+    ng = (K + group - 1) // group
+    zero_bits = 0 if fmt == synth.FMT_W8 else weight_bits(fmt)
+    return N * K * weight_bits(fmt) / 8 + N * ng * (2 + zero_bits / 8)
+
+
+def step_bytes(cfg, B, ctx_mean):
+    """bytes read per frame-step for B sessions: weights once, per-session SSM state, conv rows,
+    KV cache (ctx+1 keys), small vectors; and bytes written (state, conv row, KV append)."""
+    w = 0.0
+    for l in range(cfg.n_layers):
+        for _, N, K in synth.linear_shapes(cfg, l):
+            w += matrix_bytes(cfg.wfmt, cfg.group_size, N, K)
+        w += cfg.d_model * 4
+        if cfg.pattern[l] == "M":
+            w += (cfg.conv_dim * (cfg.conv_width + 1) + 3 * cfg.ssm_heads + cfg.d_inner) * 4
+    heads = matrix_bytes(cfg.head_fmt, cfg.group_size, cfg.vocab_text, cfg.d_model) + \
+        matrix_bytes(cfg.head_fmt, cfg.group_size, cfg.vocab_func, cfg.d_model)
+    ssm = cfg.n_mamba * cfg.ssm_heads * cfg.ssm_head_dim * cfg.ssm_state * 4
+    conv = cfg.n_mamba * (cfg.conv_width - 1) * cfg.conv_dim * 2
+    kv_frame = cfg.n_attn * 2 * cfg.attn_kv_heads * cfg.attn_head_dim * 2
+    read = w + heads + B * (ssm + conv + kv_frame * (ctx_mean + 1))
+    write = B * (ssm + cfg.n_mamba * cfg.conv_dim * 2 + kv_frame)
+    return read, write, w + heads
+
+
+def launches_per_step(cfg):
+    n = 1 + 1   # step input + heads
+    for k in cfg.pattern:
+        n += 3 if k in "M*" else 2
+    return n
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running"""
+
+    def __init__(self, index=0):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+                f = [x.strip() for x in out.stdout.strip().split(",")]
+                if len(f) >= 7:
+                    self.samples.append(f)
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def start(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[3 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle (cpu_baseline leg and --impl reference)
+# ------------------------------------------------------------------------------------------------
+
+def oracle_rate(cfg, n_steps, seed=0):
+    """time n_steps of the oracle on this host (all cores) from the same pre-filled state."""
+    import oracle
+    B = cfg.batch
+    model = oracle.Model(cfg, seed)
+    st = model.new_state(B, cfg.kv_capacity)
+    if cfg.random_state:
+        st.fill_random(seed, synth.context_lengths(cfg, seed, B))
+    t0 = time.perf_counter()
+    for s in range(n_steps):
+        model.step(st, synth.frame_inputs(cfg, seed, s, B), oracle.MIRROR)
+    dt = time.perf_counter() - t0
+    return B * n_steps / dt, dt
+
+
+def cpu_threads():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return
+    n = max(1, min(args.steps, 2 if cfg.d_model > 1000 else 64))
+    for _ in range(max(0, min(args.warmup, 1))):
+        pass
+    value, dt = oracle_rate(cfg, n)
+    sample = f"{n} frame-step(s) x batch {cfg.batch} of {cfg.name} per timed run"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "frame-steps/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * dt / n, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.batch, "ctx": cfg.ctx},
+            "cpu_baseline": {"value": value, "unit": "frame-steps/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "frame-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="nano_bf16", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="vc", choices=["vc", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    cfg = synth.CONFIGS[args.config]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+
+    import attention_frame_decode_b200 as vc
+    from attention_frame_decode_b200.synthetic import build_model, fill_state
+
+    B = cfg.batch
+    seed = 0
+    dm = build_model(cfg, seed)
+    cap = cfg.kv_capacity
+    bb = dm.backbone(B, cap, B)
+    st = dm.new_state(B, cap)
+    ctx0 = synth.context_lengths(cfg, seed, B)
+    if cfg.random_state:
+        fill_state(st, cfg, seed + rank, ctx0, cap)
+    total = args.warmup + args.steps
+    # every frame input of the run, resident in HBM before timing (rank r serves its own sessions)
+    xs = torch.empty((total, B, cfg.d_model), dtype=torch.bfloat16, device="cuda")
+    for s in range(total):
+        xs[s] = torch.from_numpy(synth.frame_inputs(cfg, seed + 1000 * rank, s, B)).view(torch.bfloat16)
+    tt = torch.zeros((B,), dtype=torch.int32, device="cuda")
+    tf = torch.zeros((B,), dtype=torch.int32, device="cuda")
+    if int(cap - ctx0.max()) < total + args.e2e_steps + 8:
+        raise SystemExit(f"kv capacity {cap} too small for {total + args.e2e_steps} steps")
+
+    for s in range(args.warmup):
+        bb.step(xs[s], st, tt, tf)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(args.warmup, total):
+        bb.step(xs[s], st, tt, tf)
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = int(st.status.cpu()[0])
+    ms_step = ms / args.steps
+    value = world * B * args.steps / (ms / 1000.0)
+    ctx_mean = float(ctx0.mean()) + args.warmup + args.steps / 2.0
+    rbytes, wbytes, weight_total = step_bytes(cfg, B, ctx_mean)
+    step_gbs = rbytes / (ms_step / 1000.0) / 1e9
+
+    # ---- roofline of the dominant kernel: the streaming GEMV on the layer MLP up projection ----
+    peak, peak_kind = load_peaks()
+    mlp = cfg.pattern.index("-")
+    up = dm.layers[mlp].up
+    K_up = cfg.d_model
+    act_ld = (K_up + 127) // 128 * 128
+    act = torch.zeros((B, act_ld), dtype=torch.bfloat16 if cfg.wfmt == synth.FMT_BF16 else torch.float16,
+                      device="cuda")
+    act[:, :K_up] = torch.randn((B, K_up), device="cuda").to(act.dtype)
+    scratch = vc.gemv_scratch()
+    ybuf = torch.empty((B, up.N), dtype=torch.float32, device="cuda")
+    wbuf = next(t for t in dm.keep if t.data_ptr() == up.data)
+    for _ in range(5):
+        vc.debug_gemv(wbuf, cfg.wfmt, cfg.group_size, up.N, up.K, act, scratch, out=ybuf)
+    reps = 50
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    g0.record()
+    for _ in range(reps):
+        vc.debug_gemv(wbuf, cfg.wfmt, cfg.group_size, up.N, up.K, act, scratch, out=ybuf)
+    g1.record()
+    torch.cuda.synchronize()
+    gemv_ms = g0.elapsed_time(g1) / reps
+    gemv_bytes = matrix_bytes(cfg.wfmt, cfg.group_size, up.N, up.K) + B * K_up * 2 + B * up.N * 4
+    gemv_gbs = gemv_bytes / (gemv_ms / 1000.0) / 1e9
+
+    # ---- end to end through the C ABI with host buffers (pinned x in, tokens out, every step) ----
+    ne = max(1, args.e2e_steps)
+    xh = torch.empty((ne, B, cfg.d_model), dtype=torch.bfloat16).pin_memory()
+    for s in range(ne):
+        xh[s] = torch.from_numpy(synth.frame_inputs(cfg, seed + 1000 * rank, total + s, B)).view(torch.bfloat16)
+    th = torch.empty((B,), dtype=torch.int32).pin_memory()
+    fh = torch.empty((B,), dtype=torch.int32).pin_memory()
+    stream = torch.cuda.current_stream()
+    bb.step_host(xh[0], st, th, fh)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for s in range(1, ne):
+        bb.step_host(xh[s], st, th, fh)
+        stream.synchronize()   # the frame's tokens are on the host before the next frame
+    e2e_s = time.perf_counter() - t0
+    if world > 1:
+        t = torch.tensor([e2e_s], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    e2e_value = world * B * (ne - 1) / e2e_s
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_or = 2 if cfg.d_model > 1000 else 64
+        v, dt = oracle_rate(cfg, n_or)
+        cpu = {"value": v, "unit": "frame-steps/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{n_or} frame-step(s) of the same workload (batch {B}) from the same pre-filled state, "
+                         f"{dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "frame-steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": {synth.FMT_BF16: "bf16", synth.FMT_W8: "w8-fp16", synth.FMT_W4: "w4-fp16",
+                      synth.FMT_W3: "w3-fp16"}[cfg.wfmt] + "-weights/fp32-accum",
+            "data": "synthetic (seeded N(0,0.02) weights, N(0,1) inputs and pre-filled state)",
+            "config": {"workload": cfg.name, "batch": B, "ctx_start": int(ctx0.max()) if B == 1 else
+                       [int(ctx0.min()), int(ctx0.max())], "layers": cfg.n_layers, "weights": synth.FMT_NAMES[cfg.wfmt],
+                       "group": cfg.group_size, "heads": synth.FMT_NAMES[cfg.head_fmt],
+                       "l2": f"no flush: {weight_total / 1e9:.2f} GB of weights per step >> 126 MB L2",
+                       "parallelism": f"replicas x{world}"},
+            "achieved_step_gbs": step_gbs, "step_bytes_read": rbytes, "step_bytes_written": wbytes,
+            "step_frac_of_peak": step_gbs / peak,
+            "roofline": {"bound": "hbm", "kernel": "gemv (mlp up projection, streaming weights)",
+                         "achieved": gemv_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": gemv_gbs / peak, "traffic": None, "launch_ms": gemv_ms,
+                         "bytes_per_launch": gemv_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "frame-steps/s", "h2d_bytes_per_step": B * cfg.d_model * 2,
+                    "d2h_bytes_per_step": 2 * B * 4, "steps": ne - 1},
+            "gpu_launches": launches_per_step(cfg) * args.steps,
+            "clocks": clk, "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    bb.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -198,6 +198,15 @@ vc_status vc_debug_mamba_step(const vc_config* cfg, const vc_layer_weights* laye
                               const int32_t* slots, float* ssm, void* conv, const int32_t* ctx_len, void* act,
                               float* parts, int32_t* status, vc_stream_t stream);
 
+/* test/measurement: y = W u with the decode step's streaming GEMV kernel.
+ * act: 16-bit [B][act_ld] (device; bf16 bits for VC_W_BF16 weights, fp16 bits for quantized
+ * ones), act_ld a multiple of 128 and >= K rounded up to 128, columns K..act_ld-1 zero;
+ * 1 <= B <= 16.  out: fp32 [B][N] (device).  scratch: device buffer of vc_gemv_scratch_bytes()
+ * bytes, zero on first use; the kernel leaves it zeroed again for the next call. */
+size_t vc_gemv_scratch_bytes(void);
+vc_status vc_debug_gemv(const vc_qmat* w, const void* act, int act_ld, int B, float* out, void* scratch,
+                        vc_stream_t stream);
+
 void vc_destroy(vc_backbone* h);
 
 const char* vc_status_string(vc_status s);

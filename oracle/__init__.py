@@ -271,6 +271,14 @@ class State:
         self.ctx_len = np.zeros((n_slots,), np.int32)
         self.c = OrState(n_slots, cap, _ptr(self.ssm), _ptr(self.conv), _ptr(self.k), _ptr(self.v), _ptr(self.ctx_len))
 
+    def clone(self) -> "State":
+        o = State.__new__(State)
+        o.cfg, o.n_slots, o.cap = self.cfg, self.n_slots, self.cap
+        o.ssm, o.conv, o.k, o.v = self.ssm.copy(), self.conv.copy(), self.k.copy(), self.v.copy()
+        o.ctx_len = self.ctx_len.copy()
+        o.c = OrState(o.n_slots, o.cap, _ptr(o.ssm), _ptr(o.conv), _ptr(o.k), _ptr(o.v), _ptr(o.ctx_len))
+        return o
+
     def fill_random(self, seed: int, ctx_lens: np.ndarray):
         """Pre-fill every slot from the seeded generator (the same tensors the GPU harness uploads)."""
         cfg = self.cfg

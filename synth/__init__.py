@@ -200,7 +200,7 @@ def nano_config(**kw) -> Config:
                ssm_state=128, ssm_groups=8, conv_width=4, norm_groups=8, attn_q_heads=40,
                attn_kv_heads=8, attn_head_dim=128, mlp_hidden=15680, vocab_text=131072,
                vocab_func=131072, wfmt=FMT_BF16, group_size=64, head_fmt=FMT_BF16, batch=1,
-               ctx=2000, steps=1000, kv_capacity=3000, random_state=True)
+               ctx=2000, steps=1000, kv_capacity=3300, random_state=True)
     return c.replace(**kw)
 
 
@@ -210,7 +210,7 @@ CONFIGS = {
     "nano_w4": nano_config(name="nano_w4", wfmt=FMT_W4, group_size=64),
     "nano_w3": nano_config(name="nano_w3", wfmt=FMT_W3, group_size=64),
     "nano_w8_b16": nano_config(name="nano_w8_b16", wfmt=FMT_W8, group_size=128, batch=16,
-                               ctx_range=(500, 6000), steps=500, kv_capacity=6500),
+                               ctx_range=(500, 6000), steps=500, kv_capacity=7000),
     "nano_prefill": nano_config(name="nano_prefill", ctx=0, prefill_T=4096, steps=0,
                                 kv_capacity=4096 + 64, random_state=False),
 }

