@@ -188,7 +188,7 @@ extern "C" size_t vc_workspace_bytes(const vc_config* cfg) {
     add((size_t)B * ldh * 2);                 // act_h
     add((size_t)B * D.zx_rows * 2);           // zx
     add((size_t)B * D.Hq * D.Dh * 2);         // q
-    add((size_t)B * ((D.d + 31) / 32) * 4);   // parts_r (units of >= 32 rows)
+    add((size_t)B * ((D.d + 15) / 16) * 4);   // parts_r (one per 16-row unit)
     add((size_t)B * 2 * D.H * 4 + 16);        // parts_g
     add((size_t)16 * 4);                      // ok
     add(gemv_partials_bytes(256));            // partials (any SM count up to 256)
@@ -225,7 +225,7 @@ static void carve(vc_backbone* h, uint8_t* base) {
     W.act_h = (uint16_t*)take((size_t)B * W.ldh * 2);
     W.zx = (uint16_t*)take((size_t)B * D.zx_rows * 2);
     W.q = (uint16_t*)take((size_t)B * D.Hq * D.Dh * 2);
-    W.parts_r = (float*)take((size_t)B * ((D.d + 31) / 32) * 4);
+    W.parts_r = (float*)take((size_t)B * ((D.d + 15) / 16) * 4);
     W.parts_g = (float*)take((size_t)B * 2 * D.H * 4 + 16);
     W.ok = (int*)take(16 * 4);
     W.partials = (float*)take(gemv_partials_bytes(256));
@@ -274,9 +274,6 @@ extern "C" vc_status vc_backbone_create(const vc_config* cfg, const vc_weights* 
     if (!qmat_ok(weights->head_text, cfg->head_fmt, grp, D.Vt, D.d) ||
         !qmat_ok(weights->head_func, cfg->head_fmt, grp, D.Vf, D.d))
         return VC_ERR_INVALID_ARG;
-    // the residual epilogue writes row-unit sums of squares: every d-row matrix must use the
-    // same unit height as the step-input kernel
-    if (layout_info(fmt, grp).R * 16 < 32) return VC_ERR_UNSUPPORTED;
 
     vc_backbone* h = new vc_backbone();
     h->cfg = *cfg;

@@ -107,26 +107,36 @@ __global__ void __launch_bounds__(kMambaThreads) mamba_step_kernel(const MambaSt
     const float dt_bias = a.dt_bias[h], A = -expf(a.A_log[h]), Dh = a.D[h];
 
     pdl_wait();
+    // one round trip for this frame's inputs: x/B/C pre-activations (kept raw for the ring),
+    // the gate z and dt_raw; the ring slot t mod W is written at the end
     const bool okb = a.ok ? a.ok[b] != 0 : true;
     const uint16_t* zx = a.zx + (size_t)b * a.zx_ld;
     const uint16_t* xBC = zx + a.E;
-    for (int i = tid; i < Ph + 2 * a.N; i += kMambaThreads) {
+    uint16_t raw[2];
+    int chan[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int i = tid + q * kMambaThreads;
+        chan[q] = -1;
+        if (i < Ph + 2 * a.N) {
+            float* dst;
+            chan[q] = channel(i, dst);
+            raw[q] = xBC[chan[q]];
+        }
+    }
+    float* zs = Cs + a.N;   // [Ph] silu(z)
+    for (int i = tid; i < Ph; i += kMambaThreads) zs[i] = silu_f(bf16_bits_to_f(zx[h * a.P + p0 + i]));
+    const float dt_raw = bf16_bits_to_f(zx[a.E + a.Cx + h]);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        if (chan[q] < 0) continue;
         float* dst;
-        const int c = channel(i, dst);
-        *dst = silu_f(*dst + a.conv_w[c * a.W + a.W - 1] * bf16_bits_to_f(xBC[c]));
+        channel(tid + q * kMambaThreads, dst);
+        *dst = silu_f(*dst + a.conv_w[chan[q] * a.W + a.W - 1] * bf16_bits_to_f(raw[q]));
     }
-    __syncthreads();   // all window reads done before the ring slot t mod W is overwritten
-    if (okb) {
-        uint16_t* rw = ring + (size_t)(t % a.W) * a.Cx;
-        for (int i = tid; i < Ph; i += kMambaThreads) rw[h * a.P + p0 + i] = xBC[h * a.P + p0 + i];
-        if (writes_bc)
-            for (int i = tid; i < 2 * a.N; i += kMambaThreads) {
-                const int c = a.E + (i < a.N ? g * a.N + i : a.G * a.N + g * a.N + (i - a.N));
-                rw[c] = xBC[c];
-            }
-    }
+    __syncthreads();
 
-    const float dt = softplus_f(bf16_bits_to_f(zx[a.E + a.Cx + h]) + dt_bias);
+    const float dt = softplus_f(dt_raw + dt_bias);
     const float decay = expf(A * dt);
 
     if (!mbar_wait(&bar, 0, a.status)) return;
@@ -147,13 +157,22 @@ __global__ void __launch_bounds__(kMambaThreads) mamba_step_kernel(const MambaSt
         if (lane == 0) {
             const int c = h * a.P + p0 + pr;
             y = fmaf(Dh, xv, y);
-            const float v = y * silu_f(bf16_bits_to_f(zx[c]));
+            const float v = y * zs[pr];
             ss += v * v;
             const float an = v * a.gnorm[c];
             a.act[(size_t)b * a.act_ld + c] = a.act_f16 ? act_bits<true>(an) : act_bits<false>(an);
         }
     }
     if (lane == 0) red[warp] = ss;
+    // the ring slot of frame t (disjoint from the W-1 slots any CTA reads this frame)
+    if (okb) {
+        uint16_t* rw = ring + (size_t)(t % a.W) * a.Cx;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int i = tid + q * kMambaThreads;
+            if (chan[q] >= 0 && (i < Ph || writes_bc)) rw[chan[q]] = raw[q];
+        }
+    }
     __syncthreads();
     if (tid == 0) {
         float tot = 0.0f;
@@ -164,7 +183,8 @@ __global__ void __launch_bounds__(kMambaThreads) mamba_step_kernel(const MambaSt
 
 cudaError_t launch_mamba_step(const MambaStepArgs& a, int pdl, cudaStream_t s) {
     const int Ph = a.P / 2;
-    const size_t smem = (size_t)(Ph * a.N + Ph + 2 * a.N) * sizeof(float);
+    if (Ph + 2 * a.N > 2 * kMambaThreads) return cudaErrorInvalidValue;
+    const size_t smem = (size_t)(Ph * a.N + 2 * Ph + 2 * a.N) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(mamba_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};

@@ -10,7 +10,7 @@ static constexpr int kMaxBDispatch = 16;
 // host launch
 // ------------------------------------------------------------------------------------------
 size_t gemv_partials_bytes(int num_sms) { return (size_t)num_sms * kWarps * 2 * (4 * 2 * 128) * sizeof(float); }
-size_t gemv_counter_ints() { return 2 * 8192; }
+size_t gemv_counter_ints() { return 2 * 65536; }
 
 cudaError_t launch_gemv(const GemvLaunch& L, const GemvArgs& a, cudaStream_t s) {
     if (a.B < 1 || a.B > kMaxBDispatch) return cudaErrorInvalidValue;

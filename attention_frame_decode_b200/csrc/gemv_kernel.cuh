@@ -24,7 +24,11 @@ namespace vc {
 
 static constexpr int kWarps = 16;   // upper bound of warps per CTA
 // warps per CTA: 16 for up to 8 batch rows (<= 128 registers each), 8 for 9..16 rows
-__host__ __device__ constexpr int warps_for(int NT) { return NT == 1 ? 16 : 8; }
+__host__ __device__ constexpr int warps_for(int) { return 8; }
+// CTAs per SM: two 8-warp CTAs for up to 8 rows (<= 128 registers, <= ~105 KB shared memory each),
+// so that under programmatic dependent launch the next kernel's CTAs can become resident and
+// start their weight copies while this kernel drains; one CTA for 9..16 rows
+__host__ __device__ constexpr int ctas_per_sm(int NT) { return NT == 1 ? 2 : 1; }
 static constexpr int kMaxB = 16;
 static constexpr int kMaxSlots = 8;          // ring slots per warp (upper bound)
 static constexpr int kRingBudget = 210 * 1024; // dynamic shared memory for the rings of one CTA
@@ -138,7 +142,7 @@ struct RingGeom {
 };
 
 template <int FMT, int GRP, int NT, int EPI>
-__global__ void __launch_bounds__(warps_for(NT) * 32, 1) gemv_kernel(const GemvArgs args, const RingGeom rg) {
+__global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kernel(const GemvArgs args, const RingGeom rg) {
     constexpr int WARPS = warps_for(NT);
     constexpr LayoutInfo L = layout_info(FMT, GRP);
     constexpr int R = L.R, SUB = L.SUB, KS = L.KS;
@@ -375,10 +379,10 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, 1) gemv_kernel(const GemvA
             for (int j = 0; j < NT; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) tot[r][j][e] = 0.0f;
-        for (long long w0 = lo; w0 <= hi; w0 += 4) {
-            float4 x[4][R * NT];
+        for (long long w0 = lo; w0 <= hi; w0 += 2) {
+            float4 x[2][R * NT];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 const long long w2 = w0 + q;
                 if (w2 > hi) break;
                 const long long fu = part_begin(w2, T, Wm) / M.KT;
@@ -387,7 +391,7 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, 1) gemv_kernel(const GemvA
                 for (int rj = 0; rj < R * NT; ++rj) x[q][rj] = __ldcg(reinterpret_cast<const float4*>(p + (rj * 32 + lane) * 4));
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 if (w0 + q > hi) break;
 #pragma unroll
                 for (int r = 0; r < R; ++r)
@@ -557,7 +561,8 @@ cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
     // as many 4 KB-class slots per warp as the budget allows: the bytes in flight per SM
     // (warps x (slots - 1) x slot) must cover HBM latency x per-SM bandwidth (~60-100 KB)
     constexpr int WARPS = warps_for(NT);
-    rg.slots = (kRingBudget - (rg.act_smem ? act_total : 0)) / (WARPS * rg.slot_bytes);
+    const int budget = kRingBudget / ctas_per_sm(NT) - 4096;   // two CTAs must fit one SM
+    rg.slots = (budget - (rg.act_smem ? act_total : 0)) / (WARPS * rg.slot_bytes);
     if (rg.slots > kMaxSlots) rg.slots = kMaxSlots;
     if (rg.slots < 2) rg.slots = 2;
     const size_t smem = (size_t)WARPS * rg.slots * rg.slot_bytes + (rg.act_smem ? act_total : 0);
@@ -566,7 +571,7 @@ cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(Lh.num_sms);
+    cfg.gridDim = dim3(Lh.num_sms * ctas_per_sm(NT));
     cfg.blockDim = dim3(WARPS * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
