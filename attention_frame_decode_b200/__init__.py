@@ -68,11 +68,17 @@ _lib.vc_step.argtypes = [_p, _p, _i, _p, C.POINTER(VcState), _p, _p, _p]
 _lib.vc_step_host.argtypes = [_p, _p, _i, _p, C.POINTER(VcState), _p, _p, _p]
 _lib.vc_prefill.argtypes = [_p, _p, _i, _i, C.POINTER(VcState), _p]
 _lib.vc_debug_set_taps.argtypes = [_p, _p, _p]
+_lib.vc_debug_set_prefill_taps.argtypes = [_p, _p]
 _lib.vc_debug_mamba_step.argtypes = [C.POINTER(VcConfig), C.POINTER(VcLayerWeights), _p, _i, _p, _p, _p, _p, _p, _p,
                                       _p, _p]
 _lib.vc_gemv_scratch_bytes.argtypes = []
 _lib.vc_gemv_scratch_bytes.restype = C.c_size_t
 _lib.vc_debug_gemv.argtypes = [C.POINTER(VcQmat), _p, _i, _i, _p, _p, _p]
+_lib.vc_debug_gemm.argtypes = [_p, _i, _i, _p, _i, _i, _i, _i, _p, _i, _p, _p]
+_lib.vc_debug_mamba_prefill_scratch_bytes.argtypes = [C.POINTER(VcConfig), _i]
+_lib.vc_debug_mamba_prefill_scratch_bytes.restype = C.c_size_t
+_lib.vc_debug_mamba_prefill.argtypes = [C.POINTER(VcConfig), C.POINTER(VcLayerWeights), _p, _i, _p, _p, _p, _p, _p,
+                                        _p]
 _lib.vc_destroy.argtypes = [_p]
 _lib.vc_destroy.restype = None
 _lib.vc_status_string.argtypes = [_i]
@@ -80,13 +86,16 @@ _lib.vc_status_string.restype = C.c_char_p
 _lib.vc_last_cuda_error.argtypes = []
 _lib.vc_last_cuda_error.restype = C.c_char_p
 for _f in ("vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant", "vc_backbone_create",
-           "vc_set_option", "vc_step", "vc_step_host", "vc_prefill", "vc_debug_set_taps", "vc_debug_mamba_step",
-           "vc_debug_gemv"):
+           "vc_set_option", "vc_step", "vc_step_host", "vc_prefill", "vc_debug_set_taps", "vc_debug_set_prefill_taps",
+           "vc_debug_mamba_step",
+           "vc_debug_gemv", "vc_debug_gemm", "vc_debug_mamba_prefill"):
     getattr(_lib, _f).restype = _i
 
 EXPORTS = ("vc_weight_bytes", "vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant",
            "vc_workspace_bytes", "vc_backbone_create", "vc_set_option", "vc_step", "vc_step_host", "vc_prefill",
-           "vc_debug_set_taps", "vc_debug_mamba_step", "vc_gemv_scratch_bytes", "vc_debug_gemv", "vc_destroy",
+           "vc_debug_set_taps", "vc_debug_set_prefill_taps", "vc_debug_mamba_step", "vc_gemv_scratch_bytes",
+           "vc_debug_gemv", "vc_debug_gemm",
+           "vc_debug_mamba_prefill_scratch_bytes", "vc_debug_mamba_prefill", "vc_destroy",
            "vc_status_string", "vc_last_cuda_error")
 
 
@@ -209,6 +218,32 @@ def debug_gemv(wbuf, fmt, group, N, K, act, scratch, out=None, stream=None):
     return out
 
 
+def debug_gemm(A, W, status, out=None, stream=None):
+    """out[M][N] = A W^T (fp32) with the prefill's tensor-core GEMM; A [M][K] and W [N][K] are bf16 or
+    fp16 CUDA tensors (same dtype; row strides multiples of 8 elements)."""
+    import torch
+    M, K = A.shape
+    N = W.shape[0]
+    assert W.shape[1] == K and A.dtype == W.dtype and A.dtype in (torch.bfloat16, torch.float16)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    _check(_lib.vc_debug_gemm(_ptr(A), A.stride(0), M, _ptr(W), W.stride(0), N, K, int(A.dtype == torch.float16),
+                              _ptr(out), out.stride(0), _ptr(status), _stream(stream)), "vc_debug_gemm")
+    return out
+
+
+def debug_mamba_prefill(cfg_c: VcConfig, layer: VcLayerWeights, zx, ssm, conv, y, act, stream=None):
+    """the prefill's Mamba-2 mixer over T = zx.shape[0] frames from an empty state"""
+    import torch
+    T = zx.shape[0]
+    nbytes = _lib.vc_debug_mamba_prefill_scratch_bytes(C.byref(cfg_c), T)
+    if nbytes == 0:
+        raise VcError(VC_ERR_INVALID_ARG, "vc_debug_mamba_prefill_scratch_bytes")
+    scratch = torch.empty((nbytes,), dtype=torch.uint8, device=zx.device)
+    _check(_lib.vc_debug_mamba_prefill(C.byref(cfg_c), C.byref(layer), _ptr(zx), T, _ptr(ssm), _ptr(conv), _ptr(y),
+                                       _ptr(act), _ptr(scratch), _stream(stream)), "vc_debug_mamba_prefill")
+
+
 def debug_mamba_step(cfg_c: VcConfig, layer: VcLayerWeights, zx, slots, ssm, conv, ctx_len, act, parts, status,
                      stream=None):
     B = zx.shape[0]
@@ -262,6 +297,10 @@ class Backbone:
     def set_taps(self, hidden=None, logits=None):
         self._taps = (hidden, logits)
         _check(_lib.vc_debug_set_taps(self.h, _ptr(hidden), _ptr(logits)), "vc_debug_set_taps")
+
+    def set_prefill_taps(self, hidden=None):
+        self._ptaps = hidden
+        _check(_lib.vc_debug_set_prefill_taps(self.h, _ptr(hidden)), "vc_debug_set_prefill_taps")
 
     def step(self, x, state: State, tok_text, tok_func, slots=None, stream=None):
         B = x.shape[0]

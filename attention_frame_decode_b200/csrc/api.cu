@@ -12,6 +12,7 @@
 #include "../../include/vc.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "layout.cuh"
 #include "prefill.cuh"
@@ -127,6 +128,7 @@ struct vc_backbone {
     int use_graph = 1, use_pdl = 1;
     float* tap_hidden = nullptr;
     float* tap_logits = nullptr;
+    float* tap_prefill = nullptr;
     struct Graph {
         cudaGraph_t graph;
         cudaGraphExec_t exec;
@@ -312,6 +314,12 @@ extern "C" vc_status vc_set_option(vc_backbone* h, int option, int value) {
     else if (option == VC_OPT_PDL) h->use_pdl = value != 0;
     else return VC_ERR_INVALID_ARG;
     clear_graphs(h);
+    return VC_OK;
+}
+
+extern "C" vc_status vc_debug_set_prefill_taps(vc_backbone* h, float* hidden) {
+    if (!h) return VC_ERR_INVALID_ARG;
+    h->tap_prefill = hidden;
     return VC_OK;
 }
 
@@ -553,6 +561,7 @@ extern "C" vc_status vc_prefill(vc_backbone* h, const void* x, int T, int slot, 
     c.ws = h->ws.prefill; c.ws_bytes = h->ws.prefill_bytes;
     c.ssm = state->ssm; c.conv = (uint16_t*)state->conv; c.k = (uint16_t*)state->k; c.v = (uint16_t*)state->v;
     c.ctx_len = state->ctx_len; c.status = state->status;
+    c.tap = h->tap_prefill;
     cudaError_t e = run_prefill(c, (const uint16_t*)x, T, slot, (cudaStream_t)stream);
     if (e == cudaErrorNotSupported) return VC_ERR_UNSUPPORTED;
     if (e == cudaErrorInvalidValue) return VC_ERR_INVALID_ARG;
@@ -605,6 +614,50 @@ extern "C" vc_status vc_debug_gemv(const vc_qmat* w, const void* act, int act_ld
     L.num_sms = sms > 256 ? 256 : sms;
     L.pdl = 0;
     CK(launch_gemv(L, a, (cudaStream_t)stream));
+    return VC_OK;
+}
+
+extern "C" size_t vc_debug_mamba_prefill_scratch_bytes(const vc_config* cfg, int T) {
+    Dims D;
+    if (!dims_from_cfg(cfg, D) || !D.nm || T < 1) return 0;
+    return prefill_mixer_scratch_bytes(T, D.E, D.Cx, D.H, D.P, D.N);
+}
+
+extern "C" vc_status vc_debug_mamba_prefill(const vc_config* cfg, const vc_layer_weights* layer, const void* zx, int T,
+                                            float* ssm, void* conv, float* y, void* act, void* scratch,
+                                            vc_stream_t stream) {
+    Dims D;
+    if (!dims_from_cfg(cfg, D) || !D.nm || !layer || !zx || !ssm || !conv || !y || !act || !scratch || T < 1)
+        return VC_ERR_INVALID_ARG;
+    if (!aligned16(scratch) || !aligned16(zx)) return VC_ERR_INVALID_ARG;
+    PfMixer m{};
+    m.T = T; m.E = D.E; m.Cx = D.Cx; m.H = D.H; m.P = D.P; m.N = D.N; m.G = D.G; m.W = D.W; m.NG = D.NG;
+    m.eps = cfg->eps;
+    m.f16 = 0;
+    m.Lw = layer;
+    m.zx = (const uint16_t*)zx;
+    carve_mixer(m, (uint8_t*)scratch);
+    m.ssm = ssm; m.ring = (uint16_t*)conv; m.act = (uint16_t*)act; m.act_ld = D.E;
+    cudaStream_t s = (cudaStream_t)stream;
+    CK(prefill_mixer(m, s));
+    CK(cudaMemcpyAsync(y, m.y, (size_t)T * D.E * 4, cudaMemcpyDeviceToDevice, s));
+    return VC_OK;
+}
+
+extern "C" vc_status vc_debug_gemm(const void* A, int lda, int M, const void* W, int ldw, int N, int K, int f16,
+                                   float* out, int ldo, int32_t* status, vc_stream_t stream) {
+    if (!A || !W || !out || !status || !aligned16(A) || !aligned16(W)) return VC_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 1 || K % 8 || lda % 8 || ldw % 8 || lda < K || ldw < K || ldo < N)
+        return VC_ERR_INVALID_ARG;
+    GemmArgs a{};
+    a.f16 = f16 != 0;
+    a.A = A; a.lda = lda; a.M = M;
+    a.W = W; a.ldw = ldw; a.N = N; a.K = K;
+    a.out_f32 = out; a.ldo32 = ldo;
+    a.status = status;
+    cudaError_t e = launch_gemm_tc(GE_F32, a, (cudaStream_t)stream);
+    if (e == cudaErrorInvalidValue) return VC_ERR_INVALID_ARG;
+    CK(e);
     return VC_OK;
 }
 

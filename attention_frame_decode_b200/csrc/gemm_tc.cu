@@ -1,0 +1,282 @@
+// gemm_tc.cu -- tcgen05 GEMM for the prefill projections (dense contraction over the frames).
+//
+// C[M][N] = A[M][K] . W[N][K]^T, bf16 x bf16 -> fp32 in tensor memory (TMEM).
+// Tile 128 x 256 x 64, 4-stage TMA ring (128-byte swizzle, no multicast), one CTA per tile:
+//   warp 0 (one thread): TMA producer, waits "empty" mbarriers, loads A and W tiles;
+//   warp 1: allocates 256 TMEM columns; one thread issues tcgen05.mma (M=128, N=256, K=16,
+//           4 per 64-wide k-block) and tcgen05.commit to free each stage and, at the end, to
+//           signal the accumulator;
+//   warps 2-5: epilogue; each reads its 32 TMEM lanes (rows) with tcgen05.ld and applies the
+//           fused epilogue (row scale of the pre-RMSNorm, squared ReLU, residual add, q/k/v split
+//           into the KV cache) while storing to global memory.
+// Every mbarrier wait is bounded; a timeout sets the status word and the CTA still frees TMEM.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+
+namespace vc {
+
+static constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+static constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
+static constexpr int GEMM_THREADS = 192;
+static constexpr int TMEM_COLS = 256;
+
+VC_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// shared-memory matrix descriptor: K-major tile, rows of 128 B (64 bf16) in 8-row swizzle atoms
+VC_DEV uint64_t desc_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);          // start address
+    d |= (uint64_t)1 << 16;                            // leading byte offset (unused, K-major swizzled)
+    d |= (uint64_t)(1024 >> 4) << 32;                  // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                            // descriptor version
+    d |= (uint64_t)2 << 61;                            // 128-byte swizzle
+    return d;
+}
+
+// instruction descriptor: 16-bit x 16-bit -> f32 (D format 1 at bit 4), A and B format at bits 7
+// and 10 (0 = fp16, 1 = bf16), both operands K-major, N >> 3 at bit 17, M >> 4 at bit 24
+template <bool F16>
+VC_DEV constexpr uint32_t idesc() {
+    return (1u << 4) | ((F16 ? 0u : 1u) << 7) | ((F16 ? 0u : 1u) << 10) | ((uint32_t)(BN >> 3) << 17) |
+           ((uint32_t)(BM >> 4) << 24);
+}
+
+VC_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+VC_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+VC_DEV void tc_mma(uint32_t tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+VC_DEV void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+VC_DEV void tc_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+        "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int EPI, bool F16>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, const GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[STAGES], empty[STAGES], accum;
+    __shared__ uint32_t tmem_base;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+    const int KB = (a.K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&accum, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int kb = 0; kb < KB; ++kb) {
+                const int s = kb % STAGES;
+                if (kb >= STAGES && !mbar_wait(&empty[s], (uint32_t)(((kb / STAGES) - 1) & 1), a.status)) break;
+                mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                tma_load_2d(smem + s * STAGE_BYTES, &tmA, kb * BK, m0, &full[s]);
+                tma_load_2d(smem + s * STAGE_BYTES + A_BYTES, &tmW, kb * BK, n0, &full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            bool ok = true;
+            for (int kb = 0; kb < KB && ok; ++kb) {
+                const int s = kb % STAGES;
+                if (!mbar_wait(&full[s], (uint32_t)((kb / STAGES) & 1), a.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t abase = smem_u32(smem + s * STAGE_BYTES), bbase = abase + A_BYTES;
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                    tc_mma(tmem, desc_sw128(abase + k * 32), desc_sw128(bbase + k * 32), idesc<F16>(), (kb | k) != 0);
+                tc_commit(&empty[s]);
+            }
+            tc_commit(&accum);   // arrives when every issued MMA has completed
+        }
+    } else {
+        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
+        const int quarter = warp & 3;
+        const int row = m0 + quarter * 32 + lane;
+        const bool ready = mbar_wait(&accum, 0, a.status);
+        tc_fence_after();
+        if (ready) {
+            const float rs = (a.row_scale && row < a.M) ? a.row_scale[row] : 1.0f;
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                float v[32];
+                tc_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, v);
+                if (row >= a.M) continue;
+                const int col0 = n0 + c0;
+                if constexpr (EPI == GE_F32) {
+                    for (int j = 0; j < 32; ++j)
+                        if (col0 + j < a.N) a.out_f32[(size_t)row * a.ldo32 + col0 + j] = v[j];
+                } else if constexpr (EPI == GE_RESID) {
+                    float* dst = a.out_f32 + (size_t)row * a.ldo32 + col0;
+                    for (int j = 0; j < 32; ++j)
+                        if (col0 + j < a.N) dst[j] += v[j];
+                } else if constexpr (EPI == GE_QKV) {
+                    const int qrows = a.Hq * a.Dh;
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = col0 + j;
+                        if (col >= a.N) break;
+                        const uint16_t bits = act_bits<false>(v[j] * rs);
+                        if (col < qrows) {
+                            a.out[(size_t)row * a.ldo + col] = bits;
+                        } else {
+                            const int rr = col - qrows, kvsel = rr / (a.Hk * a.Dh);
+                            const int jj = (rr % (a.Hk * a.Dh)) / a.Dh, d = rr % a.Dh;
+                            uint16_t* cache = kvsel == 0 ? a.kcache : a.vcache;
+                            cache[((size_t)jj * a.cap + a.t0 + row) * a.Dh + d] = bits;
+                        }
+                    }
+                } else {
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        float x0 = v[2 * j] * rs, x1 = v[2 * j + 1] * rs;
+                        if constexpr (EPI == GE_RELU2) {
+                            x0 = fmaxf(x0, 0.0f); x0 *= x0;
+                            x1 = fmaxf(x1, 0.0f); x1 *= x1;
+                        }
+                        packed[j] = (EPI == GE_RELU2 && a.out_f16)
+                                        ? ((uint32_t)act_bits<true>(x0) | ((uint32_t)act_bits<true>(x1) << 16))
+                                        : ((uint32_t)act_bits<false>(x0) | ((uint32_t)act_bits<false>(x1) << 16));
+                    }
+                    uint16_t* dst = a.out + (size_t)row * a.ldo + col0;
+                    if (col0 + 32 <= a.N && (((uintptr_t)dst) & 15) == 0) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            reinterpret_cast<uint4*>(dst)[q] =
+                                make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                    } else {
+                        for (int j = 0; j < 32 && col0 + j < a.N; ++j)
+                            dst[j] = (uint16_t)(packed[j / 2] >> (16 * (j & 1)));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// host: tensor maps and launch
+// ------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D 16-bit tensor map over rows x cols (row stride ld elements), box 64 x box_rows, 128 B swizzle
+static bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows, bool f16) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI, bool F16>
+static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mw, const GemmArgs& a, cudaStream_t s) {
+    const size_t smem = (size_t)STAGES * STAGE_BYTES + 1024;
+    auto kern = gemm_tc_kernel<EPI, F16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM);
+    kern<<<grid, GEMM_THREADS, smem, s>>>(ma, mw, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(int epi, const GemmArgs& a, cudaStream_t s) {
+    // TMA: 16-byte aligned bases, row strides a multiple of 16 bytes, K a multiple of 8 elements
+    if ((((uintptr_t)a.A) & 15) || (((uintptr_t)a.W) & 15) || (a.lda % 8) || (a.ldw % 8) || (a.K % 8) || a.M < 1 ||
+        a.N < 1 || a.K < 1)
+        return cudaErrorInvalidValue;
+    CUtensorMap ma, mw;
+    const bool f16 = a.f16 != 0;
+    if (!make_map(&ma, a.A, a.M, a.K, a.lda, BM, f16) || !make_map(&mw, a.W, a.N, a.K, a.ldw, BN, f16))
+        return cudaErrorInvalidValue;
+    if (f16) {
+        switch (epi) {
+            case GE_F32: return launch_t<GE_F32, true>(ma, mw, a, s);
+            case GE_ROWSCALE: return launch_t<GE_ROWSCALE, true>(ma, mw, a, s);
+            case GE_RELU2: return launch_t<GE_RELU2, true>(ma, mw, a, s);
+            case GE_RESID: return launch_t<GE_RESID, true>(ma, mw, a, s);
+            case GE_QKV: return launch_t<GE_QKV, true>(ma, mw, a, s);
+        }
+    } else {
+        switch (epi) {
+            case GE_F32: return launch_t<GE_F32, false>(ma, mw, a, s);
+            case GE_ROWSCALE: return launch_t<GE_ROWSCALE, false>(ma, mw, a, s);
+            case GE_RELU2: return launch_t<GE_RELU2, false>(ma, mw, a, s);
+            case GE_RESID: return launch_t<GE_RESID, false>(ma, mw, a, s);
+            case GE_QKV: return launch_t<GE_QKV, false>(ma, mw, a, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace vc

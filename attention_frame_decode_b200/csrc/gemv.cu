@@ -183,6 +183,59 @@ __global__ void dequant_kernel(int N, int K, int KT, const uint8_t* in, float* o
     (void)L;
 }
 
+// dense 16-bit row-major copy out[n][k] (row stride ldo) of a weight in the device layout, for the
+// tensor-core GEMMs of the prefill: bf16 weights are copied bit for bit; quantized weights become
+// s*(q - z) rounded once to fp16 (f16 = 1, the value the decode GEMV's dequantization produces) or
+// to bf16 (f16 = 0)
+template <int FMT, int GRP>
+__global__ void unpack_kernel(int N, int K, int KT, const uint8_t* in, uint16_t* out, int ldo, int f16) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)N * K) return;
+    const int n = (int)(i / K), k = (int)(i % K);
+    const uint32_t c = get_code<FMT, GRP>(in, KT, n, k);
+    uint16_t bits;
+    if (FMT == FMT_BF16) {
+        bits = (uint16_t)c;
+    } else {
+        CodePos P = code_pos(FMT, GRP, KT, n, k);
+        const float s = __half2float(*reinterpret_cast<const __half*>(in + P.meta + P.g * 4 + P.hi * 2));
+        int q;
+        if (FMT == FMT_W8) q = (int)c - 128;
+        else {
+            const uint32_t zb = in[P.meta + 32 + P.g];
+            q = (int)c - (int)(P.hi ? (zb >> 4) : (zb & 15u));
+        }
+        const float w = s * (float)q;   // exact in fp32
+        bits = f16 ? __half_as_ushort(__float2half_rn(w)) : __bfloat16_as_ushort(__float2bfloat16_rn(w));
+    }
+    out[(size_t)n * ldo + k] = bits;
+}
+
+template <int FMT, int GRP>
+static cudaError_t unp_t(int N, int K, const uint8_t* w, uint16_t* out, int ldo, int f16, cudaStream_t s) {
+    MatGeom G = mat_geom(FMT, GRP, N, K);
+    const long long total = (long long)N * K;
+    unpack_kernel<FMT, GRP><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(N, K, G.KT, w, out, ldo, f16);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unpack16(int fmt, int group, int N, int K, const uint8_t* w, uint16_t* out, int ldo, int f16,
+                            cudaStream_t s) {
+    switch (fmt) {
+        case FMT_BF16: return unp_t<FMT_BF16, 64>(N, K, w, out, ldo, f16, s);
+        case FMT_W8:
+            return group == 128 ? unp_t<FMT_W8, 128>(N, K, w, out, ldo, f16, s)
+                                : unp_t<FMT_W8, 64>(N, K, w, out, ldo, f16, s);
+        case FMT_W4:
+            return group == 128 ? unp_t<FMT_W4, 128>(N, K, w, out, ldo, f16, s)
+                                : unp_t<FMT_W4, 64>(N, K, w, out, ldo, f16, s);
+        case FMT_W3:
+            return group == 128 ? unp_t<FMT_W3, 128>(N, K, w, out, ldo, f16, s)
+                                : unp_t<FMT_W3, 64>(N, K, w, out, ldo, f16, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
 template <int FMT, int GRP>
 static cudaError_t prep_t(int mode, int N, int K, const float* wf, const uint16_t* wb, const uint32_t* cq,
                           const uint16_t* cs, const uint32_t* cz, uint8_t* out, cudaStream_t s) {

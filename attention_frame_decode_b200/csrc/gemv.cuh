@@ -82,5 +82,8 @@ cudaError_t launch_pack_bf16(int N, int K, const uint16_t* w, uint8_t* out, cuda
 cudaError_t launch_pack_canonical(int fmt, int group, int N, int K, const uint32_t* q, const uint16_t* scales,
                                   const uint32_t* zeros, uint8_t* out, cudaStream_t s);
 cudaError_t launch_dequant(int fmt, int group, int N, int K, const uint8_t* w, float* out, cudaStream_t s);
+// dense 16-bit row-major copy [N][ldo] (bf16, or fp16 of the dequantized value when f16 = 1)
+cudaError_t launch_unpack16(int fmt, int group, int N, int K, const uint8_t* w, uint16_t* out, int ldo, int f16,
+                            cudaStream_t s);
 
 }  // namespace vc

@@ -1,10 +1,441 @@
-// prefill.cu -- opening-context prefill (placeholder until the chunked SSD path lands).
+// prefill.cu -- opening-context prefill of one session: all T frames layer by layer.
+//
+// "system-prompt prefill, then the user's speech" ("NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM,
+// MLX", "Recipe"): before streaming, the backbone consumes a context of T frames at once.  Per
+// layer:
+//   pre-RMSNorm rows (act = bf16(r * gamma), inv_rms per row)
+//   Mamba-2 : in_proj GEMM (tcgen05) -> causal conv1d + SiLU over the frames (the last W-1 raw
+//             rows go to the session's conv ring) -> chunked SSD (Dao & Gu, "Transformers are
+//             SSMs", the SSD algorithm: per chunk of Q = 256 frames the chunk state
+//             S_c = sum_j exp(Lam_end - Lam_j) dt_j x_j (outer) B_j, a scan over chunks
+//             S_in(c+1) = exp(Lam_end(c)) S_in(c) + S_c, and the outputs
+//             y_i = sum_{j<=i} (C_i.B_j) exp(Lam_i - Lam_j) dt_j x_j + exp(Lam_i) C_i.S_in + D x_i)
+//             -> gated RMSNorm -> out_proj GEMM + residual
+//   attention: qkv GEMM (k, v written to the KV cache rows 0..T-1) -> causal GQA softmax
+//             attention -> o_proj GEMM + residual
+//   MLP      : up GEMM with squared ReLU -> down GEMM + residual
+// The SSD and attention run on fp32 CUDA cores; the projections (>95% of the FLOPs) on tcgen05.
+// The call (re)initialises the slot: the SSM state ends as the scan's final state, the conv
+// ring holds the last W-1 frames, KV rows 0..T-1 are written and ctx_len[slot] = T.
+#include <string.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
 #include "prefill.cuh"
 
 namespace vc {
 
-size_t prefill_workspace_bytes(int, int, int, int, int, int, int, int, int, int, int, int, int) { return 256; }
+static constexpr int kChunk = 256;   // SSD chunk length (frames)
 
-cudaError_t run_prefill(const PrefillCtx&, const uint16_t*, int, int, cudaStream_t) { return cudaErrorNotSupported; }
+static size_t al(size_t v) { return (v + 255) / 256 * 256; }
+
+struct PfBufs {
+    float *r, *inv, *xc, *dt, *lam, *y, *schunk, *sin;
+    uint16_t *act_d, *act_big, *zx, *q, *wdense;
+    int ld_d, ld_big;
+};
+
+static PfBufs carve_pf(uint8_t* base, int T, int d, int E, int Cx, int H, int P, int N, int Hq, int Hk, int Dh,
+                       int F, size_t* total) {
+    PfBufs b{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base ? base + off : nullptr;
+        off += al(bytes);
+        return p;
+    };
+    const int nch = (T + kChunk - 1) / kChunk;
+    b.ld_d = (d + 127) / 128 * 128;
+    int big = std::max(std::max(E, F), Hq * Dh);
+    b.ld_big = (big + 127) / 128 * 128;
+    const int zxw = E + Cx + H;
+    b.r = (float*)take((size_t)T * d * 4);
+    b.inv = (float*)take((size_t)T * 4);
+    b.act_d = (uint16_t*)take((size_t)T * b.ld_d * 2);
+    b.act_big = (uint16_t*)take((size_t)T * b.ld_big * 2);
+    b.zx = (uint16_t*)take((size_t)T * std::max(zxw, 1) * 2);
+    b.q = (uint16_t*)take((size_t)T * std::max(Hq * Dh, 1) * 2);
+    b.xc = (float*)take((size_t)T * std::max(Cx, 1) * 4);
+    b.dt = (float*)take((size_t)T * std::max(H, 1) * 4);
+    b.lam = (float*)take((size_t)T * std::max(H, 1) * 4);
+    b.y = (float*)take((size_t)T * std::max(E, 1) * 4);
+    b.schunk = (float*)take((size_t)nch * std::max(H * P * N, 1) * 4);
+    b.sin = (float*)take((size_t)nch * std::max(H * P * N, 1) * 4);
+    // the largest linear weight of a layer, unpacked to 16-bit row-major for the GEMM
+    size_t wmax = std::max((size_t)zxw * d, (size_t)d * E);
+    wmax = std::max(wmax, (size_t)(Hq + 2 * Hk) * Dh * d);
+    wmax = std::max(wmax, (size_t)d * Hq * Dh);
+    wmax = std::max(wmax, (size_t)F * d);
+    b.wdense = (uint16_t*)take(wmax * 2);
+    if (total) *total = off;
+    return b;
+}
+
+size_t prefill_workspace_bytes(int d, int L, int E, int Cx, int H, int P, int N, int G, int Hq, int Hk, int Dh, int F,
+                               int cap) {
+    (void)L; (void)G;
+    size_t total = 0;
+    carve_pf(nullptr, cap, d, E, Cx, H, P, N, Hq, Hk, Dh, F, &total);
+    return total;
+}
+
+// ------------------------------------------------------------------------------------------
+// row kernels
+// ------------------------------------------------------------------------------------------
+// r = x (first layer) or r (later layers); act = bf16(r * gamma); inv = rsqrt(mean(r^2) + eps)
+__global__ void pf_rownorm_kernel(const uint16_t* x, float* r, const float* gamma, uint16_t* act, int ld, float* inv,
+                                  int d, float eps, int f16) {
+    const int t = blockIdx.x;
+    float* rr = r + (size_t)t * d;
+    float ss = 0.0f;
+    for (int k = threadIdx.x; k < d; k += blockDim.x) {
+        float v;
+        if (x) {
+            v = bf16_bits_to_f(x[(size_t)t * d + k]);
+            rr[k] = v;
+        } else {
+            v = rr[k];
+        }
+        ss += v * v;
+        act[(size_t)t * ld + k] = f16 ? act_bits<true>(v * gamma[k]) : act_bits<false>(v * gamma[k]);
+    }
+    __shared__ float red[32];
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s = 0.0f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += red[w];
+        inv[t] = rsqrtf(s / d + eps);
+    }
+}
+
+// causal depthwise conv1d + SiLU over the frames (zero history); dt = softplus(dt_raw + bias);
+// the last W-1 raw pre-conv rows are written to the conv ring (frame t in slot t mod W)
+__global__ void pf_conv_kernel(const uint16_t* zx, int zxw, int T, int E, int Cx, int H, int W, const float* conv_w,
+                               const float* conv_b, const float* dt_bias, float* xc, float* dt, uint16_t* ring) {
+    const int t = blockIdx.x;
+    const uint16_t* xBC = zx + E;
+    for (int c = threadIdx.x; c < Cx; c += blockDim.x) {
+        float acc = conv_b[c];
+        for (int k = 0; k < W; ++k) {
+            const int tt = t - (W - 1) + k;
+            if (tt >= 0) acc += conv_w[c * W + k] * bf16_bits_to_f(xBC[(size_t)tt * zxw + c]);
+        }
+        xc[(size_t)t * Cx + c] = silu_f(acc);
+        if (t >= T - (W - 1)) ring[(size_t)(t % W) * Cx + c] = xBC[(size_t)t * zxw + c];
+    }
+    for (int h = threadIdx.x; h < H; h += blockDim.x)
+        dt[(size_t)t * H + h] = softplus_f(bf16_bits_to_f(zx[(size_t)t * zxw + E + Cx + h]) + dt_bias[h]);
+}
+
+// ------------------------------------------------------------------------------------------
+// chunked SSD
+// ------------------------------------------------------------------------------------------
+// per (chunk, head): inclusive cumulative log decay Lam and the chunk state
+//   S_c[p][n] = sum_j exp(Lam_end - Lam_j) dt_j x_j[p] B_j[n]
+__global__ void __launch_bounds__(256) pf_ssd_state_kernel(const float* xc, const float* dt, const float* A_log, int T,
+                                                           int H, int P, int N, int G, int E, int Cx, float* lam,
+                                                           float* schunk) {
+    const int c = blockIdx.x, h = blockIdx.y;
+    const int t0 = c * kChunk, len = min(kChunk, T - t0);
+    const int g = (int)((long long)h * G / H);
+    __shared__ float w[kChunk];
+    __shared__ float lam_s[kChunk];
+    const float A = -expf(A_log[h]);
+    // inclusive scan of A*dt over the chunk (one warp)
+    if (threadIdx.x < 32) {
+        float run = 0.0f;
+        for (int base = 0; base < len; base += 32) {
+            const int i = base + threadIdx.x;
+            float v = i < len ? A * dt[(size_t)(t0 + i) * H + h] : 0.0f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, v, o);
+                if (threadIdx.x >= o) v += u;
+            }
+            v += run;
+            if (i < len) lam_s[i] = v;
+            run = __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    __syncthreads();
+    const float lend = lam_s[len - 1];
+    for (int i = threadIdx.x; i < len; i += blockDim.x) {
+        w[i] = expf(lend - lam_s[i]) * dt[(size_t)(t0 + i) * H + h];
+        lam[(size_t)(t0 + i) * H + h] = lam_s[i];
+    }
+    __syncthreads();
+    float* S = schunk + ((size_t)c * H + h) * P * N;
+    for (int idx = threadIdx.x; idx < P * N; idx += blockDim.x) {
+        const int p = idx / N, n = idx % N;
+        const float* xcol = xc + (size_t)t0 * Cx + h * P + p;
+        const float* bcol = xc + (size_t)t0 * Cx + E + g * N + n;
+        float acc = 0.0f;
+        for (int j = 0; j < len; ++j) acc = fmaf(w[j] * xcol[(size_t)j * Cx], bcol[(size_t)j * Cx], acc);
+        S[idx] = acc;
+    }
+}
+
+// scan over chunks: S_in(0) = 0, S_in(c+1) = exp(Lam_end(c)) S_in(c) + S_c; final -> ssm state
+__global__ void pf_ssd_scan_kernel(const float* schunk, const float* lam, int T, int H, int P, int N, float* sin,
+                                   float* ssm_out) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long per_head = (long long)P * N;
+    if (idx >= (long long)H * per_head) return;
+    const int h = (int)(idx / per_head);
+    const int nch = (T + kChunk - 1) / kChunk;
+    float s = 0.0f;
+    for (int c = 0; c < nch; ++c) {
+        sin[(size_t)c * H * per_head + idx] = s;
+        const int tend = min(T, (c + 1) * kChunk) - 1;
+        s = expf(lam[(size_t)tend * H + h]) * s + schunk[(size_t)c * H * per_head + idx];
+    }
+    ssm_out[idx] = s;
+}
+
+// outputs per (chunk, head, 64-row slice): y_i[p] = sum_{j<=i} (C_i.B_j) exp(Lam_i - Lam_j) dt_j x_j[p]
+//                                                 + exp(Lam_i) sum_n C_i[n] S_in[p][n] + D x_i[p]
+__global__ void __launch_bounds__(256) pf_ssd_out_kernel(const float* xc, const float* dt, const float* lam,
+                                                         const float* sin, const float* Dv, int T, int H, int P, int N,
+                                                         int G, int E, int Cx, float* y) {
+    const int c = blockIdx.x, h = blockIdx.y, slice = blockIdx.z;
+    const int t0 = c * kChunk, len = min(kChunk, T - t0);
+    const int i0 = slice * 64;
+    if (i0 >= len) return;
+    const int i1 = min(len, i0 + 64);
+    const int g = (int)((long long)h * G / H);
+    extern __shared__ float sm[];
+    float* cb = sm;                          // [64][i1] weights (C_i.B_j) exp(.) dt_j, j <= i
+    float* lam_s = cb + 64 * kChunk;         // [len]
+    float* dt_s = lam_s + kChunk;            // [len]
+    for (int i = threadIdx.x; i < i1; i += blockDim.x) {
+        lam_s[i] = lam[(size_t)(t0 + i) * H + h];
+        dt_s[i] = dt[(size_t)(t0 + i) * H + h];
+    }
+    __syncthreads();
+    // C_i . B_j for i in the slice, j <= i
+    for (int idx = threadIdx.x; idx < (i1 - i0) * i1; idx += blockDim.x) {
+        const int ii = idx / i1, j = idx % i1, i = i0 + ii;
+        float v = 0.0f;
+        if (j <= i) {
+            const float* Ci = xc + (size_t)(t0 + i) * Cx + E + G * N + g * N;
+            const float* Bj = xc + (size_t)(t0 + j) * Cx + E + g * N;
+            float acc = 0.0f;
+            for (int n = 0; n < N; ++n) acc = fmaf(Ci[n], Bj[n], acc);
+            v = acc * expf(lam_s[i] - lam_s[j]) * dt_s[j];
+        }
+        cb[ii * kChunk + j] = v;
+    }
+    __syncthreads();
+    const float* Sp = sin + ((size_t)c * H + h) * P * N;
+    for (int idx = threadIdx.x; idx < (i1 - i0) * P; idx += blockDim.x) {
+        const int ii = idx / P, p = idx % P, i = i0 + ii;
+        float acc = 0.0f;
+        for (int j = 0; j <= i; ++j) acc = fmaf(cb[ii * kChunk + j], xc[(size_t)(t0 + j) * Cx + h * P + p], acc);
+        const float* Ci = xc + (size_t)(t0 + i) * Cx + E + G * N + g * N;
+        float off = 0.0f;
+        for (int n = 0; n < N; ++n) off = fmaf(Ci[n], Sp[(size_t)p * N + n], off);
+        const float xv = xc[(size_t)(t0 + i) * Cx + h * P + p];
+        y[(size_t)(t0 + i) * E + h * P + p] = acc + expf(lam_s[i]) * off + Dv[h] * xv;
+    }
+}
+
+// v = y * silu(z); per row and norm group: act = bf16(v * rsqrt(mean(v^2) + eps) * gamma)
+__global__ void pf_gated_norm_kernel(const float* y, const uint16_t* zx, int zxw, const float* gnorm, int E, int NG,
+                                     float eps, uint16_t* act, int ld, int f16) {
+    const int t = blockIdx.x, q = blockIdx.y;
+    const int gs = E / NG, c0 = q * gs;
+    __shared__ float red[32];
+    float ss = 0.0f;
+    for (int c = c0 + threadIdx.x; c < c0 + gs; c += blockDim.x) {
+        const float v = y[(size_t)t * E + c] * silu_f(bf16_bits_to_f(zx[(size_t)t * zxw + c]));
+        ss += v * v;
+    }
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float s = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+        s = warp_sum(s);
+        if (threadIdx.x == 0) red[0] = rsqrtf(s / gs + eps);
+    }
+    __syncthreads();
+    const float ginv = red[0];
+    for (int c = c0 + threadIdx.x; c < c0 + gs; c += blockDim.x) {
+        const float v = y[(size_t)t * E + c] * silu_f(bf16_bits_to_f(zx[(size_t)t * zxw + c]));
+        const float u = v * ginv * gnorm[c];
+        act[(size_t)t * ld + c] = f16 ? act_bits<true>(u) : act_bits<false>(u);
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// causal GQA attention over the prefilled frames (fp32, online softmax), one warp per
+// (frame, query head); keys/values come from the KV cache rows just written
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) pf_attn_kernel(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int T,
+                                                      int Hq, int Hk, int Dh, int cap, uint16_t* out, int ld,
+                                                      int f16) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+    const int i = blockIdx.y;
+    if (t >= T) return;
+    const int j = (int)((long long)i * Hk / Hq);
+    const float scale = rsqrtf((float)Dh);
+    const int per = Dh / 32;   // dims per lane (Dh <= 256)
+    float qv[8], o[8];
+    for (int e = 0; e < per; ++e) {
+        qv[e] = bf16_bits_to_f(q[(size_t)t * Hq * Dh + (size_t)i * Dh + lane * per + e]) * scale;
+        o[e] = 0.0f;
+    }
+    const uint16_t* K = kc + (size_t)j * cap * Dh;
+    const uint16_t* V = vc + (size_t)j * cap * Dh;
+    float m = -INFINITY, l = 0.0f;
+    for (int tau = 0; tau <= t; ++tau) {
+        float s = 0.0f;
+        for (int e = 0; e < per; ++e) s = fmaf(qv[e], bf16_bits_to_f(K[(size_t)tau * Dh + lane * per + e]), s);
+        s = warp_sum(s);
+        const float mn = fmaxf(m, s);
+        const float corr = expf(m - mn), p = expf(s - mn);
+        l = l * corr + p;
+        for (int e = 0; e < per; ++e) o[e] = o[e] * corr + p * bf16_bits_to_f(V[(size_t)tau * Dh + lane * per + e]);
+        m = mn;
+    }
+    for (int e = 0; e < per; ++e) {
+        const float u = o[e] / l;
+        out[(size_t)t * ld + (size_t)i * Dh + lane * per + e] = f16 ? act_bits<true>(u) : act_bits<false>(u);
+    }
+}
+
+__global__ void pf_finish_kernel(int32_t* ctx_len, int slot, int T) { ctx_len[slot] = T; }
+
+// ------------------------------------------------------------------------------------------
+// Mamba-2 mixer over the frames (conv -> chunked SSD -> gated norm), shared by the prefill and
+// its kernel-level test entry
+// ------------------------------------------------------------------------------------------
+size_t prefill_mixer_scratch_bytes(int T, int E, int Cx, int H, int P, int N) {
+    const size_t nch = (size_t)(T + kChunk - 1) / kChunk;
+    return al((size_t)T * Cx * 4) + 2 * al((size_t)T * H * 4) + al((size_t)T * E * 4) + 2 * al(nch * H * P * N * 4);
+}
+
+void carve_mixer(PfMixer& m, uint8_t* base) {
+    const size_t nch = (size_t)(m.T + kChunk - 1) / kChunk;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base + off;
+        off += al(bytes);
+        return (float*)p;
+    };
+    m.xc = take((size_t)m.T * m.Cx * 4);
+    m.dt = take((size_t)m.T * m.H * 4);
+    m.lam = take((size_t)m.T * m.H * 4);
+    m.y = take((size_t)m.T * m.E * 4);
+    m.schunk = take(nch * m.H * m.P * m.N * 4);
+    m.sin = take(nch * m.H * m.P * m.N * 4);
+}
+
+cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
+    const int T = m.T, E = m.E, Cx = m.Cx, H = m.H, P = m.P, N = m.N, W = m.W;
+    const int zxw = E + Cx + H;
+    const int nch = (T + kChunk - 1) / kChunk;
+    const vc_layer_weights& Lw = *m.Lw;
+    const size_t osm = (size_t)(64 * kChunk + 2 * kChunk) * 4;
+    cudaError_t e = cudaFuncSetAttribute(pf_ssd_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)osm);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(m.ring, 0, (size_t)W * Cx * 2, s)) != cudaSuccess) return e;
+    pf_conv_kernel<<<T, 256, 0, s>>>(m.zx, zxw, T, E, Cx, H, W, Lw.conv_w, Lw.conv_b, Lw.dt_bias, m.xc, m.dt, m.ring);
+    pf_ssd_state_kernel<<<dim3(nch, H), 256, 0, s>>>(m.xc, m.dt, Lw.A_log, T, H, P, N, m.G, E, Cx, m.lam, m.schunk);
+    const long long n = (long long)H * P * N;
+    pf_ssd_scan_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(m.schunk, m.lam, T, H, P, N, m.sin, m.ssm);
+    pf_ssd_out_kernel<<<dim3(nch, H, kChunk / 64), 256, osm, s>>>(m.xc, m.dt, m.lam, m.sin, Lw.D, T, H, P, N, m.G, E,
+                                                                  Cx, m.y);
+    pf_gated_norm_kernel<<<dim3(T, m.NG), 256, 0, s>>>(m.y, m.zx, zxw, Lw.gnorm, E, m.NG, m.eps, m.act, m.act_ld,
+                                                       m.f16);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// orchestration
+// ------------------------------------------------------------------------------------------
+struct PfGemm {
+    const PrefillCtx& c;
+    const PfBufs& b;
+    int f16;
+    cudaStream_t s;
+    // unpack w to 16-bit row-major, then out = epilogue(A . w^T)
+    cudaError_t operator()(int epi, const uint16_t* A, int lda, int M, const vc_qmat& w, const float* row_scale,
+                           uint16_t* out, int ldo, float* out32, int ldo32, const GemmArgs* qkv = nullptr) const {
+        cudaError_t e = launch_unpack16(w.fmt, w.fmt == VC_W_BF16 ? 64 : w.group, w.N, w.K, (const uint8_t*)w.data,
+                                        b.wdense, w.K, f16, s);
+        if (e != cudaSuccess) return e;
+        GemmArgs a = qkv ? *qkv : GemmArgs{};
+        a.f16 = f16; a.out_f16 = f16;
+        a.A = A; a.lda = lda; a.M = M;
+        a.W = b.wdense; a.ldw = w.K; a.N = w.N; a.K = w.K;
+        a.row_scale = row_scale; a.out = out; a.ldo = ldo; a.out_f32 = out32; a.ldo32 = ldo32; a.status = c.status;
+        return launch_gemm_tc(epi, a, s);
+    }
+};
+
+cudaError_t run_prefill(const PrefillCtx& c, const uint16_t* x, int T, int slot, cudaStream_t s) {
+    const int d = c.d, E = c.E, Cx = c.Cx, H = c.H, P = c.P, N = c.N, W = c.W;
+    const int zxw = E + Cx + H;
+    if (T < 1 || T > c.cap) return cudaErrorInvalidValue;
+    if (strchr(c.cfg->pattern, '*') && (c.Dh % 32 || c.Dh > 256)) return cudaErrorNotSupported;
+    const PfBufs b = carve_pf(c.ws, T, d, E, Cx, H, P, N, c.Hq, c.Hk, c.Dh, c.F, nullptr);
+    const int f16 = c.cfg->wfmt != VC_W_BF16;   // quantized weights: fp16 operands, as in the decode GEMV
+    const PfGemm gemm{c, b, f16, s};
+    const float eps = c.cfg->eps;
+    cudaError_t e;
+    pf_rownorm_kernel<<<T, 256, 0, s>>>(x, b.r, c.layers[0].norm, b.act_d, b.ld_d, b.inv, d, eps, f16);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t rbytes = (size_t)T * d * 4;
+    if (c.tap && (e = cudaMemcpyAsync(c.tap, b.r, rbytes, cudaMemcpyDeviceToDevice, s)) != cudaSuccess) return e;
+    int mi = 0, ai = 0;
+    for (int l = 0; l < c.L; ++l) {
+        const vc_layer_weights& Lw = c.layers[l];
+        const char kind = c.cfg->pattern[l];
+        if (l > 0) {
+            pf_rownorm_kernel<<<T, 256, 0, s>>>(nullptr, b.r, Lw.norm, b.act_d, b.ld_d, b.inv, d, eps, f16);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        if (kind == 'M') {
+            PfMixer m{};
+            m.T = T; m.E = E; m.Cx = Cx; m.H = H; m.P = P; m.N = N; m.G = c.G; m.W = W; m.NG = c.NG;
+            m.eps = eps; m.f16 = f16; m.Lw = &Lw;
+            m.xc = b.xc; m.dt = b.dt; m.lam = b.lam; m.y = b.y; m.schunk = b.schunk; m.sin = b.sin;
+            m.ssm = c.ssm + ((size_t)mi * c.n_slots + slot) * H * P * N;
+            m.ring = c.conv + ((size_t)mi * c.n_slots + slot) * W * Cx;
+            m.act = b.act_big; m.act_ld = b.ld_big;
+            // the GEMM's GE_ROWSCALE outputs are the bf16 in_proj values (the decode path's zx)
+            if ((e = gemm(GE_ROWSCALE, b.act_d, b.ld_d, T, Lw.in_proj, b.inv, b.zx, zxw, nullptr, 0))) return e;
+            m.zx = b.zx;
+            if ((e = prefill_mixer(m, s))) return e;
+            if ((e = gemm(GE_RESID, b.act_big, b.ld_big, T, Lw.out_proj, nullptr, nullptr, 0, b.r, d))) return e;
+            mi++;
+        } else if (kind == '*') {
+            const size_t kvl = ((size_t)ai * c.n_slots + slot) * c.Hk * c.cap * c.Dh;
+            GemmArgs qa{};
+            qa.Hq = c.Hq; qa.Hk = c.Hk; qa.Dh = c.Dh; qa.cap = c.cap; qa.t0 = 0;
+            qa.kcache = c.k + kvl; qa.vcache = c.v + kvl;
+            if ((e = gemm(GE_QKV, b.act_d, b.ld_d, T, Lw.qkv, b.inv, b.q, c.Hq * c.Dh, nullptr, 0, &qa))) return e;
+            pf_attn_kernel<<<dim3((T + 7) / 8, c.Hq), 256, 0, s>>>(b.q, qa.kcache, qa.vcache, T, c.Hq, c.Hk, c.Dh, c.cap,
+                                                                   b.act_big, b.ld_big, f16);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            if ((e = gemm(GE_RESID, b.act_big, b.ld_big, T, Lw.o, nullptr, nullptr, 0, b.r, d))) return e;
+            ai++;
+        } else {
+            if ((e = gemm(GE_RELU2, b.act_d, b.ld_d, T, Lw.up, b.inv, b.act_big, b.ld_big, nullptr, 0))) return e;
+            if ((e = gemm(GE_RESID, b.act_big, b.ld_big, T, Lw.down, nullptr, nullptr, 0, b.r, d))) return e;
+        }
+        if (c.tap && (e = cudaMemcpyAsync(c.tap + (size_t)(l + 1) * T * d, b.r, rbytes, cudaMemcpyDeviceToDevice, s)))
+            return e;
+    }
+    pf_finish_kernel<<<1, 1, 0, s>>>(c.ctx_len, slot, T);
+    return cudaGetLastError();
+}
 
 }  // namespace vc

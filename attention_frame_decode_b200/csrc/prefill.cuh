@@ -19,7 +19,25 @@ struct PrefillCtx {
     uint16_t *conv, *k, *v;
     int32_t* ctx_len;
     int32_t* status;
+    float* tap;   // test tap or null: residual stream [L+1][T][d] (entry 0 = input, l+1 after layer l)
 };
+
+// Mamba-2 mixer of one layer over T frames from zero state: conv (ring written), chunked SSD
+// (final state written to ssm), y (before gating) and the gated-norm output act
+struct PfMixer {
+    int T, E, Cx, H, P, N, G, W, NG, f16;
+    float eps;
+    const vc_layer_weights* Lw;
+    const uint16_t* zx;                              // bf16 [T][E+Cx+H]
+    float *xc, *dt, *lam, *y, *schunk, *sin;         // scratch (carve_mixer); y fp32 [T][E]
+    float* ssm;                                      // [H][P][N]
+    uint16_t* ring;                                  // [W][Cx]
+    uint16_t* act;                                   // [T][act_ld]
+    int act_ld;
+};
+size_t prefill_mixer_scratch_bytes(int T, int E, int Cx, int H, int P, int N);
+void carve_mixer(PfMixer& m, uint8_t* base);
+cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s);
 
 size_t prefill_workspace_bytes(int d, int L, int E, int Cx, int H, int P, int N, int G, int Hq, int Hk, int Dh, int F,
                                int cap);

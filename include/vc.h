@@ -189,6 +189,11 @@ vc_status vc_prefill(vc_backbone* h, const void* x, int T, int slot, const vc_st
  * logits [2][B][max(vocab_text, vocab_func)] (text, function). */
 vc_status vc_debug_set_taps(vc_backbone* h, float* hidden, float* logits);
 
+/* test/debug tap for the next vc_prefill calls (device fp32 buffer or NULL): hidden
+ * [n_layers+1][T][d], the residual stream of every prefilled frame after each layer (entry 0 =
+ * input), for the T of that call; the caller sizes it. */
+vc_status vc_debug_set_prefill_taps(vc_backbone* h, float* hidden);
+
 /* test/debug: one Mamba-2 mixer step (the kernel vc_step runs for a Mamba-2 layer) on given
  * inputs.  zx: bf16 [B][E+Cx+H] in_proj outputs; ssm/conv: this layer's state slices
  * ([n_slots][H][P][N] fp32, [n_slots][W][Cx] bf16); slots [B] or NULL; ctx_len [n_slots] is read,
@@ -206,6 +211,25 @@ vc_status vc_debug_mamba_step(const vc_config* cfg, const vc_layer_weights* laye
 size_t vc_gemv_scratch_bytes(void);
 vc_status vc_debug_gemv(const vc_qmat* w, const void* act, int act_ld, int B, float* out, void* scratch,
                         vc_stream_t stream);
+
+/* test: the prefill's Mamba-2 mixer of one layer over T frames of one session that starts empty
+ * (the kernels vc_prefill runs between a Mamba-2 layer's two projections): causal conv + SiLU,
+ * chunked SSD with chunks of 256 frames, gated RMSNorm.
+ * zx: bf16 [T][E+Cx+H] in_proj outputs (device).  Outputs (device): ssm fp32 [H][P][N] final state,
+ * conv bf16 [W][Cx] ring (frame t in slot t mod W, the other slots zero), y fp32 [T][E] the SSM
+ * output before gating, act bf16 [T][E] = bf16(y*silu(z) * rsqrt(mean over the norm group + eps)
+ * * gnorm).  scratch: device, vc_debug_mamba_prefill_scratch_bytes(cfg, T) bytes, 16-byte aligned. */
+size_t vc_debug_mamba_prefill_scratch_bytes(const vc_config* cfg, int T);
+vc_status vc_debug_mamba_prefill(const vc_config* cfg, const vc_layer_weights* layer, const void* zx, int T, float* ssm,
+                                 void* conv, float* y, void* act, void* scratch, vc_stream_t stream);
+
+/* test/measurement: out = A . W^T with the prefill's tensor-core GEMM (tcgen05, fp32 accumulation
+ * in tensor memory), the contraction of the prefill projections over the frames.
+ * A: [M][lda] and W: [N][ldw] 16-bit row-major (device, 16-byte aligned; bf16 bits, or fp16 bits
+ * when f16 != 0), K a multiple of 8, lda and ldw multiples of 8 and >= K.  out: fp32 [M][ldo]
+ * (device).  status: device word; VC_DEV_TIMEOUT is or-ed in if an internal wait ran out. */
+vc_status vc_debug_gemm(const void* A, int lda, int M, const void* W, int ldw, int N, int K, int f16, float* out,
+                        int ldo, int32_t* status, vc_stream_t stream);
 
 void vc_destroy(vc_backbone* h);
 
