@@ -74,6 +74,9 @@ _lib.vc_debug_mamba_step.argtypes = [C.POINTER(VcConfig), C.POINTER(VcLayerWeigh
 _lib.vc_gemv_scratch_bytes.argtypes = []
 _lib.vc_gemv_scratch_bytes.restype = C.c_size_t
 _lib.vc_debug_gemv.argtypes = [C.POINTER(VcQmat), _p, _i, _i, _p, _p, _p]
+_lib.vc_gemv_noalloc_scratch_bytes.argtypes = []
+_lib.vc_gemv_noalloc_scratch_bytes.restype = C.c_size_t
+_lib.vc_debug_gemv_noalloc.argtypes = [C.POINTER(VcQmat), _p, _i, _i, _p, _p]
 _lib.vc_debug_gemm.argtypes = [_p, _i, _i, _p, _i, _i, _i, _i, _p, _i, _p, _p]
 _lib.vc_debug_mamba_prefill_scratch_bytes.argtypes = [C.POINTER(VcConfig), _i]
 _lib.vc_debug_mamba_prefill_scratch_bytes.restype = C.c_size_t
@@ -88,13 +91,13 @@ _lib.vc_last_cuda_error.restype = C.c_char_p
 for _f in ("vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant", "vc_backbone_create",
            "vc_set_option", "vc_step", "vc_step_host", "vc_prefill", "vc_debug_set_taps", "vc_debug_set_prefill_taps",
            "vc_debug_mamba_step",
-           "vc_debug_gemv", "vc_debug_gemm", "vc_debug_mamba_prefill"):
+           "vc_debug_gemv", "vc_debug_gemm", "vc_debug_mamba_prefill", "vc_debug_gemv_noalloc"):
     getattr(_lib, _f).restype = _i
 
 EXPORTS = ("vc_weight_bytes", "vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant",
            "vc_workspace_bytes", "vc_backbone_create", "vc_set_option", "vc_step", "vc_step_host", "vc_prefill",
            "vc_debug_set_taps", "vc_debug_set_prefill_taps", "vc_debug_mamba_step", "vc_gemv_scratch_bytes",
-           "vc_debug_gemv", "vc_debug_gemm",
+           "vc_debug_gemv", "vc_debug_gemm", "vc_gemv_noalloc_scratch_bytes", "vc_debug_gemv_noalloc",
            "vc_debug_mamba_prefill_scratch_bytes", "vc_debug_mamba_prefill", "vc_destroy",
            "vc_status_string", "vc_last_cuda_error")
 
@@ -215,6 +218,19 @@ def debug_gemv(wbuf, fmt, group, N, K, act, scratch, out=None, stream=None):
     m = qmat(wbuf, fmt, group, N, K)
     _check(_lib.vc_debug_gemv(C.byref(m), _ptr(act), act_ld, B, _ptr(out), _ptr(scratch), _stream(stream)),
            "vc_debug_gemv")
+    return out
+
+
+def debug_gemv_noalloc(wbuf, fmt, group, N, K, act, out=None, stream=None):
+    """as debug_gemv, with the library's static scratch (no scratch argument, nothing allocated
+    by the library)"""
+    import torch
+    B, act_ld = act.shape
+    if out is None:
+        out = torch.empty((B, N), dtype=torch.float32, device=act.device)
+    m = qmat(wbuf, fmt, group, N, K)
+    _check(_lib.vc_debug_gemv_noalloc(C.byref(m), _ptr(act), act_ld, B, _ptr(out), _stream(stream)),
+           "vc_debug_gemv_noalloc")
     return out
 
 

@@ -25,6 +25,11 @@ static vc_status cuda_fail(cudaError_t e, const char* where) {
     snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", where, cudaGetErrorString(e));
     return VC_ERR_CUDA;
 }
+namespace vc {
+// error recording for the C ABI functions defined in other translation units
+vc_status record_cuda_failure(cudaError_t e, const char* where) { return cuda_fail(e, where); }
+}  // namespace vc
+
 #define CK(call)                                         \
     do {                                                 \
         cudaError_t e_ = (call);                         \

@@ -231,6 +231,22 @@ vc_status vc_debug_mamba_prefill(const vc_config* cfg, const vc_layer_weights* l
 vc_status vc_debug_gemm(const void* A, int lda, int M, const void* W, int ldw, int N, int K, int f16, float* out,
                         int ldo, int32_t* status, vc_stream_t stream);
 
+/* The GEMV of vc_debug_gemv for callers that cannot allocate device memory (a per-frame
+ * real-time loop, where cudaMalloc/cudaFree can synchronize the device and stall the frame; a
+ * host whose device memory belongs to another allocator).  No counterpart in the method's
+ * sources: an operational variant of the decode GEMV, nothing the model computes differs.
+ * Same arguments, results and validation as vc_debug_gemv, without the scratch argument: the
+ * scratch is a static device array of vc_gemv_noalloc_scratch_bytes() = 4.25 MiB in the
+ * library (4 MiB of partial sums, 65536 arrival counters that are zero at load and that every
+ * call leaves zero), and the launch uses at most 32 SMs' worth of CTAs.  A weight with more than
+ * 65536 row units (16*R rows each) returns VC_ERR_CAPACITY.  The first call on a device looks
+ * up the array's device address for that device; make it before any stream capture begins.
+ * All calls on a device share the array: calls that overlap in time race and give wrong
+ * results, so callers order them.  Allocates nothing. */
+size_t vc_gemv_noalloc_scratch_bytes(void);
+vc_status vc_debug_gemv_noalloc(const vc_qmat* w, const void* act, int act_ld, int B, float* out,
+                                vc_stream_t stream);
+
 void vc_destroy(vc_backbone* h);
 
 const char* vc_status_string(vc_status s);
