@@ -89,7 +89,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __shared__ uint32_t tmem_base;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+    // M-tile fastest: the CTAs resident at one time share a few W column tiles (each streamed
+    // from HBM once) while the activation rows, re-read per W tile, stay in L2
+    const int mt = (a.M + BM - 1) / BM;
+    const int n0 = (int)(blockIdx.x / mt) * BN, m0 = (int)(blockIdx.x % mt) * BM;
     const int KB = (a.K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
@@ -245,7 +248,7 @@ static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mw, const 
     auto kern = gemm_tc_kernel<EPI, F16>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM);
+    dim3 grid((unsigned)(((a.N + BN - 1) / BN) * ((a.M + BM - 1) / BM)));
     kern<<<grid, GEMM_THREADS, smem, s>>>(ma, mw, a);
     return cudaGetLastError();
 }

@@ -24,6 +24,7 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "prefill_mma.cuh"
 #include "prefill.cuh"
 
 namespace vc {
@@ -137,14 +138,23 @@ __global__ void pf_conv_kernel(const uint16_t* zx, int zxw, int T, int E, int Cx
 // ------------------------------------------------------------------------------------------
 // per (chunk, head): inclusive cumulative log decay Lam and the chunk state
 //   S_c[p][n] = sum_j exp(Lam_end - Lam_j) dt_j x_j[p] B_j[n]
-__global__ void __launch_bounds__(256) pf_ssd_state_kernel(const float* xc, const float* dt, const float* A_log, int T,
-                                                           int H, int P, int N, int G, int E, int Cx, float* lam,
-                                                           float* schunk) {
+// in fp32 (the state the decode steps continue from), frames staged 32 at a time in shared
+// memory; a 16 x 16 thread grid, each thread RP x RN outputs (p = pg + 16 r, n = ng + 16 q)
+static constexpr int kStJ = 32;
+
+template <int RP, int RN>
+__global__ void __launch_bounds__(256) pf_ssd_state_kernel(const float* __restrict__ xc, const float* __restrict__ dt,
+                                                           const float* __restrict__ A_log, int T, int H, int P, int N,
+                                                           int G, int E, int Cx, float* __restrict__ lam,
+                                                           float* __restrict__ schunk) {
     const int c = blockIdx.x, h = blockIdx.y;
     const int t0 = c * kChunk, len = min(kChunk, T - t0);
     const int g = (int)((long long)h * G / H);
     __shared__ float w[kChunk];
     __shared__ float lam_s[kChunk];
+    extern __shared__ float stage[];   // xw [kStJ][P], bs [kStJ][N]
+    float* xw = stage;
+    float* bs = stage + kStJ * P;
     const float A = -expf(A_log[h]);
     // inclusive scan of A*dt over the chunk (one warp)
     if (threadIdx.x < 32) {
@@ -155,7 +165,7 @@ __global__ void __launch_bounds__(256) pf_ssd_state_kernel(const float* xc, cons
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float u = __shfl_up_sync(0xffffffffu, v, o);
-                if (threadIdx.x >= o) v += u;
+                if ((int)threadIdx.x >= o) v += u;
             }
             v += run;
             if (i < len) lam_s[i] = v;
@@ -168,16 +178,47 @@ __global__ void __launch_bounds__(256) pf_ssd_state_kernel(const float* xc, cons
         w[i] = expf(lend - lam_s[i]) * dt[(size_t)(t0 + i) * H + h];
         lam[(size_t)(t0 + i) * H + h] = lam_s[i];
     }
-    __syncthreads();
-    float* S = schunk + ((size_t)c * H + h) * P * N;
-    for (int idx = threadIdx.x; idx < P * N; idx += blockDim.x) {
-        const int p = idx / N, n = idx % N;
-        const float* xcol = xc + (size_t)t0 * Cx + h * P + p;
-        const float* bcol = xc + (size_t)t0 * Cx + E + g * N + n;
-        float acc = 0.0f;
-        for (int j = 0; j < len; ++j) acc = fmaf(w[j] * xcol[(size_t)j * Cx], bcol[(size_t)j * Cx], acc);
-        S[idx] = acc;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ng = lane & 15, pg = warp * 2 + (lane >> 4);
+    float acc[RP][RN];
+#pragma unroll
+    for (int r = 0; r < RP; ++r)
+#pragma unroll
+        for (int q = 0; q < RN; ++q) acc[r][q] = 0.0f;
+    const float* xh = xc + (size_t)t0 * Cx + (size_t)h * P;
+    const float* bg = xc + (size_t)t0 * Cx + E + (size_t)g * N;
+    for (int jb = 0; jb < len; jb += kStJ) {
+        const int nj = min(kStJ, len - jb);
+        __syncthreads();   // w ready (first pass) / previous stage consumed
+        for (int idx = threadIdx.x; idx < nj * P; idx += blockDim.x) {
+            const int j = idx / P, p = idx - j * P;
+            xw[j * P + p] = w[jb + j] * xh[(size_t)(jb + j) * Cx + p];
+        }
+        for (int idx = threadIdx.x; idx < nj * N; idx += blockDim.x) {
+            const int j = idx / N, n = idx - j * N;
+            bs[j * N + n] = bg[(size_t)(jb + j) * Cx + n];
+        }
+        __syncthreads();
+        for (int j = 0; j < nj; ++j) {
+            float xv[RP], bv[RN];
+#pragma unroll
+            for (int r = 0; r < RP; ++r) xv[r] = pg + 16 * r < P ? xw[j * P + pg + 16 * r] : 0.0f;
+#pragma unroll
+            for (int q = 0; q < RN; ++q) bv[q] = ng + 16 * q < N ? bs[j * N + ng + 16 * q] : 0.0f;
+#pragma unroll
+            for (int r = 0; r < RP; ++r)
+#pragma unroll
+                for (int q = 0; q < RN; ++q) acc[r][q] = fmaf(xv[r], bv[q], acc[r][q]);
+        }
     }
+    float* S = schunk + ((size_t)c * H + h) * P * N;
+#pragma unroll
+    for (int r = 0; r < RP; ++r)
+#pragma unroll
+        for (int q = 0; q < RN; ++q) {
+            const int p = pg + 16 * r, n = ng + 16 * q;
+            if (p < P && n < N) S[(size_t)p * N + n] = acc[r][q];
+        }
 }
 
 // scan over chunks: S_in(0) = 0, S_in(c+1) = exp(Lam_end(c)) S_in(c) + S_c; final -> ssm state
@@ -195,53 +236,6 @@ __global__ void pf_ssd_scan_kernel(const float* schunk, const float* lam, int T,
         s = expf(lam[(size_t)tend * H + h]) * s + schunk[(size_t)c * H * per_head + idx];
     }
     ssm_out[idx] = s;
-}
-
-// outputs per (chunk, head, 64-row slice): y_i[p] = sum_{j<=i} (C_i.B_j) exp(Lam_i - Lam_j) dt_j x_j[p]
-//                                                 + exp(Lam_i) sum_n C_i[n] S_in[p][n] + D x_i[p]
-__global__ void __launch_bounds__(256) pf_ssd_out_kernel(const float* xc, const float* dt, const float* lam,
-                                                         const float* sin, const float* Dv, int T, int H, int P, int N,
-                                                         int G, int E, int Cx, float* y) {
-    const int c = blockIdx.x, h = blockIdx.y, slice = blockIdx.z;
-    const int t0 = c * kChunk, len = min(kChunk, T - t0);
-    const int i0 = slice * 64;
-    if (i0 >= len) return;
-    const int i1 = min(len, i0 + 64);
-    const int g = (int)((long long)h * G / H);
-    extern __shared__ float sm[];
-    float* cb = sm;                          // [64][i1] weights (C_i.B_j) exp(.) dt_j, j <= i
-    float* lam_s = cb + 64 * kChunk;         // [len]
-    float* dt_s = lam_s + kChunk;            // [len]
-    for (int i = threadIdx.x; i < i1; i += blockDim.x) {
-        lam_s[i] = lam[(size_t)(t0 + i) * H + h];
-        dt_s[i] = dt[(size_t)(t0 + i) * H + h];
-    }
-    __syncthreads();
-    // C_i . B_j for i in the slice, j <= i
-    for (int idx = threadIdx.x; idx < (i1 - i0) * i1; idx += blockDim.x) {
-        const int ii = idx / i1, j = idx % i1, i = i0 + ii;
-        float v = 0.0f;
-        if (j <= i) {
-            const float* Ci = xc + (size_t)(t0 + i) * Cx + E + G * N + g * N;
-            const float* Bj = xc + (size_t)(t0 + j) * Cx + E + g * N;
-            float acc = 0.0f;
-            for (int n = 0; n < N; ++n) acc = fmaf(Ci[n], Bj[n], acc);
-            v = acc * expf(lam_s[i] - lam_s[j]) * dt_s[j];
-        }
-        cb[ii * kChunk + j] = v;
-    }
-    __syncthreads();
-    const float* Sp = sin + ((size_t)c * H + h) * P * N;
-    for (int idx = threadIdx.x; idx < (i1 - i0) * P; idx += blockDim.x) {
-        const int ii = idx / P, p = idx % P, i = i0 + ii;
-        float acc = 0.0f;
-        for (int j = 0; j <= i; ++j) acc = fmaf(cb[ii * kChunk + j], xc[(size_t)(t0 + j) * Cx + h * P + p], acc);
-        const float* Ci = xc + (size_t)(t0 + i) * Cx + E + G * N + g * N;
-        float off = 0.0f;
-        for (int n = 0; n < N; ++n) off = fmaf(Ci[n], Sp[(size_t)p * N + n], off);
-        const float xv = xc[(size_t)(t0 + i) * Cx + h * P + p];
-        y[(size_t)(t0 + i) * E + h * P + p] = acc + expf(lam_s[i]) * off + Dv[h] * xv;
-    }
 }
 
 // v = y * silu(z); per row and norm group: act = bf16(v * rsqrt(mean(v^2) + eps) * gamma)
@@ -273,10 +267,11 @@ __global__ void pf_gated_norm_kernel(const float* y, const uint16_t* zx, int zxw
 }
 
 // ------------------------------------------------------------------------------------------
-// causal GQA attention over the prefilled frames (fp32, online softmax), one warp per
-// (frame, query head); keys/values come from the KV cache rows just written
+// causal GQA attention for head dimensions without a tensor-core instance (multiples of 32 up
+// to 256): fp32, online softmax, one warp per (frame, query head) over the KV cache rows just
+// written
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) pf_attn_kernel(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int T,
+__global__ void __launch_bounds__(256) pf_attn_scalar_kernel(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int T,
                                                       int Hq, int Hk, int Dh, int cap, uint16_t* out, int ld,
                                                       int f16) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -342,16 +337,29 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
     const int zxw = E + Cx + H;
     const int nch = (T + kChunk - 1) / kChunk;
     const vc_layer_weights& Lw = *m.Lw;
-    const size_t osm = (size_t)(64 * kChunk + 2 * kChunk) * 4;
-    cudaError_t e = cudaFuncSetAttribute(pf_ssd_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)osm);
+    if (P % 8 || P > 128 || N % 16 || N > 256 || H % m.G) return cudaErrorNotSupported;
+    const SsdLayout SL = ssd_layout(N, P);
+    if (SL.total > 227 * 1024) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(pf_ssd_out_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SL.total);
     if (e != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(m.ring, 0, (size_t)W * Cx * 2, s)) != cudaSuccess) return e;
     pf_conv_kernel<<<T, 256, 0, s>>>(m.zx, zxw, T, E, Cx, H, W, Lw.conv_w, Lw.conv_b, Lw.dt_bias, m.xc, m.dt, m.ring);
-    pf_ssd_state_kernel<<<dim3(nch, H), 256, 0, s>>>(m.xc, m.dt, Lw.A_log, T, H, P, N, m.G, E, Cx, m.lam, m.schunk);
+    const size_t st_smem = (size_t)kStJ * (P + N) * 4;
+    const dim3 sg(nch, H);
+    if (P <= 80 && P > 64 && N <= 128 && N > 112)
+        pf_ssd_state_kernel<5, 8><<<sg, 256, st_smem, s>>>(m.xc, m.dt, Lw.A_log, T, H, P, N, m.G, E, Cx, m.lam,
+                                                             m.schunk);
+    else if (P <= 32 && N <= 16)
+        pf_ssd_state_kernel<2, 1><<<sg, 256, st_smem, s>>>(m.xc, m.dt, Lw.A_log, T, H, P, N, m.G, E, Cx, m.lam,
+                                                             m.schunk);
+    else
+        pf_ssd_state_kernel<8, 16><<<sg, 256, st_smem, s>>>(m.xc, m.dt, Lw.A_log, T, H, P, N, m.G, E, Cx, m.lam,
+                                                              m.schunk);
     const long long n = (long long)H * P * N;
     pf_ssd_scan_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(m.schunk, m.lam, T, H, P, N, m.sin, m.ssm);
-    pf_ssd_out_kernel<<<dim3(nch, H, kChunk / 64), 256, osm, s>>>(m.xc, m.dt, m.lam, m.sin, Lw.D, T, H, P, N, m.G, E,
-                                                                  Cx, m.y);
+    pf_ssd_out_mma_kernel<<<dim3(nch, m.G, kChunk / kSsdTi), 256, SL.total, s>>>(m.xc, m.dt, m.lam, m.sin, Lw.D, T, H,
+                                                                                 P, N, m.G, E, Cx, m.y);
     pf_gated_norm_kernel<<<dim3(T, m.NG), 256, 0, s>>>(m.y, m.zx, zxw, Lw.gnorm, E, m.NG, m.eps, m.act, m.act_ld,
                                                        m.f16);
     return cudaGetLastError();
@@ -422,8 +430,15 @@ cudaError_t run_prefill(const PrefillCtx& c, const uint16_t* x, int T, int slot,
             qa.Hq = c.Hq; qa.Hk = c.Hk; qa.Dh = c.Dh; qa.cap = c.cap; qa.t0 = 0;
             qa.kcache = c.k + kvl; qa.vcache = c.v + kvl;
             if ((e = gemm(GE_QKV, b.act_d, b.ld_d, T, Lw.qkv, b.inv, b.q, c.Hq * c.Dh, nullptr, 0, &qa))) return e;
-            pf_attn_kernel<<<dim3((T + 7) / 8, c.Hq), 256, 0, s>>>(b.q, qa.kcache, qa.vcache, T, c.Hq, c.Hk, c.Dh, c.cap,
-                                                                   b.act_big, b.ld_big, f16);
+            if (c.Dh == 128)
+                pf_flash_kernel<128><<<dim3((T + 63) / 64, c.Hq), 128, 0, s>>>(b.q, qa.kcache, qa.vcache, T, c.Hq, c.Hk,
+                                                                               c.cap, b.act_big, b.ld_big, f16);
+            else if (c.Dh == 64)
+                pf_flash_kernel<64><<<dim3((T + 63) / 64, c.Hq), 128, 0, s>>>(b.q, qa.kcache, qa.vcache, T, c.Hq, c.Hk,
+                                                                              c.cap, b.act_big, b.ld_big, f16);
+            else
+                pf_attn_scalar_kernel<<<dim3((T + 7) / 8, c.Hq), 256, 0, s>>>(b.q, qa.kcache, qa.vcache, T, c.Hq, c.Hk,
+                                                                              c.Dh, c.cap, b.act_big, b.ld_big, f16);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             if ((e = gemm(GE_RESID, b.act_big, b.ld_big, T, Lw.o, nullptr, nullptr, 0, b.r, d))) return e;
             ai++;

@@ -1,0 +1,406 @@
+// prefill_mma.cuh -- the chunk contractions of the prefill on warp-level tensor-core MMA
+// (mma.sync m16n8k16, 16-bit operands, fp32 accumulation): the chunked SSD outputs and causal
+// flash attention.  Together they are ~2.5% of the prefill's FLOPs (the projections, on tcgen05,
+// are the rest), on tiles whose head dimensions (P = 80, Dh = 128) are small, so register-fragment
+// MMA with shared-memory staging keeps them off the critical path without a TMEM pipeline.
+//
+// Fragment layouts of m16n8k16 (g = lane / 4, t = lane % 4):
+//   A 16x16 row-major: a0 = A[g][2t..2t+1], a1 = A[g+8][2t..], a2 = A[g][2t+8..], a3 = A[g+8][2t+8..]
+//   B 16x8  (k x n):   b0 = B[2t..2t+1][g], b1 = B[2t+8..2t+9][g]
+//   C 16x8:            c0 = C[g][2t], c1 = C[g][2t+1], c2 = C[g+8][2t], c3 = C[g+8][2t+1]
+// Shared-memory rows are padded so the 8 rows a fragment load touches fall in distinct banks.
+#pragma once
+#include "common.cuh"
+
+namespace vc {
+
+VC_DEV uint32_t lds32(const uint16_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
+VC_DEV uint16_t bf16_bits(float v) {
+    __nv_bfloat16 b = __float2bfloat16_rn(v);
+    return *reinterpret_cast<uint16_t*>(&b);
+}
+
+VC_DEV uint32_t pack_bf16x2(float lo, float hi) { return (uint32_t)bf16_bits(lo) | ((uint32_t)bf16_bits(hi) << 16); }
+
+// fp16 bits, saturated to the finite range
+VC_DEV uint16_t f16_bits(float v) {
+    __half h = __float2half_rn(fminf(fmaxf(v, -65504.0f), 65504.0f));
+    return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// ------------------------------------------------------------------------------------------
+// chunked SSD, outputs.  CTA = (chunk c, B/C group g, 64-row tile of the chunk).  The group's
+// C.B^T block (64 x j) is computed once and reused by the H/G heads of the group.  The
+// intra-chunk products take fp16 operands (C, B, the decay-weighted C.B^T and x: 11-bit
+// significands; y is heavy-tailed, and bf16's 8 bits leave its largest elements ~10% of the
+// RMS off), the entering-state product bf16 operands (the state's range):
+//   y_i[p] = sum_{j<=i} (C_i.B_j) exp(Lam_i - Lam_j) dt_j x_j[p]      (intra-chunk, W . X)
+//          + exp(Lam_i) sum_n C_i[n] S_in[p][n]                        (state entering the chunk)
+//          + D x_i[p]
+// ------------------------------------------------------------------------------------------
+static constexpr int kSsdChunk = 256;
+static constexpr int kSsdTi = 64;
+
+struct SsdLayout {
+    int sc, sb, scb, sw, ss, sx;               // row strides (elements)
+    size_t off_c, off_c2, off_b, off_w, off_s, off_cb, off_x, off_l, total;
+};
+
+__host__ __device__ inline SsdLayout ssd_layout(int N, int P) {
+    SsdLayout L{};
+    L.sc = N + 8;
+    L.sb = N + 8;
+    L.scb = kSsdChunk + 4;
+    L.sw = kSsdChunk + 8;
+    L.ss = N + 8;
+    L.sx = kSsdChunk + 8;
+    auto a16 = [](size_t v) { return (v + 15) / 16 * 16; };
+    const size_t rc = a16((size_t)kSsdTi * L.sc * 2);
+    const size_t rb_b = (size_t)kSsdChunk * L.sb * 2;
+    const size_t rw = a16((size_t)kSsdTi * L.sw * 2);
+    const size_t rs = a16((size_t)P * L.ss * 2);
+    const size_t rb = a16(rb_b > rw + rs ? rb_b : rw + rs);   // B is dead once C.B^T is formed
+    L.off_c = 0;
+    L.off_c2 = rc;
+    L.off_b = 2 * rc;
+    L.off_w = 2 * rc;
+    L.off_s = 2 * rc + rw;
+    L.off_cb = 2 * rc + rb;
+    L.off_x = L.off_cb + a16((size_t)kSsdTi * L.scb * 4);
+    L.off_l = L.off_x + a16((size_t)P * L.sx * 2);
+    L.total = L.off_l + 2 * kSsdChunk * 4;
+    return L;
+}
+
+__global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __restrict__ xc, const float* __restrict__ dt,
+                                                             const float* __restrict__ lam,
+                                                             const float* __restrict__ sin, const float* __restrict__ Dv,
+                                                             int T, int H, int P, int N, int G, int E, int Cx,
+                                                             float* __restrict__ y) {
+    extern __shared__ __align__(16) unsigned char smraw[];
+    const int c = blockIdx.x, g = blockIdx.y, it = blockIdx.z;
+    const int t0 = c * kSsdChunk, len = min(kSsdChunk, T - t0);
+    const int i0 = it * kSsdTi;
+    if (i0 >= len) return;
+    const int i1 = min(len, i0 + kSsdTi);
+    const int jn = i1;                       // frames j < jn are visible to some row of the tile
+    const int jn16 = (jn + 15) & ~15;
+    const int jn32 = (jn + 31) & ~31;
+    const SsdLayout L = ssd_layout(N, P);
+    uint16_t* Cs = reinterpret_cast<uint16_t*>(smraw + L.off_c);     // C rows, fp16
+    uint16_t* Cb = reinterpret_cast<uint16_t*>(smraw + L.off_c2);    // C rows, bf16
+    uint16_t* Bs = reinterpret_cast<uint16_t*>(smraw + L.off_b);
+    uint16_t* Ws = reinterpret_cast<uint16_t*>(smraw + L.off_w);
+    uint16_t* Sb = reinterpret_cast<uint16_t*>(smraw + L.off_s);
+    float* CBs = reinterpret_cast<float*>(smraw + L.off_cb);
+    uint16_t* Xt = reinterpret_cast<uint16_t*>(smraw + L.off_x);
+    float* lam_s = reinterpret_cast<float*>(smraw + L.off_l);
+    float* dts = lam_s + kSsdChunk;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    const float* Cg = xc + (size_t)t0 * Cx + E + (size_t)G * N + (size_t)g * N;
+    const float* Bg = xc + (size_t)t0 * Cx + E + (size_t)g * N;
+
+    // 1. the group's C rows of the tile (fp16 and bf16) and B rows 0..jn-1 (fp16), zero padded
+    for (int idx = tid; idx < kSsdTi * N; idx += blockDim.x) {
+        const int ii = idx / N, n = idx - ii * N;
+        const float v = i0 + ii < i1 ? Cg[(size_t)(i0 + ii) * Cx + n] : 0.0f;
+        Cs[ii * L.sc + n] = f16_bits(v);
+        Cb[ii * L.sc + n] = bf16_bits(v);
+    }
+    for (int idx = tid; idx < jn32 * N; idx += blockDim.x) {
+        const int j = idx / N, n = idx - j * N;
+        Bs[j * L.sb + n] = f16_bits(j < jn ? Bg[(size_t)j * Cx + n] : 0.0f);
+    }
+    __syncthreads();
+
+    // 2. CB[ii][j] = C_i . B_j: warp w forms columns 32w .. 32w+31 of all 64 rows
+    if (32 * warp < jn) {
+        float acc[4][4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[a][b][e] = 0.0f;
+        for (int k0 = 0; k0 < N; k0 += 16) {
+            uint32_t af[4][4];
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) {
+                const uint16_t* r = Cs + (mt * 16 + gq) * L.sc + k0 + 2 * tq;
+                af[mt][0] = lds32(r);
+                af[mt][1] = lds32(r + 8 * L.sc);
+                af[mt][2] = lds32(r + 8);
+                af[mt][3] = lds32(r + 8 * L.sc + 8);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const uint16_t* r = Bs + (32 * warp + nt * 8 + gq) * L.sb + k0 + 2 * tq;
+                const uint32_t b0 = lds32(r), b1 = lds32(r + 8);
+#pragma unroll
+                for (int mt = 0; mt < 4; ++mt) mma_f16(acc[mt][nt], af[mt], b0, b1, acc[mt][nt]);
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                float* r = CBs + (mt * 16 + gq) * L.scb + 32 * warp + nt * 8 + 2 * tq;
+                *reinterpret_cast<float2*>(r) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+                *reinterpret_cast<float2*>(r + 8 * L.scb) = make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+            }
+    }
+    __syncthreads();
+
+    // 3. the heads of the group
+    const int hpg = H / G;
+    const int nt8 = P / 8;
+    const int wm = warp & 3, wn = warp >> 2;
+    const int half = (nt8 + 1) / 2;
+    const int q0 = wn * half;
+    const int qn = min(nt8, q0 + half) - q0;
+    const int kend = min(jn16, i0 + wm * 16 + 16);   // rows of this warp see j < i0 + 16 (wm + 1)
+    for (int hh = 0; hh < hpg; ++hh) {
+        const int h = g * hpg + hh;
+        for (int j = tid; j < jn16; j += blockDim.x) {
+            lam_s[j] = j < jn ? lam[(size_t)(t0 + j) * H + h] : 0.0f;
+            dts[j] = j < jn ? dt[(size_t)(t0 + j) * H + h] : 0.0f;
+        }
+        const float* xh = xc + (size_t)t0 * Cx + (size_t)h * P;
+        for (int idx = tid; idx < jn16 * P; idx += blockDim.x) {
+            const int j = idx / P, p = idx - j * P;
+            Xt[p * L.sx + j] = f16_bits(j < jn ? xh[(size_t)j * Cx + p] : 0.0f);
+        }
+        const float* Sh = sin + ((size_t)c * H + h) * P * N;
+        for (int idx = tid; idx < P * N; idx += blockDim.x) {
+            const int p = idx / N, n = idx - p * N;
+            Sb[p * L.ss + n] = bf16_bits(Sh[idx]);
+        }
+        __syncthreads();
+        for (int idx = tid; idx < kSsdTi * jn16; idx += blockDim.x) {
+            const int ii = idx / jn16, j = idx - ii * jn16;
+            const int i = i0 + ii;
+            float v = 0.0f;
+            if (i < i1 && j <= i) v = CBs[ii * L.scb + j] * __expf(lam_s[i] - lam_s[j]) * dts[j];
+            Ws[ii * L.sw + j] = f16_bits(v);
+        }
+        __syncthreads();
+        float acc[8][4], acc2[8][4];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[q][e] = acc2[q][e] = 0.0f;
+        for (int k0 = 0; k0 < kend; k0 += 16) {
+            uint32_t af[4];
+            const uint16_t* r = Ws + (wm * 16 + gq) * L.sw + k0 + 2 * tq;
+            af[0] = lds32(r);
+            af[1] = lds32(r + 8 * L.sw);
+            af[2] = lds32(r + 8);
+            af[3] = lds32(r + 8 * L.sw + 8);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < qn) {
+                    const uint16_t* br = Xt + ((q0 + q) * 8 + gq) * L.sx + k0 + 2 * tq;
+                    mma_f16(acc[q], af, lds32(br), lds32(br + 8), acc[q]);
+                }
+        }
+        for (int k0 = 0; k0 < N; k0 += 16) {
+            uint32_t af[4];
+            const uint16_t* r = Cb + (wm * 16 + gq) * L.sc + k0 + 2 * tq;
+            af[0] = lds32(r);
+            af[1] = lds32(r + 8 * L.sc);
+            af[2] = lds32(r + 8);
+            af[3] = lds32(r + 8 * L.sc + 8);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < qn) {
+                    const uint16_t* br = Sb + ((q0 + q) * 8 + gq) * L.ss + k0 + 2 * tq;
+                    mma_bf16(acc2[q], af, lds32(br), lds32(br + 8), acc2[q]);
+                }
+        }
+        const float Dh_ = Dv[h];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int i = i0 + wm * 16 + gq + 8 * r;
+            if (i < i1) {
+                const float el = __expf(lam_s[i]);
+                const float* xi = xh + (size_t)i * Cx;
+                float* yi = y + (size_t)(t0 + i) * E + (size_t)h * P;
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (q < qn) {
+                        const int p = (q0 + q) * 8 + 2 * tq;
+                        const float2 xv = *reinterpret_cast<const float2*>(xi + p);
+                        float2 o;
+                        o.x = acc[q][2 * r] + el * acc2[q][2 * r] + Dh_ * xv.x;
+                        o.y = acc[q][2 * r + 1] + el * acc2[q][2 * r + 1] + Dh_ * xv.y;
+                        *reinterpret_cast<float2*>(yi + p) = o;
+                    }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// causal GQA attention (flash form): CTA = (64 query frames, q head), 4 warps of 16 rows; keys
+// and values in tiles of 64 frames from the KV cache rows the qkv projection just wrote; online
+// softmax in fp32 (exp2 with the 1/sqrt(Dh) scale folded in), P rounded to bf16 for P.V.
+// q head i reads KV head floor(i Hk / Hq); no positional encoding.
+// ------------------------------------------------------------------------------------------
+VC_DEV void ldsm_x4_trans(uint32_t (&r)[4], const uint16_t* p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+
+template <int DH>
+__global__ void __launch_bounds__(128) pf_flash_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
+                                                       const uint16_t* __restrict__ vc, int T, int Hq, int Hk, int cap,
+                                                       uint16_t* __restrict__ out, int ld, int f16) {
+    constexpr int SK = DH + 8;
+    __shared__ __align__(16) uint16_t Ks[64 * SK];
+    __shared__ __align__(16) uint16_t Vs[64 * SK];
+    const int nqt = (T + 63) / 64;
+    const int qt = nqt - 1 - (int)blockIdx.x;   // the longest rows first
+    const int hq = blockIdx.y;
+    const int hk = (int)((long long)hq * Hk / Hq);
+    const int r0 = qt * 64;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    const uint16_t* K = kc + (size_t)hk * cap * DH;
+    const uint16_t* V = vc + (size_t)hk * cap * DH;
+    const int qld = Hq * DH;
+
+    uint32_t qa[DH / 16][4];
+    {
+        const int ra = r0 + warp * 16 + gq, rb = ra + 8;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+            const int col = hq * DH + kk * 16 + 2 * tq;
+            qa[kk][0] = ra < T ? lds32(q + (size_t)ra * qld + col) : 0u;
+            qa[kk][1] = rb < T ? lds32(q + (size_t)rb * qld + col) : 0u;
+            qa[kk][2] = ra < T ? lds32(q + (size_t)ra * qld + col + 8) : 0u;
+            qa[kk][3] = rb < T ? lds32(q + (size_t)rb * qld + col + 8) : 0u;
+        }
+    }
+    float o[DH / 8][4];
+#pragma unroll
+    for (int d = 0; d < DH / 8; ++d)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[d][e] = 0.0f;
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
+    const float sl2 = rsqrtf((float)DH) * 1.4426950408889634f;
+    const int row[2] = {r0 + warp * 16 + gq, r0 + warp * 16 + gq + 8};
+
+    for (int kt = 0; kt <= qt; ++kt) {
+        const int key0 = kt * 64;
+        __syncthreads();
+        for (int idx = tid; idx < 64 * DH / 8; idx += blockDim.x) {
+            const int key = idx / (DH / 8), c8 = idx - key * (DH / 8);
+            uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+            if (key0 + key < T) {
+                kv = *reinterpret_cast<const uint4*>(K + (size_t)(key0 + key) * DH + c8 * 8);
+                vv = *reinterpret_cast<const uint4*>(V + (size_t)(key0 + key) * DH + c8 * 8);
+            }
+            *reinterpret_cast<uint4*>(Ks + key * SK + c8 * 8) = kv;
+            *reinterpret_cast<uint4*>(Vs + key * SK + c8 * 8) = vv;
+        }
+        __syncthreads();
+        float s[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[nt][e] = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const uint16_t* br = Ks + (nt * 8 + gq) * SK + kk * 16 + 2 * tq;
+                mma_bf16(s[nt], qa[kk], lds32(br), lds32(br + 8), s[nt]);
+            }
+        // causal mask (keys beyond the row or beyond T) and the running max of each row
+        const bool diag = kt == qt;
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int key = key0 + nt * 8 + 2 * tq + (e & 1);
+                const int r = e >> 1;
+                if ((diag && key > row[r]) || key >= T) s[nt][e] = -INFINITY;
+                mx[r] = fmaxf(mx[r], s[nt][e]);
+            }
+        float corr[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+            const float mn = fmaxf(m[r], mx[r]);
+            corr[r] = m[r] == -INFINITY ? 0.0f : exp2f((m[r] - mn) * sl2);
+            m[r] = mn;
+        }
+        float ls[2] = {0.0f, 0.0f};
+        uint32_t pa[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = e >> 1;
+                p[e] = s[nt][e] == -INFINITY ? 0.0f : exp2f((s[nt][e] - m[r]) * sl2);
+                ls[r] += p[e];
+            }
+            // C fragment of key tile nt -> A fragment (keys 16 kb .. 16 kb + 15) of P . V
+            const int kb = nt >> 1;
+            if ((nt & 1) == 0) {
+                pa[kb][0] = pack_bf16x2(p[0], p[1]);
+                pa[kb][1] = pack_bf16x2(p[2], p[3]);
+            } else {
+                pa[kb][2] = pack_bf16x2(p[0], p[1]);
+                pa[kb][3] = pack_bf16x2(p[2], p[3]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) l[r] = l[r] * corr[r] + ls[r];
+#pragma unroll
+        for (int d = 0; d < DH / 8; ++d) {
+            o[d][0] *= corr[0];
+            o[d][1] *= corr[0];
+            o[d][2] *= corr[1];
+            o[d][3] *= corr[1];
+        }
+        // O += P . V; V fragments by transposing 8x8 loads: lanes 0-7 keys 0-7, 8-15 keys 8-15
+        // (dims d0..d0+7), 16-23 and 24-31 the same keys at dims d0+8..d0+15
+        const int lk = (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int ld8 = 8 * (lane >> 4);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+            for (int d = 0; d < DH / 8; d += 2) {
+                uint32_t vb[4];
+                ldsm_x4_trans(vb, Vs + (kb * 16 + lk) * SK + d * 8 + ld8);
+                mma_bf16(o[d], pa[kb], vb[0], vb[1], o[d]);
+                mma_bf16(o[d + 1], pa[kb], vb[2], vb[3], o[d + 1]);
+            }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        if (row[r] >= T) continue;
+        const float inv = 1.0f / l[r];
+        uint16_t* orow = out + (size_t)row[r] * ld + (size_t)hq * DH;
+#pragma unroll
+        for (int d = 0; d < DH / 8; ++d) {
+            const float u0 = o[d][2 * r] * inv, u1 = o[d][2 * r + 1] * inv;
+            const uint32_t w = f16 ? ((uint32_t)act_bits<true>(u0) | ((uint32_t)act_bits<true>(u1) << 16))
+                                   : ((uint32_t)act_bits<false>(u0) | ((uint32_t)act_bits<false>(u1) << 16));
+            *reinterpret_cast<uint32_t*>(orow + d * 8 + 2 * tq) = w;
+        }
+    }
+}
+
+}  // namespace vc

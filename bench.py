@@ -6,7 +6,8 @@ Default workload: the Nemotron-Nano-9B-v2-shaped backbone with bf16 weights, bat
 state decode at a context of 2000 frames (KV cache and SSM state pre-filled from N(0,1)),
 synthetic seeded weights N(0, 0.02) and inputs N(0, 1).  One "step" is one frame through all
 56 layers and both vocabulary heads.  Other workloads: --config nano_w4 | nano_w3 |
-nano_w8_b16 | tiny_w8 (see synth.CONFIGS).
+nano_w8_b16 | tiny_w8 (see synth.CONFIGS), and nano_prefill: one step is then one prefill of the
+4096-frame opening context (tensor-core GEMMs, chunked SSD, causal attention).
 
 With N > 1 (torchrun) every rank serves its own independent sessions with a full replica of
 the weights (no collective on the data path); the reported value is the sum over ranks of
@@ -151,6 +152,19 @@ def cpu_threads():
 def run_reference(args, cfg, rank):
     if rank != 0:
         return
+    if cfg.prefill_T:
+        Ts = 16
+        value, dt = prefill_oracle_rate(cfg, Ts)
+        sample = f"prefill of the first {Ts} frames of the {cfg.prefill_T}-frame context per timed run"
+        line = {"impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "frames/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * dt,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": cfg.name, "frames": cfg.prefill_T, "batch": 1},
+                "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cpu_threads(), "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
     n = max(1, min(args.steps, 2 if cfg.d_model > 1000 else 64))
     for _ in range(max(0, min(args.warmup, 1))):
         pass
@@ -164,6 +178,151 @@ def run_reference(args, cfg, rank):
                              "sample": sample},
             "e2e": {"value": value, "unit": "frame-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# prefill workload (--config nano_prefill): one step = one vc_prefill of the opening context
+# ------------------------------------------------------------------------------------------------
+
+PREFILL_METRIC = "prefill frames/s & ms per opening context (T frames, batch 1); tensor-pipe TFLOP/s"
+
+
+def prefill_flops(cfg, T):
+    """algorithmic FLOPs of one prefill of T frames: the projections (2 T N K each), the causal
+    attention (QK^T and PV over the T(T+1)/2 visible pairs per q head) and the chunked SSD
+    (intra-chunk C.B^T and its product with x, chunk states, off-diagonal readout), chunk 256."""
+    proj = sum(2.0 * T * N * K for l in range(cfg.n_layers) for _, N, K in synth.linear_shapes(cfg, l))
+    attn = cfg.n_attn * cfg.attn_q_heads * 2 * 2.0 * cfg.attn_head_dim * T * (T + 1) / 2
+    Q = 256
+    H, P, N, G = cfg.ssm_heads, cfg.ssm_head_dim, cfg.ssm_state, cfg.ssm_groups
+    nch = (T + Q - 1) // Q
+    per_chunk = (G * 2.0 * Q * Q * N / 2       # C.B^T, lower triangle, per group
+                 + H * 2.0 * Q * Q * P / 2     # weighted sum over j <= i, per head
+                 + H * 2.0 * Q * P * N         # chunk state
+                 + H * 2.0 * Q * P * N)        # off-diagonal readout C.S_in
+    ssd = cfg.n_mamba * nch * per_chunk
+    return proj, attn, ssd
+
+
+def prefill_oracle_rate(cfg, T, seed=0):
+    import oracle
+    model = oracle.Model(cfg, seed)
+    st = model.new_state(1, max(T, 1) + 8)
+    x = synth.prefill_inputs(cfg, seed, T)
+    t0 = time.perf_counter()
+    model.prefill(st, 0, x, oracle.MIRROR, ssd_chunk=256)
+    dt = time.perf_counter() - t0
+    return T / dt, dt
+
+
+def run_prefill_bench(args, cfg, world, rank, local):
+    import torch
+    import torch.distributed as dist
+    import attention_frame_decode_b200 as vc
+    from attention_frame_decode_b200.synthetic import build_model
+    T = cfg.prefill_T
+    seed = 0
+    dm = build_model(cfg, seed)
+    cap = cfg.kv_capacity
+    bb = dm.backbone(1, cap, 1)
+    st = dm.new_state(1, cap)
+    x = torch.from_numpy(synth.prefill_inputs(cfg, seed + 1000 * rank, T)).cuda().view(torch.bfloat16)
+    for _ in range(args.warmup):
+        bb.prefill(x, 0, st)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        bb.prefill(x, 0, st)
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * T * args.steps / (ms / 1000.0)
+    proj, attn, ssd = prefill_flops(cfg, T)
+    step_tflops = (proj + attn + ssd) / (ms_step / 1000.0) / 1e12
+
+    # ---- roofline of the dominant kernel: the tcgen05 GEMM on the MLP up projection shape ----
+    pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
+    peak = float(pk["bf16_tflops"]) if pk else 1590.0
+    M, N, K = T, cfg.mlp_hidden, cfg.d_model
+    A = torch.randn((M, K), device="cuda").to(torch.bfloat16)
+    W = (0.02 * torch.randn((N, K), device="cuda")).to(torch.bfloat16)
+    out = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        vc.debug_gemm(A, W, status, out=out)
+    reps = 20
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    g0.record()
+    for _ in range(reps):
+        vc.debug_gemm(A, W, status, out=out)
+    g1.record()
+    torch.cuda.synchronize()
+    gemm_ms = g0.elapsed_time(g1) / reps
+    gemm_tf = 2.0 * M * N * K / (gemm_ms / 1000.0) / 1e12
+
+    # ---- end to end: the context from pinned host memory, the slot's ctx_len back to the host ----
+    xh = torch.from_numpy(synth.prefill_inputs(cfg, seed + 1000 * rank, T)).view(torch.bfloat16).pin_memory()
+    ch = torch.empty((1,), dtype=torch.int32).pin_memory()
+    xd = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    ne = max(2, min(args.steps, 10))
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(ne):
+        xd.copy_(xh, non_blocking=True)
+        bb.prefill(xd, 0, st)
+        ch.copy_(st.ctx_len[:1], non_blocking=True)
+        stream.synchronize()
+    e2e_s = time.perf_counter() - t0
+    assert int(ch[0]) == T
+    e2e_value = world * T * ne / e2e_s
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        Ts = 16
+        v, dt = prefill_oracle_rate(cfg, Ts)
+        cpu = {"value": v, "unit": "frames/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"prefill of the first {Ts} frames of the same context on the same model, {dt:.1f} s"}
+    if rank == 0:
+        n_launch = 2 + sum({"M": 9, "*": 5, "-": 5}[k] for k in cfg.pattern)
+        line = {
+            "metric": PREFILL_METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16-operands/fp32-accum", "data": "synthetic (seeded)",
+            "config": {"workload": cfg.name, "frames": T, "batch": 1, "layers": cfg.n_layers, "ssd_chunk": 256,
+                       "l2": "no flush: 15.4 GB of weights per prefill >> 126 MB L2",
+                       "parallelism": f"replicas x{world}"},
+            "step_tflops": step_tflops, "flops_per_step": {"projections": proj, "attention": attn, "ssd": ssd},
+            "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMM (MLP up projection shape)", "achieved": gemm_tf,
+                         "peak": peak, "peak_kind": "measured burst" if pk else "fallback", "unit": "TFLOP/s",
+                         "frac": gemm_tf / peak, "traffic": None, "launch_ms": gemm_ms,
+                         "flops_per_launch": 2.0 * M * N * K},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "frames/s", "h2d_bytes_per_step": T * cfg.d_model * 2,
+                    "d2h_bytes_per_step": 4, "steps": ne},
+            "gpu_launches": n_launch * args.steps, "clocks": clk, "device_status": int(st.status.cpu()[0]),
+        }
+        print(json.dumps(line), flush=True)
+    bb.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 # ------------------------------------------------------------------------------------------------
@@ -197,6 +356,10 @@ def main():
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+
+    if cfg.prefill_T:
+        run_prefill_bench(args, cfg, world, rank, local)
+        return
 
     import attention_frame_decode_b200 as vc
     from attention_frame_decode_b200.synthetic import build_model, fill_state

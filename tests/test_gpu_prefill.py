@@ -3,9 +3,12 @@ fp64 references and the CPU oracle, on the same seeded inputs.
 
 Tolerances:
   * tensor-core GEMM, fp32 accumulation of 16-bit products: max |gpu - fp64| <= 1e-4 * RMS(fp64);
-  * Mamba-2 mixer over the frames on identical bf16 inputs (conv + chunked SSD, fp32):
-    final SSM state and y within 1e-4 * RMS of the oracle's sequential recurrence, conv ring
-    bit-exact, gated-norm output within one bf16 ulp of the exact value;
+  * Mamba-2 mixer over the frames on identical bf16 inputs: final SSM state (fp32 chunk states
+    and scan) within 1e-4 * RMS of the oracle's sequential recurrence; y (intra-chunk products
+    on fp16, entering-state products on bf16 tensor-core operands) within one bf16 ulp of each
+    element plus 2e-2 * RMS; conv ring
+    bit-exact; gated-norm output within one bf16 ulp of the value exact arithmetic gives from
+    the kernel's own y;
   * whole stacks: state after the prefill (SSM per head, conv rows, KV rows) and the hidden
     states / logits of the decode steps that follow within max(2e-2, 2 x floor) * RMS, floor the
     oracle's own response to 1-ulp flips in ~1% of the prefill inputs (for the bf16-stored conv
@@ -42,12 +45,12 @@ def rel_heads(a, b):
     return float(np.max(np.max(np.abs(a - b), axis=1) / rms))
 
 
-def rel_stored(a, b):
+def rel_stored(a, b, ulp=2.0 ** -7):
     """as rel, for values both sides store in bf16: a rounding decision that went the other way
     (one bf16 ulp, at most 2^-7 of the value) is not counted"""
     a = np.asarray(a, np.float64)
     b = np.asarray(b, np.float64)
-    excess = np.maximum(np.abs(a - b) - 2.0 ** -7 * np.abs(b), 0.0)
+    excess = np.maximum(np.abs(a - b) - ulp * np.abs(b), 0.0)
     return float(np.max(excess) / max(np.sqrt(np.mean(b * b)), 1e-30))
 
 
@@ -151,7 +154,11 @@ def test_mamba_prefill_mixer(cuda, T, tiny):
     hist = np.zeros((W - 1, Cx), np.float64)
     yo, vo = om.mamba_mixer(0, synth.bf16_to_f32(zx_bits).astype(np.float64), S, hist, 0)
     assert rel(ssm.cpu().numpy(), S) < SSM_TOL
-    assert rel(y.cpu().numpy(), yo) < SSM_TOL
+    # y: the intra-chunk products run on fp16 tensor-core operands, the entering-state product on
+    # bf16 ones.  y feeds a bf16 storage point (the gated-norm output), so each element may be off
+    # by one bf16 ulp of itself (2^-8) on top of the 2e-2 * RMS bound; y is heavy-tailed (max/RMS
+    # ~ 27 here), and bf16 operands would exceed this bound where fp16 ones stay well inside it.
+    assert rel_stored(y.cpu().numpy(), yo, ulp=2.0 ** -8) < HID_TOL
     ring = conv.view(torch.int16).cpu().numpy().view(np.uint16)
     got_hist = ring_to_history(ring, T, W)
     want_hist = np.zeros((W - 1, Cx), np.uint16)
@@ -161,10 +168,11 @@ def test_mamba_prefill_mixer(cuda, T, tiny):
             want_hist[i] = zx_bits[t, E:E + Cx]
     assert np.array_equal(got_hist, want_hist)
     assert np.all(ring[T % W] == 0)
-    # gated RMSNorm output: one bf16 rounding of the exact value (within one bf16 ulp of it,
-    # 2^-8 relative, plus the fp32 arithmetic before the rounding)
+    # gated RMSNorm output from the kernel's own y: one bf16 rounding of the exact value (within
+    # one bf16 ulp of it, 2^-8 relative, plus the fp32 arithmetic before the rounding)
     gs = E // cfg.norm_groups
-    v = vo.reshape(T, cfg.norm_groups, gs)
+    z = synth.bf16_to_f32(zx_bits[:, :E]).astype(np.float64)
+    v = (y.cpu().numpy().astype(np.float64) * (z / (1.0 + np.exp(-z)))).reshape(T, cfg.norm_groups, gs)
     inv = 1.0 / np.sqrt((v * v).mean(axis=2, keepdims=True) + cfg.eps)
     ref = (v * inv).reshape(T, E) * small["gnorm"].astype(np.float64)
     got = act.float().cpu().numpy().astype(np.float64)
