@@ -338,6 +338,9 @@ def main():
     ap.add_argument("--impl", default="vc", choices=["vc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch each step's kernels directly instead of replaying a CUDA graph (for profilers "
+                         "that cannot replay graph kernel nodes with programmatic dependencies)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     cfg = synth.CONFIGS[args.config]
@@ -369,6 +372,8 @@ def main():
     dm = build_model(cfg, seed)
     cap = cfg.kv_capacity
     bb = dm.backbone(B, cap, B)
+    if args.no_graph:
+        bb.set_option(vc.OPT_GRAPH, 0)
     st = dm.new_state(B, cap)
     ctx0 = synth.context_lengths(cfg, seed, B)
     if cfg.random_state:
@@ -482,7 +487,7 @@ def main():
                        [int(ctx0.min()), int(ctx0.max())], "layers": cfg.n_layers, "weights": synth.FMT_NAMES[cfg.wfmt],
                        "group": cfg.group_size, "heads": synth.FMT_NAMES[cfg.head_fmt],
                        "l2": f"no flush: {weight_total / 1e9:.2f} GB of weights per step >> 126 MB L2",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}", "launch": "direct" if args.no_graph else "cuda graph"},
             "achieved_step_gbs": step_gbs, "step_bytes_read": rbytes, "step_bytes_written": wbytes,
             "step_frac_of_peak": step_gbs / peak,
             "roofline": {"bound": "hbm", "kernel": "gemv (mlp up projection, streaming weights)",

@@ -177,11 +177,15 @@ vc_status vc_step(vc_backbone* h, const void* x, int B, const int32_t* slots, co
 vc_status vc_step_host(vc_backbone* h, const void* x_host, int B, const int32_t* slots, const vc_state* state,
                        int32_t* tok_text_host, int32_t* tok_func_host, vc_stream_t stream);
 
-/* Prefill of T frames x bf16 [T][d_model] (device) into session `slot`, which must be empty
- * (ctx_len[slot] == 0, checked on the device: a non-empty slot sets VC_DEV_CAPACITY and the
- * call writes nothing).  Mamba-2 layers run the chunked SSD scan (chunk 256) over the frames,
- * attention layers causal GQA; the call writes the final SSM state, conv ring and KV[0..T) of
- * the slot and sets ctx_len[slot] = T.  No tokens are produced.  T <= kv_capacity. */
+/* Prefill of T frames x bf16 [T][d_model] (device) into session `slot` -- the opening context a
+ * streaming session consumes before its frames ("NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM,
+ * MLX", Recipe: system-prompt prefill, then the user's speech).  The slot starts empty: whatever
+ * it held is overwritten.  Mamba-2 layers run the chunked SSD (Dao & Gu, "Transformers are SSMs",
+ * chunk 256) over the frames, attention layers causal GQA; the call writes the final SSM state,
+ * the conv ring (the last W-1 frames' rows, frame t in slot t mod W, the other slot zero) and
+ * KV rows 0..T-1 of the slot and sets ctx_len[slot] = T.  No tokens are produced.
+ * 1 <= T <= kv_capacity (else VC_ERR_CAPACITY / VC_ERR_INVALID_ARG, nothing launched).  Uses the
+ * backbone's workspace (prefill scratch sized for kv_capacity frames); asynchronous on stream. */
 vc_status vc_prefill(vc_backbone* h, const void* x, int T, int slot, const vc_state* state, vc_stream_t stream);
 
 /* test/debug taps for the next vc_step calls (device fp32 buffers or NULL):
