@@ -142,6 +142,8 @@ struct vc_backbone {
     };
     std::map<GraphKey, Graph> graphs;
     cudaStream_t capture_stream = nullptr;
+    cudaStream_t prefill_side = nullptr;   // unpacks the next layer weight while a GEMM runs
+    cudaEvent_t pf_ev[5] = {};              // unpacked[2], gemm done[2], call start
 };
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -297,6 +299,8 @@ extern "C" vc_status vc_backbone_create(const vc_config* cfg, const vc_weights* 
     carve(h, (uint8_t*)workspace);
     cudaError_t e = cudaMemsetAsync(workspace, 0, vc_workspace_bytes(cfg), (cudaStream_t)stream);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->capture_stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->prefill_side, cudaStreamNonBlocking);
+    for (int i = 0; i < 5 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&h->pf_ev[i], cudaEventDisableTiming);
     if (e != cudaSuccess) {
         delete h;
         return cuda_fail(e, "vc_backbone_create");
@@ -567,6 +571,8 @@ extern "C" vc_status vc_prefill(vc_backbone* h, const void* x, int T, int slot, 
     c.ssm = state->ssm; c.conv = (uint16_t*)state->conv; c.k = (uint16_t*)state->k; c.v = (uint16_t*)state->v;
     c.ctx_len = state->ctx_len; c.status = state->status;
     c.tap = h->tap_prefill;
+    c.side = h->prefill_side;
+    for (int i = 0; i < 5; ++i) c.ev[i] = h->pf_ev[i];
     cudaError_t e = run_prefill(c, (const uint16_t*)x, T, slot, (cudaStream_t)stream);
     if (e == cudaErrorNotSupported) return VC_ERR_UNSUPPORTED;
     if (e == cudaErrorInvalidValue) return VC_ERR_INVALID_ARG;
@@ -670,6 +676,9 @@ extern "C" void vc_destroy(vc_backbone* h) {
     if (!h) return;
     clear_graphs(h);
     if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
+    if (h->prefill_side) cudaStreamDestroy(h->prefill_side);
+    for (int i = 0; i < 5; ++i)
+        if (h->pf_ev[i]) cudaEventDestroy(h->pf_ev[i]);
     delete h;
 }
 

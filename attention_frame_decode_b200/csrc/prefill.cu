@@ -20,6 +20,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <vector>
 
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -34,8 +35,9 @@ static constexpr int kChunk = 256;   // SSD chunk length (frames)
 static size_t al(size_t v) { return (v + 255) / 256 * 256; }
 
 struct PfBufs {
-    float *r, *inv, *xc, *dt, *lam, *y, *schunk, *sin;
-    uint16_t *act_d, *act_big, *zx, *q, *wdense;
+    float *r, *inv, *xc, *dt, *lam, *y, *schunk;
+    uint16_t *act_d, *act_big, *zx, *q, *xc16, *sin16;
+    uint16_t* wdense[2];   // double buffer: the GEMM reads one while the next weight is unpacked
     int ld_d, ld_big;
 };
 
@@ -64,13 +66,15 @@ static PfBufs carve_pf(uint8_t* base, int T, int d, int E, int Cx, int H, int P,
     b.lam = (float*)take((size_t)T * std::max(H, 1) * 4);
     b.y = (float*)take((size_t)T * std::max(E, 1) * 4);
     b.schunk = (float*)take((size_t)nch * std::max(H * P * N, 1) * 4);
-    b.sin = (float*)take((size_t)nch * std::max(H * P * N, 1) * 4);
+    b.sin16 = (uint16_t*)take((size_t)nch * std::max(H * P * N, 1) * 2);
+    b.xc16 = (uint16_t*)take((size_t)T * std::max(Cx, 1) * 2);
     // the largest linear weight of a layer, unpacked to 16-bit row-major for the GEMM
     size_t wmax = std::max((size_t)zxw * d, (size_t)d * E);
     wmax = std::max(wmax, (size_t)(Hq + 2 * Hk) * Dh * d);
     wmax = std::max(wmax, (size_t)d * Hq * Dh);
     wmax = std::max(wmax, (size_t)F * d);
-    b.wdense = (uint16_t*)take(wmax * 2);
+    b.wdense[0] = (uint16_t*)take(wmax * 2);
+    b.wdense[1] = (uint16_t*)take(wmax * 2);
     if (total) *total = off;
     return b;
 }
@@ -117,7 +121,8 @@ __global__ void pf_rownorm_kernel(const uint16_t* x, float* r, const float* gamm
 // causal depthwise conv1d + SiLU over the frames (zero history); dt = softplus(dt_raw + bias);
 // the last W-1 raw pre-conv rows are written to the conv ring (frame t in slot t mod W)
 __global__ void pf_conv_kernel(const uint16_t* zx, int zxw, int T, int E, int Cx, int H, int W, const float* conv_w,
-                               const float* conv_b, const float* dt_bias, float* xc, float* dt, uint16_t* ring) {
+                               const float* conv_b, const float* dt_bias, float* xc, uint16_t* xc16, float* dt,
+                               uint16_t* ring) {
     const int t = blockIdx.x;
     const uint16_t* xBC = zx + E;
     for (int c = threadIdx.x; c < Cx; c += blockDim.x) {
@@ -126,7 +131,9 @@ __global__ void pf_conv_kernel(const uint16_t* zx, int zxw, int T, int E, int Cx
             const int tt = t - (W - 1) + k;
             if (tt >= 0) acc += conv_w[c * W + k] * bf16_bits_to_f(xBC[(size_t)tt * zxw + c]);
         }
-        xc[(size_t)t * Cx + c] = silu_f(acc);
+        const float v = silu_f(acc);
+        xc[(size_t)t * Cx + c] = v;
+        xc16[(size_t)t * Cx + c] = f16_bits(v);
         if (t >= T - (W - 1)) ring[(size_t)(t % W) * Cx + c] = xBC[(size_t)t * zxw + c];
     }
     for (int h = threadIdx.x; h < H; h += blockDim.x)
@@ -190,13 +197,20 @@ __global__ void __launch_bounds__(256) pf_ssd_state_kernel(const float* __restri
     for (int jb = 0; jb < len; jb += kStJ) {
         const int nj = min(kStJ, len - jb);
         __syncthreads();   // w ready (first pass) / previous stage consumed
-        for (int idx = threadIdx.x; idx < nj * P; idx += blockDim.x) {
-            const int j = idx / P, p = idx - j * P;
-            xw[j * P + p] = w[jb + j] * xh[(size_t)(jb + j) * Cx + p];
+        const int P4 = P / 4, N4 = N / 4;
+#pragma unroll 4
+        for (int idx = threadIdx.x; idx < nj * P4; idx += blockDim.x) {
+            const int j = idx / P4, q = idx - j * P4;
+            float4 v = *reinterpret_cast<const float4*>(xh + (size_t)(jb + j) * Cx + 4 * q);
+            const float wj = w[jb + j];
+            v.x *= wj; v.y *= wj; v.z *= wj; v.w *= wj;
+            *reinterpret_cast<float4*>(xw + j * P + 4 * q) = v;
         }
-        for (int idx = threadIdx.x; idx < nj * N; idx += blockDim.x) {
-            const int j = idx / N, n = idx - j * N;
-            bs[j * N + n] = bg[(size_t)(jb + j) * Cx + n];
+#pragma unroll 4
+        for (int idx = threadIdx.x; idx < nj * N4; idx += blockDim.x) {
+            const int j = idx / N4, q = idx - j * N4;
+            *reinterpret_cast<float4*>(bs + j * N + 4 * q) =
+                *reinterpret_cast<const float4*>(bg + (size_t)(jb + j) * Cx + 4 * q);
         }
         __syncthreads();
         for (int j = 0; j < nj; ++j) {
@@ -222,8 +236,8 @@ __global__ void __launch_bounds__(256) pf_ssd_state_kernel(const float* __restri
 }
 
 // scan over chunks: S_in(0) = 0, S_in(c+1) = exp(Lam_end(c)) S_in(c) + S_c; final -> ssm state
-__global__ void pf_ssd_scan_kernel(const float* schunk, const float* lam, int T, int H, int P, int N, float* sin,
-                                   float* ssm_out) {
+__global__ void pf_ssd_scan_kernel(const float* schunk, const float* lam, int T, int H, int P, int N,
+                                   uint16_t* sin16, float* ssm_out) {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long per_head = (long long)P * N;
     if (idx >= (long long)H * per_head) return;
@@ -231,7 +245,7 @@ __global__ void pf_ssd_scan_kernel(const float* schunk, const float* lam, int T,
     const int nch = (T + kChunk - 1) / kChunk;
     float s = 0.0f;
     for (int c = 0; c < nch; ++c) {
-        sin[(size_t)c * H * per_head + idx] = s;
+        sin16[(size_t)c * H * per_head + idx] = bf16_bits(s);
         const int tend = min(T, (c + 1) * kChunk) - 1;
         s = expf(lam[(size_t)tend * H + h]) * s + schunk[(size_t)c * H * per_head + idx];
     }
@@ -313,7 +327,8 @@ __global__ void pf_finish_kernel(int32_t* ctx_len, int slot, int T) { ctx_len[sl
 // ------------------------------------------------------------------------------------------
 size_t prefill_mixer_scratch_bytes(int T, int E, int Cx, int H, int P, int N) {
     const size_t nch = (size_t)(T + kChunk - 1) / kChunk;
-    return al((size_t)T * Cx * 4) + 2 * al((size_t)T * H * 4) + al((size_t)T * E * 4) + 2 * al(nch * H * P * N * 4);
+    return al((size_t)T * Cx * 4) + 2 * al((size_t)T * H * 4) + al((size_t)T * E * 4) + al(nch * H * P * N * 4) +
+           al(nch * H * P * N * 2) + al((size_t)T * Cx * 2);
 }
 
 void carve_mixer(PfMixer& m, uint8_t* base) {
@@ -329,7 +344,8 @@ void carve_mixer(PfMixer& m, uint8_t* base) {
     m.lam = take((size_t)m.T * m.H * 4);
     m.y = take((size_t)m.T * m.E * 4);
     m.schunk = take(nch * m.H * m.P * m.N * 4);
-    m.sin = take(nch * m.H * m.P * m.N * 4);
+    m.sin16 = (uint16_t*)take(nch * m.H * m.P * m.N * 2);
+    m.xc16 = (uint16_t*)take((size_t)m.T * m.Cx * 2);
 }
 
 cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
@@ -344,7 +360,8 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
                                          (int)SL.total);
     if (e != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(m.ring, 0, (size_t)W * Cx * 2, s)) != cudaSuccess) return e;
-    pf_conv_kernel<<<T, 256, 0, s>>>(m.zx, zxw, T, E, Cx, H, W, Lw.conv_w, Lw.conv_b, Lw.dt_bias, m.xc, m.dt, m.ring);
+    pf_conv_kernel<<<T, 256, 0, s>>>(m.zx, zxw, T, E, Cx, H, W, Lw.conv_w, Lw.conv_b, Lw.dt_bias, m.xc, m.xc16, m.dt,
+                                     m.ring);
     const size_t st_smem = (size_t)kStJ * (P + N) * 4;
     const dim3 sg(nch, H);
     if (P <= 80 && P > 64 && N <= 128 && N > 112)
@@ -357,8 +374,8 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
         pf_ssd_state_kernel<8, 16><<<sg, 256, st_smem, s>>>(m.xc, m.dt, Lw.A_log, T, H, P, N, m.G, E, Cx, m.lam,
                                                               m.schunk);
     const long long n = (long long)H * P * N;
-    pf_ssd_scan_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(m.schunk, m.lam, T, H, P, N, m.sin, m.ssm);
-    pf_ssd_out_mma_kernel<<<dim3(nch, m.G, kChunk / kSsdTi), 256, SL.total, s>>>(m.xc, m.dt, m.lam, m.sin, Lw.D, T, H,
+    pf_ssd_scan_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(m.schunk, m.lam, T, H, P, N, m.sin16, m.ssm);
+    pf_ssd_out_mma_kernel<<<dim3(nch, m.G, kChunk / kSsdTi), 256, SL.total, s>>>(m.xc, m.xc16, m.dt, m.lam, m.sin16, Lw.D, T, H,
                                                                                  P, N, m.G, E, Cx, m.y);
     pf_gated_norm_kernel<<<dim3(T, m.NG), 256, 0, s>>>(m.y, m.zx, zxw, Lw.gnorm, E, m.NG, m.eps, m.act, m.act_ld,
                                                        m.f16);
@@ -368,23 +385,50 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
 // ------------------------------------------------------------------------------------------
 // orchestration
 // ------------------------------------------------------------------------------------------
+// The projections of one prefill, in order.  Weight i is unpacked (device layout -> row-major
+// 16-bit) into buffer i % 2 on the side stream while GEMM i - 1 runs on the caller's stream:
+//   side: wait "GEMM i-2 done" -> unpack i -> record "unpacked i % 2"
+//   main: wait "unpacked i % 2" -> GEMM i -> record "GEMM done i % 2"
 struct PfGemm {
     const PrefillCtx& c;
     const PfBufs& b;
     int f16;
     cudaStream_t s;
-    // unpack w to 16-bit row-major, then out = epilogue(A . w^T)
+    std::vector<const vc_qmat*> seq;
+    size_t next = 0;   // index of the next GEMM
+
+    cudaError_t unpack(size_t i) {
+        if (i >= seq.size()) return cudaSuccess;
+        const vc_qmat& w = *seq[i];
+        const int k = (int)(i & 1);
+        cudaError_t e = cudaStreamWaitEvent(c.side, i >= 2 ? c.ev[2 + k] : c.ev[4], 0);
+        if (e == cudaSuccess)
+            e = launch_unpack16(w.fmt, w.fmt == VC_W_BF16 ? 64 : w.group, w.N, w.K, (const uint8_t*)w.data,
+                                b.wdense[k], w.K, f16, c.side);
+        if (e == cudaSuccess) e = cudaEventRecord(c.ev[k], c.side);
+        return e;
+    }
+    cudaError_t start() {
+        cudaError_t e = cudaEventRecord(c.ev[4], s);   // buffers free once the caller's prior work is done
+        if (e == cudaSuccess) e = unpack(0);
+        return e;
+    }
+    // out = epilogue(A . w^T) for the next weight of the sequence
     cudaError_t operator()(int epi, const uint16_t* A, int lda, int M, const vc_qmat& w, const float* row_scale,
-                           uint16_t* out, int ldo, float* out32, int ldo32, const GemmArgs* qkv = nullptr) const {
-        cudaError_t e = launch_unpack16(w.fmt, w.fmt == VC_W_BF16 ? 64 : w.group, w.N, w.K, (const uint8_t*)w.data,
-                                        b.wdense, w.K, f16, s);
+                           uint16_t* out, int ldo, float* out32, int ldo32, const GemmArgs* qkv = nullptr) {
+        const size_t i = next++;
+        if (i >= seq.size() || seq[i] != &w) return cudaErrorInvalidValue;
+        const int k = (int)(i & 1);
+        cudaError_t e = cudaStreamWaitEvent(s, c.ev[k], 0);
         if (e != cudaSuccess) return e;
         GemmArgs a = qkv ? *qkv : GemmArgs{};
         a.f16 = f16; a.out_f16 = f16;
         a.A = A; a.lda = lda; a.M = M;
-        a.W = b.wdense; a.ldw = w.K; a.N = w.N; a.K = w.K;
+        a.W = b.wdense[k]; a.ldw = w.K; a.N = w.N; a.K = w.K;
         a.row_scale = row_scale; a.out = out; a.ldo = ldo; a.out_f32 = out32; a.ldo32 = ldo32; a.status = c.status;
-        return launch_gemm_tc(epi, a, s);
+        if ((e = launch_gemm_tc(epi, a, s)) != cudaSuccess) return e;
+        if ((e = cudaEventRecord(c.ev[2 + k], s)) != cudaSuccess) return e;
+        return unpack(i + 1);
     }
 };
 
@@ -395,9 +439,17 @@ cudaError_t run_prefill(const PrefillCtx& c, const uint16_t* x, int T, int slot,
     if (strchr(c.cfg->pattern, '*') && (c.Dh % 32 || c.Dh > 256)) return cudaErrorNotSupported;
     const PfBufs b = carve_pf(c.ws, T, d, E, Cx, H, P, N, c.Hq, c.Hk, c.Dh, c.F, nullptr);
     const int f16 = c.cfg->wfmt != VC_W_BF16;   // quantized weights: fp16 operands, as in the decode GEMV
-    const PfGemm gemm{c, b, f16, s};
+    PfGemm gemm{c, b, f16, s, {}, 0};
+    for (int l = 0; l < c.L; ++l) {
+        const vc_layer_weights& Lw = c.layers[l];
+        const char kind = c.cfg->pattern[l];
+        if (kind == 'M') gemm.seq.insert(gemm.seq.end(), {&Lw.in_proj, &Lw.out_proj});
+        else if (kind == '*') gemm.seq.insert(gemm.seq.end(), {&Lw.qkv, &Lw.o});
+        else gemm.seq.insert(gemm.seq.end(), {&Lw.up, &Lw.down});
+    }
     const float eps = c.cfg->eps;
-    cudaError_t e;
+    cudaError_t e = gemm.start();
+    if (e != cudaSuccess) return e;
     pf_rownorm_kernel<<<T, 256, 0, s>>>(x, b.r, c.layers[0].norm, b.act_d, b.ld_d, b.inv, d, eps, f16);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t rbytes = (size_t)T * d * 4;
@@ -414,7 +466,7 @@ cudaError_t run_prefill(const PrefillCtx& c, const uint16_t* x, int T, int slot,
             PfMixer m{};
             m.T = T; m.E = E; m.Cx = Cx; m.H = H; m.P = P; m.N = N; m.G = c.G; m.W = W; m.NG = c.NG;
             m.eps = eps; m.f16 = f16; m.Lw = &Lw;
-            m.xc = b.xc; m.dt = b.dt; m.lam = b.lam; m.y = b.y; m.schunk = b.schunk; m.sin = b.sin;
+            m.xc = b.xc; m.dt = b.dt; m.lam = b.lam; m.y = b.y; m.schunk = b.schunk; m.sin16 = b.sin16; m.xc16 = b.xc16;
             m.ssm = c.ssm + ((size_t)mi * c.n_slots + slot) * H * P * N;
             m.ring = c.conv + ((size_t)mi * c.n_slots + slot) * W * Cx;
             m.act = b.act_big; m.act_ld = b.ld_big;

@@ -20,6 +20,8 @@ struct PrefillCtx {
     int32_t* ctx_len;
     int32_t* status;
     float* tap;   // test tap or null: residual stream [L+1][T][d] (entry 0 = input, l+1 after layer l)
+    cudaStream_t side;   // weight unpacking, one GEMM ahead of the caller's stream
+    cudaEvent_t ev[5];   // unpacked[2], gemm done[2], call start
 };
 
 // Mamba-2 mixer of one layer over T frames from zero state: conv (ring written), chunked SSD
@@ -29,7 +31,9 @@ struct PfMixer {
     float eps;
     const vc_layer_weights* Lw;
     const uint16_t* zx;                              // bf16 [T][E+Cx+H]
-    float *xc, *dt, *lam, *y, *schunk, *sin;         // scratch (carve_mixer); y fp32 [T][E]
+    float *xc, *dt, *lam, *y, *schunk;               // scratch (carve_mixer); y fp32 [T][E]
+    uint16_t* xc16;                                  // fp16 copy of xc [T][Cx] (tensor-core operands)
+    uint16_t* sin16;                                 // bf16 state entering each chunk [nch][H][P][N]
     float* ssm;                                      // [H][P][N]
     uint16_t* ring;                                  // [W][Cx]
     uint16_t* act;                                   // [T][act_ld]

@@ -23,6 +23,12 @@ VC_DEV uint16_t bf16_bits(float v) {
 
 VC_DEV uint32_t pack_bf16x2(float lo, float hi) { return (uint32_t)bf16_bits(lo) | ((uint32_t)bf16_bits(hi) << 16); }
 
+VC_DEV void ldsm_x4_trans(uint32_t (&r)[4], const uint16_t* p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+
 // fp16 bits, saturated to the finite range
 VC_DEV uint16_t f16_bits(float v) {
     __half h = __float2half_rn(fminf(fmaxf(v, -65504.0f), 65504.0f));
@@ -43,7 +49,7 @@ static constexpr int kSsdChunk = 256;
 static constexpr int kSsdTi = 64;
 
 struct SsdLayout {
-    int sc, sb, scb, sw, ss, sx;               // row strides (elements)
+    int sc, sb, scb, sw, ss, sx;               // row strides (elements); x is stored [j][p]
     size_t off_c, off_c2, off_b, off_w, off_s, off_cb, off_x, off_l, total;
 };
 
@@ -54,7 +60,7 @@ __host__ __device__ inline SsdLayout ssd_layout(int N, int P) {
     L.scb = kSsdChunk + 4;
     L.sw = kSsdChunk + 8;
     L.ss = N + 8;
-    L.sx = kSsdChunk + 8;
+    L.sx = P + 8;
     auto a16 = [](size_t v) { return (v + 15) / 16 * 16; };
     const size_t rc = a16((size_t)kSsdTi * L.sc * 2);
     const size_t rb_b = (size_t)kSsdChunk * L.sb * 2;
@@ -68,14 +74,17 @@ __host__ __device__ inline SsdLayout ssd_layout(int N, int P) {
     L.off_s = 2 * rc + rw;
     L.off_cb = 2 * rc + rb;
     L.off_x = L.off_cb + a16((size_t)kSsdTi * L.scb * 4);
-    L.off_l = L.off_x + a16((size_t)P * L.sx * 2);
+    L.off_l = L.off_x + a16((size_t)kSsdChunk * L.sx * 2);
     L.total = L.off_l + 2 * kSsdChunk * 4;
     return L;
 }
 
-__global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __restrict__ xc, const float* __restrict__ dt,
+__global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __restrict__ xc,
+                                                             const uint16_t* __restrict__ xc16,
+                                                             const float* __restrict__ dt,
                                                              const float* __restrict__ lam,
-                                                             const float* __restrict__ sin, const float* __restrict__ Dv,
+                                                             const uint16_t* __restrict__ sin16,
+                                                             const float* __restrict__ Dv,
                                                              int T, int H, int P, int N, int G, int E, int Cx,
                                                              float* __restrict__ y) {
     extern __shared__ __align__(16) unsigned char smraw[];
@@ -94,23 +103,36 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
     uint16_t* Ws = reinterpret_cast<uint16_t*>(smraw + L.off_w);
     uint16_t* Sb = reinterpret_cast<uint16_t*>(smraw + L.off_s);
     float* CBs = reinterpret_cast<float*>(smraw + L.off_cb);
-    uint16_t* Xt = reinterpret_cast<uint16_t*>(smraw + L.off_x);
+    uint16_t* Xs = reinterpret_cast<uint16_t*>(smraw + L.off_x);     // x rows of the head, fp16 [j][p]
     float* lam_s = reinterpret_cast<float*>(smraw + L.off_l);
     float* dts = lam_s + kSsdChunk;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-    const float* Cg = xc + (size_t)t0 * Cx + E + (size_t)G * N + (size_t)g * N;
-    const float* Bg = xc + (size_t)t0 * Cx + E + (size_t)g * N;
+    const size_t coff = (size_t)t0 * Cx + E + (size_t)G * N + (size_t)g * N;
+    const size_t boff = (size_t)t0 * Cx + E + (size_t)g * N;
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    const int n8 = N / 8;
 
-    // 1. the group's C rows of the tile (fp16 and bf16) and B rows 0..jn-1 (fp16), zero padded
-    for (int idx = tid; idx < kSsdTi * N; idx += blockDim.x) {
-        const int ii = idx / N, n = idx - ii * N;
-        const float v = i0 + ii < i1 ? Cg[(size_t)(i0 + ii) * Cx + n] : 0.0f;
-        Cs[ii * L.sc + n] = f16_bits(v);
-        Cb[ii * L.sc + n] = bf16_bits(v);
+    // 1. the group's C rows of the tile (fp16 copies, and bf16 for the entering-state product)
+    //    and B rows 0..jn-1 (fp16), zero padded; 16-byte copies from the fp16 image of xc
+#pragma unroll 4
+    for (int idx = tid; idx < kSsdTi * n8; idx += blockDim.x) {
+        const int ii = idx / n8, c8 = idx - ii * n8;
+        const bool ok = i0 + ii < i1;
+        *reinterpret_cast<uint4*>(Cs + ii * L.sc + c8 * 8) =
+            ok ? *reinterpret_cast<const uint4*>(xc16 + coff + (size_t)(i0 + ii) * Cx + c8 * 8) : z4;
+        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+        if (ok) {
+            v0 = *reinterpret_cast<const float4*>(xc + coff + (size_t)(i0 + ii) * Cx + c8 * 8);
+            v1 = *reinterpret_cast<const float4*>(xc + coff + (size_t)(i0 + ii) * Cx + c8 * 8 + 4);
+        }
+        *reinterpret_cast<uint4*>(Cb + ii * L.sc + c8 * 8) =
+            make_uint4(pack_bf16x2(v0.x, v0.y), pack_bf16x2(v0.z, v0.w), pack_bf16x2(v1.x, v1.y), pack_bf16x2(v1.z, v1.w));
     }
-    for (int idx = tid; idx < jn32 * N; idx += blockDim.x) {
-        const int j = idx / N, n = idx - j * N;
-        Bs[j * L.sb + n] = f16_bits(j < jn ? Bg[(size_t)j * Cx + n] : 0.0f);
+#pragma unroll 4
+    for (int idx = tid; idx < jn32 * n8; idx += blockDim.x) {
+        const int j = idx / n8, c8 = idx - j * n8;
+        *reinterpret_cast<uint4*>(Bs + j * L.sb + c8 * 8) =
+            j < jn ? *reinterpret_cast<const uint4*>(xc16 + boff + (size_t)j * Cx + c8 * 8) : z4;
     }
     __syncthreads();
 
@@ -167,14 +189,19 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
             dts[j] = j < jn ? dt[(size_t)(t0 + j) * H + h] : 0.0f;
         }
         const float* xh = xc + (size_t)t0 * Cx + (size_t)h * P;
-        for (int idx = tid; idx < jn16 * P; idx += blockDim.x) {
-            const int j = idx / P, p = idx - j * P;
-            Xt[p * L.sx + j] = f16_bits(j < jn ? xh[(size_t)j * Cx + p] : 0.0f);
+        const uint16_t* xh16 = xc16 + (size_t)t0 * Cx + (size_t)h * P;
+        const int p8 = P / 8;
+#pragma unroll 4
+        for (int idx = tid; idx < jn16 * p8; idx += blockDim.x) {
+            const int j = idx / p8, c8 = idx - j * p8;
+            *reinterpret_cast<uint4*>(Xs + j * L.sx + c8 * 8) =
+                j < jn ? *reinterpret_cast<const uint4*>(xh16 + (size_t)j * Cx + c8 * 8) : z4;
         }
-        const float* Sh = sin + ((size_t)c * H + h) * P * N;
-        for (int idx = tid; idx < P * N; idx += blockDim.x) {
-            const int p = idx / N, n = idx - p * N;
-            Sb[p * L.ss + n] = bf16_bits(Sh[idx]);
+        const uint16_t* Sh = sin16 + ((size_t)c * H + h) * P * N;
+#pragma unroll 4
+        for (int idx = tid; idx < P * n8; idx += blockDim.x) {
+            const int p = idx / n8, c8 = idx - p * n8;
+            *reinterpret_cast<uint4*>(Sb + p * L.ss + c8 * 8) = *reinterpret_cast<const uint4*>(Sh + (size_t)p * N + c8 * 8);
         }
         __syncthreads();
         for (int idx = tid; idx < kSsdTi * jn16; idx += blockDim.x) {
@@ -190,6 +217,10 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
         for (int q = 0; q < 8; ++q)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[q][e] = acc2[q][e] = 0.0f;
+        // x fragments by transposing 8x8 loads of the [j][p] rows: lanes 0-7 rows k0..k0+7,
+        // 8-15 rows k0+8..k0+15 (columns p0..p0+7), 16-31 the same rows at columns p0+8..p0+15
+        const int lk = (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int lp = 8 * (lane >> 4);
         for (int k0 = 0; k0 < kend; k0 += 16) {
             uint32_t af[4];
             const uint16_t* r = Ws + (wm * 16 + gq) * L.sw + k0 + 2 * tq;
@@ -198,10 +229,12 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
             af[2] = lds32(r + 8);
             af[3] = lds32(r + 8 * L.sw + 8);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
+            for (int q = 0; q < 8; q += 2)
                 if (q < qn) {
-                    const uint16_t* br = Xt + ((q0 + q) * 8 + gq) * L.sx + k0 + 2 * tq;
-                    mma_f16(acc[q], af, lds32(br), lds32(br + 8), acc[q]);
+                    uint32_t xb[4];
+                    ldsm_x4_trans(xb, Xs + (k0 + lk) * L.sx + (q0 + q) * 8 + lp);
+                    mma_f16(acc[q], af, xb[0], xb[1], acc[q]);
+                    if (q + 1 < qn) mma_f16(acc[q + 1], af, xb[2], xb[3], acc[q + 1]);
                 }
         }
         for (int k0 = 0; k0 < N; k0 += 16) {
@@ -248,11 +281,6 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
 // softmax in fp32 (exp2 with the 1/sqrt(Dh) scale folded in), P rounded to bf16 for P.V.
 // q head i reads KV head floor(i Hk / Hq); no positional encoding.
 // ------------------------------------------------------------------------------------------
-VC_DEV void ldsm_x4_trans(uint32_t (&r)[4], const uint16_t* p) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(smem_u32(p)));
-}
 
 template <int DH>
 __global__ void __launch_bounds__(128) pf_flash_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
