@@ -4,6 +4,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <map>
 #include <string>
 #include <tuple>
@@ -99,6 +100,7 @@ struct Workspace {
     int* ok;
     float* partials;
     int* counters;
+    float* accum;
     float* attn_scratch;
     int* attn_counters;
     unsigned long long* keys;
@@ -182,6 +184,20 @@ static bool dims_from_cfg(const vc_config* c, Dims& D) {
     return true;
 }
 
+// fp32 accumulators of the step's split GEMV units: the largest launch's units x R x NT x 128
+static size_t accum_floats(const vc_config* c, const Dims& D) {
+    const int NT = D.B > 8 ? 2 : 1;
+    auto units = [&](int fmt, int N) {
+        const int grp = fmt == VC_W_BF16 ? 64 : c->group_size;
+        const LayoutInfo L = layout_info(fmt, grp);
+        return (size_t)((N + 16 * L.R - 1) / (16 * L.R)) * L.R * NT * 128;
+    };
+    size_t m = 0;
+    for (int N : {D.zx_rows, D.qkv_rows, D.F, D.d}) m = std::max(m, units(c->wfmt, N));
+    m = std::max(m, units(c->head_fmt, D.Vt) + units(c->head_fmt, D.Vf));
+    return m;
+}
+
 extern "C" size_t vc_workspace_bytes(const vc_config* cfg) {
     Dims D;
     if (!dims_from_cfg(cfg, D)) return 0;
@@ -209,6 +225,7 @@ extern "C" size_t vc_workspace_bytes(const vc_config* cfg) {
     add((size_t)B * D.d * 2);                 // x staging
     add(2 * 16 * 4);                          // token staging
     add(prefill_workspace_bytes(D.d, D.L, D.E, D.Cx, D.H, D.P, D.N, D.G, D.Hq, D.Hk, D.Dh, D.F, D.cap));
+    add(accum_floats(cfg, D) * 4);            // split-unit accumulators
     return align_up(total, 256);
 }
 
@@ -247,6 +264,7 @@ static void carve(vc_backbone* h, uint8_t* base) {
     W.tok_stage = (int32_t*)take(2 * 16 * 4);
     W.prefill_bytes = prefill_workspace_bytes(D.d, D.L, D.E, D.Cx, D.H, D.P, D.N, D.G, D.Hq, D.Hk, D.Dh, D.F, D.cap);
     W.prefill = take(W.prefill_bytes);
+    W.accum = (float*)take(accum_floats(&h->cfg, D) * 4);
 }
 
 static bool qmat_ok(const vc_qmat& m, int fmt, int group, int N, int K) {
@@ -370,7 +388,8 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
     pre.inv_width = 1.0f / D.d; pre.eps = h->cfg.eps;
 
     GemvArgs base{};
-    base.nmat = 1; base.B = B; base.partials = W.partials; base.counters = W.counters; base.status = st->status;
+    base.nmat = 1; base.B = B; base.partials = W.partials; base.counters = W.counters; base.accum = W.accum;
+    base.status = st->status;
     base.slots = slots; base.ok = W.ok; base.ctx_len = st->ctx_len;
     GemvLaunch gl{};
     gl.fmt = fmt; gl.group = grp; gl.num_sms = h->num_sms; gl.pdl = pdl;

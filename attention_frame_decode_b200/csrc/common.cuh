@@ -149,6 +149,11 @@ VC_DEV uint16_t act_bits(float v) {
     }
 }
 
+// fp32 vector reduction into global memory (performed at L2), no return value
+VC_DEV void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
 VC_DEV float bf16_bits_to_f(uint16_t u) { return __uint_as_float((uint32_t)u << 16); }
 
 VC_DEV float warp_sum(float v) {

@@ -61,6 +61,11 @@ struct GemvArgs {
     // scratch + status
     float* partials;
     int* counters;
+    // optional: per-unit fp32 accumulators (zero on entry, left zero), R*NT*128 floats per unit
+    // of every matrix of the launch.  When set, contributors to a split unit add their fragment
+    // sums atomically and the last one reads the total once (shorter tail; the summation order
+    // then varies from run to run); when null, partials are summed in worker order.
+    float* accum;
     int* status;
 };
 

@@ -356,6 +356,36 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
             epilogue(u, acc);
             return;
         }
+        if (args.accum) {
+            float* au = args.accum + ((size_t)(m ? args.mat[0].NU : 0) + u) * (R * NT * 128);
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int j = 0; j < NT; ++j)
+                    red_add_v4(au + ((r * NT + j) * 32 + lane) * 4, acc[r][j][0], acc[r][j][1], acc[r][j][2],
+                               acc[r][j][3]);
+            __threadfence();
+            __syncwarp();
+            int old = 0;
+            int* cnt = args.counters + (m ? args.mat[0].NU : 0) + u;
+            if (lane == 0) old = atomicAdd(cnt, 1);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            if (old != (int)(hi - lo)) return;
+            __threadfence();
+            float tot[R][NT][4];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    float4* p4 = reinterpret_cast<float4*>(au + ((r * NT + j) * 32 + lane) * 4);
+                    const float4 v = __ldcg(p4);
+                    __stcg(p4, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+                    tot[r][j][0] = v.x; tot[r][j][1] = v.y; tot[r][j][2] = v.z; tot[r][j][3] = v.w;
+                }
+            if (lane == 0) *cnt = 0;
+            epilogue(u, tot);
+            return;
+        }
         const long long first_u = f0 / M.KT;
         float* mine = args.partials + ((size_t)(wbase + wl) * 2 + (u == first_u ? 0 : 1)) * (R * NT * 128);
 #pragma unroll
