@@ -637,6 +637,14 @@ extern "C" vc_status vc_debug_gemv(const vc_qmat* w, const void* act, int act_ld
     a.tap_ld = w->N;
     a.partials = (float*)scratch;
     a.counters = (int*)((uint8_t*)scratch + align_up(gemv_partials_bytes(256), 256));
+    // split units are summed as in the step (fp32 accumulators in the zeroed partial area, left
+    // zeroed) when they fit there; otherwise contributors' partials are summed in worker order
+    {
+        const int grp = w->fmt == VC_W_BF16 ? 64 : w->group;
+        const LayoutInfo Lw = layout_info(w->fmt, grp);
+        const size_t need = (size_t)a.mat[0].NU * Lw.R * (B > 8 ? 2 : 1) * 128 * 4;
+        if (need <= gemv_partials_bytes(256)) a.accum = a.partials;
+    }
     GemvLaunch L{};
     L.fmt = w->fmt;
     L.group = w->fmt == VC_W_BF16 ? 64 : w->group;

@@ -76,6 +76,16 @@ def launches_per_step(cfg):
     return n
 
 
+# DRAM bytes (read + write) per launch of the roofline kernel, from one ncu capture of the same
+# kernel and shape (profiles/gemv_mlp_shapes_bf16_w4.md, profiles/gemm_tc_prefill_4096x15680x4480.md);
+# None where no capture of the current kernel exists.
+TRAFFIC = {
+    "nano_bf16": 141.117440e6 + 4.171776e6,      # gemv bf16 15680 x 4480, B = 1
+    "nano_w4": 38.452480e6 + 0.0,                # gemv W4 g64 15680 x 4480, B = 1
+    "nano_prefill": 241.034496e6 + 236.244736e6,  # tcgen05 GEMM 4096 x 15680 x 4480
+}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -311,7 +321,7 @@ def run_prefill_bench(args, cfg, world, rank, local):
             "step_tflops": step_tflops, "flops_per_step": {"projections": proj, "attention": attn, "ssd": ssd},
             "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMM (MLP up projection shape)", "achieved": gemm_tf,
                          "peak": peak, "peak_kind": "measured burst" if pk else "fallback", "unit": "TFLOP/s",
-                         "frac": gemm_tf / peak, "traffic": None, "launch_ms": gemm_ms,
+                         "frac": gemm_tf / peak, "traffic": TRAFFIC.get(cfg.name), "launch_ms": gemm_ms,
                          "flops_per_launch": 2.0 * M * N * K},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "frames/s", "h2d_bytes_per_step": T * cfg.d_model * 2,
@@ -492,7 +502,7 @@ def main():
             "step_frac_of_peak": step_gbs / peak,
             "roofline": {"bound": "hbm", "kernel": "gemv (mlp up projection, streaming weights)",
                          "achieved": gemv_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": gemv_gbs / peak, "traffic": None, "launch_ms": gemv_ms,
+                         "frac": gemv_gbs / peak, "traffic": TRAFFIC.get(cfg.name), "launch_ms": gemv_ms,
                          "bytes_per_launch": gemv_bytes},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "frame-steps/s", "h2d_bytes_per_step": B * cfg.d_model * 2,

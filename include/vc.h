@@ -211,7 +211,9 @@ vc_status vc_debug_mamba_step(const vc_config* cfg, const vc_layer_weights* laye
  * act: 16-bit [B][act_ld] (device; bf16 bits for VC_W_BF16 weights, fp16 bits for quantized
  * ones), act_ld a multiple of 128 and >= K rounded up to 128, columns K..act_ld-1 zero;
  * 1 <= B <= 16.  out: fp32 [B][N] (device).  scratch: device buffer of vc_gemv_scratch_bytes()
- * bytes, zero on first use; the kernel leaves it zeroed again for the next call. */
+ * bytes, zero on first use; every call returns the counters and accumulators it uses to zero.
+ * Split row units are summed as in vc_step (fp32 reductions into accumulators, order varying
+ * from run to run) when their accumulators fit the scratch, else in worker order. */
 size_t vc_gemv_scratch_bytes(void);
 vc_status vc_debug_gemv(const vc_qmat* w, const void* act, int act_ld, int B, float* out, void* scratch,
                         vc_stream_t stream);
