@@ -86,6 +86,25 @@ TRAFFIC = {
 }
 
 
+def max_over_ranks(value: float, world: int) -> float:
+    """the largest of every rank's value (device timings are taken as the max over ranks);
+    the tensor lives where the process group's backend wants it (CUDA for NCCL, CPU for gloo)"""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_rate(units_per_rank: float, world: int, seconds: float) -> float:
+    """whole-job throughput of `world` independent replicas that each processed
+    units_per_rank units in at most `seconds` (the max over ranks)"""
+    return world * units_per_rank / seconds
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -255,12 +274,9 @@ def run_prefill_bench(args, cfg, world, rank, local):
         dist.barrier()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
-    value = world * T * args.steps / (ms / 1000.0)
+    value = replica_rate(T * args.steps, world, ms / 1000.0)
     proj, attn, ssd = prefill_flops(cfg, T)
     step_tflops = (proj + attn + ssd) / (ms_step / 1000.0) / 1e12
 
@@ -417,13 +433,10 @@ def main():
         dist.barrier()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     status = int(st.status.cpu()[0])
     ms_step = ms / args.steps
-    value = world * B * args.steps / (ms / 1000.0)
+    value = replica_rate(B * args.steps, world, ms / 1000.0)
     ctx_mean = float(ctx0.mean()) + args.warmup + args.steps / 2.0
     rbytes, wbytes, weight_total = step_bytes(cfg, B, ctx_mean)
     step_gbs = rbytes / (ms_step / 1000.0) / 1e9
@@ -471,10 +484,7 @@ def main():
         bb.step_host(xh[s], st, th, fh)
         stream.synchronize()   # the frame's tokens are on the host before the next frame
     e2e_s = time.perf_counter() - t0
-    if world > 1:
-        t = torch.tensor([e2e_s], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks(e2e_s, world)
     e2e_value = world * B * (ne - 1) / e2e_s
 
     cpu = None
