@@ -1,14 +1,18 @@
 // gemm_tc.cu -- tcgen05 GEMM for the prefill projections (dense contraction over the frames).
 //
-// C[M][N] = A[M][K] . W[N][K]^T, bf16 x bf16 -> fp32 in tensor memory (TMEM).
-// Tile 128 x 256 x 64, 4-stage TMA ring (128-byte swizzle, no multicast), one CTA per tile:
-//   warp 0 (one thread): TMA producer, waits "empty" mbarriers, loads A and W tiles;
-//   warp 1: allocates 256 TMEM columns; one thread issues tcgen05.mma (M=128, N=256, K=16,
-//           4 per 64-wide k-block) and tcgen05.commit to free each stage and, at the end, to
-//           signal the accumulator;
-//   warps 2-5: epilogue; each reads its 32 TMEM lanes (rows) with tcgen05.ld and applies the
-//           fused epilogue (row scale of the pre-RMSNorm, squared ReLU, residual add, q/k/v split
-//           into the KV cache) while storing to global memory.
+// C[M][N] = A[M][K] . W[N][K]^T, 16-bit x 16-bit -> fp32 in tensor memory (TMEM).
+// Persistent: one CTA per SM walks the 128 x 256 output tiles (M-tile fastest, so the CTAs
+// resident together share a few W column tiles, each streamed from HBM once, while the
+// activation rows stay in L2).  Per CTA:
+//   warp 0 (one thread): TMA producer over a 4-stage ring of 64-wide k-blocks (128-byte swizzle,
+//           no multicast), across tile boundaries;
+//   warp 1: allocates 512 TMEM columns = two 128 x 256 fp32 accumulators; one thread issues
+//           tcgen05.mma (M=128, N=256, K=16, 4 per k-block) into accumulator (tile & 1),
+//           commits each stage back to the producer and each finished tile to the epilogue;
+//   warps 2-5: epilogue; each reads its 32 TMEM lanes (rows) with tcgen05.ld, applies the fused
+//           epilogue (row scale of the pre-RMSNorm, squared ReLU, residual add, q/k/v split into
+//           the KV cache), stores, and hands the accumulator back -- while the MMAs of the next
+//           tile already run into the other accumulator.
 // Every mbarrier wait is bounded; a timeout sets the status word and the CTA still frees TMEM.
 #include <cuda.h>
 
@@ -20,7 +24,7 @@ namespace vc {
 static constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 static constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 static constexpr int GEMM_THREADS = 192;
-static constexpr int TMEM_COLS = 256;
+static constexpr int TMEM_COLS = 512;   // two accumulators of BN fp32 columns
 
 VC_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
@@ -85,14 +89,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, const GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full[STAGES], empty[STAGES], accum;
+    __shared__ uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2];
     __shared__ uint32_t tmem_base;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // M-tile fastest: the CTAs resident at one time share a few W column tiles (each streamed
-    // from HBM once) while the activation rows, re-read per W tile, stay in L2
     const int mt = (a.M + BM - 1) / BM;
-    const int n0 = (int)(blockIdx.x / mt) * BN, m0 = (int)(blockIdx.x % mt) * BM;
+    const int tiles = mt * ((a.N + BN - 1) / BN);
     const int KB = (a.K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
@@ -100,7 +102,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(&accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 128);
+        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -116,49 +121,90 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % STAGES;
-                if (kb >= STAGES && !mbar_wait(&empty[s], (uint32_t)(((kb / STAGES) - 1) & 1), a.status)) break;
-                mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-                tma_load_2d(smem + s * STAGE_BYTES, &tmA, kb * BK, m0, &full[s]);
-                tma_load_2d(smem + s * STAGE_BYTES + A_BYTES, &tmW, kb * BK, n0, &full[s]);
+            int it = 0;   // k-blocks issued by this CTA so far
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+                const int n0 = (tile / mt) * BN, m0 = (tile % mt) * BM;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (it >= STAGES && !mbar_wait(&empty[s], (uint32_t)(((it / STAGES) - 1) & 1), a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                    tma_load_2d(smem + s * STAGE_BYTES, &tmA, kb * BK, m0, &full[s]);
+                    tma_load_2d(smem + s * STAGE_BYTES + A_BYTES, &tmW, kb * BK, n0, &full[s]);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
+            int it = 0, lt = 0;
             bool ok = true;
-            for (int kb = 0; kb < KB && ok; ++kb) {
-                const int s = kb % STAGES;
-                if (!mbar_wait(&full[s], (uint32_t)((kb / STAGES) & 1), a.status)) { ok = false; break; }
+            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++lt) {
+                const int b = lt & 1;
+                // the epilogue has drained this accumulator (its use two tiles ago)
+                if (lt >= 2 && !mbar_wait(&acc_empty[b], (uint32_t)(((lt >> 1) - 1) & 1), a.status)) break;
                 tc_fence_after();
-                const uint32_t abase = smem_u32(smem + s * STAGE_BYTES), bbase = abase + A_BYTES;
+                const uint32_t dacc = tmem + (uint32_t)(b * BN);
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&full[s], (uint32_t)((it / STAGES) & 1), a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t abase = smem_u32(smem + s * STAGE_BYTES), bbase = abase + A_BYTES;
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k)
-                    tc_mma(tmem, desc_sw128(abase + k * 32), desc_sw128(bbase + k * 32), idesc<F16>(), (kb | k) != 0);
-                tc_commit(&empty[s]);
+                    for (int k = 0; k < BK / 16; ++k)
+                        tc_mma(dacc, desc_sw128(abase + k * 32), desc_sw128(bbase + k * 32), idesc<F16>(),
+                               (kb | k) != 0);
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(&acc_full[b]);   // arrives when every MMA of the tile has completed
             }
-            tc_commit(&accum);   // arrives when every issued MMA has completed
         }
     } else {
         // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
         const int quarter = warp & 3;
-        const int row = m0 + quarter * 32 + lane;
-        const bool ready = mbar_wait(&accum, 0, a.status);
-        tc_fence_after();
-        if (ready) {
+        int lt = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
+            const int b = lt & 1;
+            const int n0 = (tile / mt) * BN, m0 = (tile % mt) * BM;
+            const int row = m0 + quarter * 32 + lane;
+            const bool ready = mbar_wait(&acc_full[b], (uint32_t)((lt >> 1) & 1), a.status);
+            tc_fence_after();
+            if (!ready) break;
             const float rs = (a.row_scale && row < a.M) ? a.row_scale[row] : 1.0f;
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 float v[32];
-                tc_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, v);
+                tc_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN + c0), v);
                 if (row >= a.M) continue;
                 const int col0 = n0 + c0;
                 if constexpr (EPI == GE_F32) {
-                    for (int j = 0; j < 32; ++j)
-                        if (col0 + j < a.N) a.out_f32[(size_t)row * a.ldo32 + col0 + j] = v[j];
+                    float* dst = a.out_f32 + (size_t)row * a.ldo32 + col0;
+                    if (col0 + 32 <= a.N && (((uintptr_t)dst) & 15) == 0) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            reinterpret_cast<float4*>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    } else {
+                        for (int j = 0; j < 32; ++j)
+                            if (col0 + j < a.N) dst[j] = v[j];
+                    }
                 } else if constexpr (EPI == GE_RESID) {
                     float* dst = a.out_f32 + (size_t)row * a.ldo32 + col0;
-                    for (int j = 0; j < 32; ++j)
-                        if (col0 + j < a.N) dst[j] += v[j];
+                    if (col0 + 32 <= a.N && (((uintptr_t)dst) & 15) == 0) {
+                        float4 r4[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) r4[q] = reinterpret_cast<const float4*>(dst)[q];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            reinterpret_cast<float4*>(dst)[q] = make_float4(r4[q].x + v[4 * q], r4[q].y + v[4 * q + 1],
+                                                                           r4[q].z + v[4 * q + 2], r4[q].w + v[4 * q + 3]);
+                    } else {
+                        for (int j = 0; j < 32; ++j)
+                            if (col0 + j < a.N) dst[j] += v[j];
+                    }
                 } else if constexpr (EPI == GE_QKV) {
                     const int qrows = a.Hq * a.Dh;
                     for (int j = 0; j < 32; ++j) {
@@ -199,6 +245,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     }
                 }
             }
+            // accumulator b may take the tile after next
+            tc_fence_before();
+            mbar_arrive(&acc_empty[b]);
         }
     }
     tc_fence_before();
@@ -248,7 +297,14 @@ static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mw, const 
     auto kern = gemm_tc_kernel<EPI, F16>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)(((a.N + BN - 1) / BN) * ((a.M + BM - 1) / BM)));
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    }
+    const int tiles = ((a.N + BN - 1) / BN) * ((a.M + BM - 1) / BM);
+    dim3 grid((unsigned)(tiles < sms ? tiles : sms));
     kern<<<grid, GEMM_THREADS, smem, s>>>(ma, mw, a);
     return cudaGetLastError();
 }
