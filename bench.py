@@ -396,15 +396,16 @@ def main():
     B = cfg.batch
     seed = 0
     dm = build_model(cfg, seed)
-    cap = cfg.kv_capacity
+    ctx0 = synth.context_lengths(cfg, seed, B)
+    total = args.warmup + args.steps
+    # the workload's cache capacity, grown when the run itself needs more frames than it holds
+    cap = max(cfg.kv_capacity, int(ctx0.max()) + total + args.e2e_steps + 8)
     bb = dm.backbone(B, cap, B)
     if args.no_graph:
         bb.set_option(vc.OPT_GRAPH, 0)
     st = dm.new_state(B, cap)
-    ctx0 = synth.context_lengths(cfg, seed, B)
     if cfg.random_state:
         fill_state(st, cfg, seed + rank, ctx0, cap)
-    total = args.warmup + args.steps
     # every frame input of the run, resident in HBM before timing (rank r serves its own sessions)
     xs = torch.empty((total, B, cfg.d_model), dtype=torch.bfloat16, device="cuda")
     for s in range(total):
