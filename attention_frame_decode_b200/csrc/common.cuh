@@ -118,15 +118,6 @@ VC_DEV uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
     return h2_as_u32(__hfma2(u32_as_h2(a), u32_as_h2(b), u32_as_h2(c)));
 }
 
-// release / acquire counters for cross-warp hand-offs (no full memory barrier on the producer)
-VC_DEV void red_release_add(int* p, int v) {
-    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-VC_DEV int ld_acquire(const int* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 
 // orderable key for float max with lowest-index tie-break: larger key <=> larger value, then smaller index
 VC_DEV unsigned long long argmax_key(float v, int idx) {

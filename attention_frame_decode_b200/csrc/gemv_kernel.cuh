@@ -1,10 +1,10 @@
 // gemv_kernel.cuh -- streaming weight GEMV for the per-frame decode step (B <= 16 sessions).
 //
-// The per-frame LLM step is memory-bandwidth bound ("The LLM step is limited by memory
-// bandwidth, so fewer bits read means a faster step", NemotronLabs VoiceChat 11B: GPTQ 3-bit
-// LLM, MLX, "Measurements"), so the kernel is built to read every weight byte exactly once at
-// full HBM rate:
-//   * persistent grid (one 8-warp CTA per SM); each warp is a worker that owns one contiguous
+// The per-frame LLM step is bound by memory bandwidth, and its time falls with the bits per
+// weight (NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM, MLX, the measurement bullets of the
+// introduction), so the kernel is built to read every weight byte exactly once at full HBM rate:
+//   * persistent grid (two 8-warp CTAs per SM for up to 8 batch rows, one for 9..16); each warp
+//     is a worker that owns one contiguous
 //     byte range of the matrix (see layout.cuh) and streams it through its own ring of shared
 //     memory slots with 1-D bulk copies (cp.async.bulk, TMA engine) completing on mbarriers;
 //   * the weight copies of the first ring slots are issued before griddepcontrol.wait, so they
@@ -12,9 +12,11 @@
 //   * dequantization is a few lop3/prmt + one fp16 op per pair of weights (exponent-field
 //     trick: OR a code into the mantissa of 1024.0, subtract 1024 + z) feeding mma.sync
 //     m16n8k16 with fp32 accumulation; quantization-group scales multiply the fp32 group sums;
-//   * a unit (16R rows) cut between workers is finished by the last of them (atomic counter),
-//     which adds the others' fp32 partials in worker order (deterministic), then runs the
-//     fused epilogue.
+//   * a unit (16R rows) cut between workers is finished by the last of them (atomic counter):
+//     in the step the contributors add their fp32 sums into a per-unit accumulator with vector
+//     reductions and the last one reads the total once; without an accumulator (test entries)
+//     the last one adds the others' fp32 partials in worker order (deterministic); then it runs
+//     the fused epilogue.
 #pragma once
 #include "common.cuh"
 #include "gemv.cuh"
@@ -22,8 +24,8 @@
 
 namespace vc {
 
-static constexpr int kWarps = 16;   // upper bound of warps per CTA
-// warps per CTA: 16 for up to 8 batch rows (<= 128 registers each), 8 for 9..16 rows
+static constexpr int kWarps = 16;   // upper bound of warps per CTA (sizes the partial-sum scratch)
+// warps per CTA: 8 for every batch size
 __host__ __device__ constexpr int warps_for(int) { return 8; }
 // CTAs per SM: two 8-warp CTAs for up to 8 rows (<= 128 registers, <= ~105 KB shared memory each),
 // so that under programmatic dependent launch the next kernel's CTAs can become resident and
