@@ -211,6 +211,34 @@ __global__ void unpack_kernel(int N, int K, int KT, const uint8_t* in, uint16_t*
     out[(size_t)n * ldo + k] = bits;
 }
 
+// bf16 weights: one warp per 16-row tile of a block.  Lane (g, t) holds, in its four 16-byte
+// words (s = 0..3), rows g and g + 8 at columns 16 t + 4 s + {0..3} (words 0/2: row g, words 1/3:
+// row g + 8), so it writes 16 consecutive columns of both rows with two 16-byte stores each.
+__global__ void unpack_bf16_tiles_kernel(int N, int K, int KT, int tiles, const uint8_t* in, uint16_t* out, int ldo) {
+    constexpr LayoutInfo L = layout_info(FMT_BF16, 64);
+    const int warp = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (warp >= tiles) return;
+    const int r = warp % L.R, blk = warp / L.R;
+    const int u = blk / KT, kt = blk % KT;
+    const uint8_t* tile = in + (size_t)blk * L.block_bytes + (size_t)r * L.tile_bytes;
+    uint4 v[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) v[s] = *reinterpret_cast<const uint4*>(tile + (s * 32 + lane) * 16);
+    const int g = lane >> 2, t = lane & 3;
+    const int col = kt * 64 + 16 * t;
+    const int row0 = u * 16 * L.R + 16 * r + g;
+    const uint4 lo0 = make_uint4(v[0].x, v[0].z, v[1].x, v[1].z), lo1 = make_uint4(v[2].x, v[2].z, v[3].x, v[3].z);
+    const uint4 hi0 = make_uint4(v[0].y, v[0].w, v[1].y, v[1].w), hi1 = make_uint4(v[2].y, v[2].w, v[3].y, v[3].w);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int row = row0 + 8 * h;
+        if (row >= N) continue;
+        uint16_t* dst = out + (size_t)row * ldo + col;
+        if (col < K) *reinterpret_cast<uint4*>(dst) = h ? hi0 : lo0;
+        if (col + 8 < K) *reinterpret_cast<uint4*>(dst + 8) = h ? hi1 : lo1;
+    }
+}
+
 template <int FMT, int GRP>
 static cudaError_t unp_t(int N, int K, const uint8_t* w, uint16_t* out, int ldo, int f16, cudaStream_t s) {
     MatGeom G = mat_geom(FMT, GRP, N, K);
@@ -221,6 +249,13 @@ static cudaError_t unp_t(int N, int K, const uint8_t* w, uint16_t* out, int ldo,
 
 cudaError_t launch_unpack16(int fmt, int group, int N, int K, const uint8_t* w, uint16_t* out, int ldo, int f16,
                             cudaStream_t s) {
+    if (fmt == FMT_BF16 && K % 8 == 0 && ldo % 8 == 0 && (((uintptr_t)out) & 15) == 0) {
+        constexpr LayoutInfo L = layout_info(FMT_BF16, 64);
+        const MatGeom G = mat_geom(FMT_BF16, 64, N, K);
+        const int tiles = G.NU * G.KT * L.R;
+        unpack_bf16_tiles_kernel<<<(unsigned)((tiles + 7) / 8), 256, 0, s>>>(N, K, G.KT, tiles, w, out, ldo);
+        return cudaGetLastError();
+    }
     switch (fmt) {
         case FMT_BF16: return unp_t<FMT_BF16, 64>(N, K, w, out, ldo, f16, s);
         case FMT_W8:
