@@ -118,26 +118,67 @@ __global__ void pf_rownorm_kernel(const uint16_t* x, float* r, const float* gamm
     }
 }
 
-// causal depthwise conv1d + SiLU over the frames (zero history); dt = softplus(dt_raw + bias);
-// the last W-1 raw pre-conv rows are written to the conv ring (frame t in slot t mod W)
-__global__ void pf_conv_kernel(const uint16_t* zx, int zxw, int T, int E, int Cx, int H, int W, const float* conv_w,
-                               const float* conv_b, const float* dt_bias, float* xc, uint16_t* xc16, float* dt,
-                               uint16_t* ring) {
-    const int t = blockIdx.x;
-    const uint16_t* xBC = zx + E;
-    for (int c = threadIdx.x; c < Cx; c += blockDim.x) {
-        float acc = conv_b[c];
-        for (int k = 0; k < W; ++k) {
-            const int tt = t - (W - 1) + k;
-            if (tt >= 0) acc += conv_w[c * W + k] * bf16_bits_to_f(xBC[(size_t)tt * zxw + c]);
-        }
+// causal depthwise conv1d + SiLU over the frames (zero history), a tile of 64 frames x 256
+// channels per CTA: each thread keeps its channel's W taps and last W-1 inputs in registers, so
+// every input row is read once and every access is coalesced across the channels.  The last W-1
+// raw pre-conv rows go to the conv ring (frame t in slot t mod W).
+static constexpr int kConvTF = 64;
+
+__global__ void __launch_bounds__(256) pf_conv_kernel(const uint16_t* __restrict__ zx, int zxw, int T, int E, int Cx,
+                                                      int W, const float* __restrict__ conv_w,
+                                                      const float* __restrict__ conv_b, float* __restrict__ xc,
+                                                      uint16_t* __restrict__ xc16, uint16_t* __restrict__ ring) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= Cx) return;
+    const int t0 = blockIdx.y * kConvTF, t1 = min(T, t0 + kConvTF);
+    const uint16_t* col = zx + E + c;
+    float w[8], hist[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        w[k] = k < W ? conv_w[c * W + k] : 0.0f;
+        const int tt = t0 - (W - 1) + k;
+        hist[k] = (k < W - 1 && tt >= 0) ? bf16_bits_to_f(col[(size_t)tt * zxw]) : 0.0f;
+    }
+    const float bias = conv_b[c];
+    constexpr int U = 8;   // frames whose inputs are loaded together
+    for (int tb = t0; tb < t1; tb += U) {
+      uint16_t raws[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) raws[u] = tb + u < t1 ? col[(size_t)(tb + u) * zxw] : (uint16_t)0;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = tb + u;
+        if (t >= t1) break;
+        const uint16_t raw = raws[u];
+        const float xv = bf16_bits_to_f(raw);
+        float acc = bias;
+#pragma unroll
+        for (int k = 0; k < 7; ++k)
+            if (k < W - 1) acc += w[k] * hist[k];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (k == W - 1) acc += w[k] * xv;
+#pragma unroll
+        for (int k = 0; k < 7; ++k)
+            if (k < W - 2) hist[k] = hist[k + 1];
+#pragma unroll
+        for (int k = 0; k < 7; ++k)
+            if (k == W - 2) hist[k] = xv;
         const float v = silu_f(acc);
         xc[(size_t)t * Cx + c] = v;
         xc16[(size_t)t * Cx + c] = f16_bits(v);
-        if (t >= T - (W - 1)) ring[(size_t)(t % W) * Cx + c] = xBC[(size_t)t * zxw + c];
+        if (t >= T - (W - 1)) ring[(size_t)(t % W) * Cx + c] = raw;
+      }
     }
-    for (int h = threadIdx.x; h < H; h += blockDim.x)
-        dt[(size_t)t * H + h] = softplus_f(bf16_bits_to_f(zx[(size_t)t * zxw + E + Cx + h]) + dt_bias[h]);
+}
+
+// dt = softplus(dt_raw + dt_bias) for every frame and head
+__global__ void pf_dt_kernel(const uint16_t* __restrict__ zx, int zxw, int T, int off, int H,
+                             const float* __restrict__ dt_bias, float* __restrict__ dt) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)T * H) return;
+    const int t = (int)(i / H), h = (int)(i % H);
+    dt[i] = softplus_f(bf16_bits_to_f(zx[(size_t)t * zxw + off + h]) + dt_bias[h]);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -252,30 +293,27 @@ __global__ void pf_ssd_scan_kernel(const float* schunk, const float* lam, int T,
     ssm_out[idx] = s;
 }
 
-// v = y * silu(z); per row and norm group: act = bf16(v * rsqrt(mean(v^2) + eps) * gamma)
-__global__ void pf_gated_norm_kernel(const float* y, const uint16_t* zx, int zxw, const float* gnorm, int E, int NG,
-                                     float eps, uint16_t* act, int ld, int f16) {
-    const int t = blockIdx.x, q = blockIdx.y;
+// v = y * silu(z); per row and norm group: act = bf16(v * rsqrt(mean(v^2) + eps) * gamma).
+// CTA = one frame, one warp per norm group (warp-level reductions only)
+__global__ void pf_gated_norm_kernel(const float* __restrict__ y, const uint16_t* __restrict__ zx, int zxw,
+                                     const float* __restrict__ gnorm, int E, int NG, float eps,
+                                     uint16_t* __restrict__ act, int ld, int f16) {
+    const int t = blockIdx.x, q = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (q >= NG) return;
     const int gs = E / NG, c0 = q * gs;
-    __shared__ float red[32];
+    const float* yr = y + (size_t)t * E;
+    const uint16_t* zr = zx + (size_t)t * zxw;
     float ss = 0.0f;
-    for (int c = c0 + threadIdx.x; c < c0 + gs; c += blockDim.x) {
-        const float v = y[(size_t)t * E + c] * silu_f(bf16_bits_to_f(zx[(size_t)t * zxw + c]));
+#pragma unroll 4
+    for (int c = c0 + lane; c < c0 + gs; c += 32) {
+        const float v = yr[c] * silu_f(bf16_bits_to_f(zr[c]));
         ss += v * v;
     }
     ss = warp_sum(ss);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        float s = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
-        s = warp_sum(s);
-        if (threadIdx.x == 0) red[0] = rsqrtf(s / gs + eps);
-    }
-    __syncthreads();
-    const float ginv = red[0];
-    for (int c = c0 + threadIdx.x; c < c0 + gs; c += blockDim.x) {
-        const float v = y[(size_t)t * E + c] * silu_f(bf16_bits_to_f(zx[(size_t)t * zxw + c]));
-        const float u = v * ginv * gnorm[c];
+    const float ginv = rsqrtf(ss / gs + eps);
+#pragma unroll 4
+    for (int c = c0 + lane; c < c0 + gs; c += 32) {
+        const float u = yr[c] * silu_f(bf16_bits_to_f(zr[c])) * ginv * gnorm[c];
         act[(size_t)t * ld + c] = f16 ? act_bits<true>(u) : act_bits<false>(u);
     }
 }
@@ -360,8 +398,10 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
                                          (int)SL.total);
     if (e != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(m.ring, 0, (size_t)W * Cx * 2, s)) != cudaSuccess) return e;
-    pf_conv_kernel<<<T, 256, 0, s>>>(m.zx, zxw, T, E, Cx, H, W, Lw.conv_w, Lw.conv_b, Lw.dt_bias, m.xc, m.xc16, m.dt,
-                                     m.ring);
+    if (W > 8 || m.NG > 32) return cudaErrorNotSupported;
+    pf_conv_kernel<<<dim3((Cx + 255) / 256, (T + kConvTF - 1) / kConvTF), 256, 0, s>>>(m.zx, zxw, T, E, Cx, W, Lw.conv_w,
+                                                                                       Lw.conv_b, m.xc, m.xc16, m.ring);
+    pf_dt_kernel<<<(unsigned)(((long long)T * H + 255) / 256), 256, 0, s>>>(m.zx, zxw, T, E + Cx, H, Lw.dt_bias, m.dt);
     const size_t st_smem = (size_t)kStJ * (P + N) * 4;
     const dim3 sg(nch, H);
     if (P <= 80 && P > 64 && N <= 128 && N > 112)
@@ -377,7 +417,7 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
     pf_ssd_scan_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(m.schunk, m.lam, T, H, P, N, m.sin16, m.ssm);
     pf_ssd_out_mma_kernel<<<dim3(nch, m.G, kChunk / kSsdTi), 256, SL.total, s>>>(m.xc, m.xc16, m.dt, m.lam, m.sin16, Lw.D, T, H,
                                                                                  P, N, m.G, E, Cx, m.y);
-    pf_gated_norm_kernel<<<dim3(T, m.NG), 256, 0, s>>>(m.y, m.zx, zxw, Lw.gnorm, E, m.NG, m.eps, m.act, m.act_ld,
+    pf_gated_norm_kernel<<<T, 32 * m.NG, 0, s>>>(m.y, m.zx, zxw, Lw.gnorm, E, m.NG, m.eps, m.act, m.act_ld,
                                                        m.f16);
     return cudaGetLastError();
 }

@@ -36,57 +36,48 @@ VC_DEV uint16_t f16_bits(float v) {
 }
 
 // ------------------------------------------------------------------------------------------
-// chunked SSD, outputs.  CTA = (chunk c, B/C group g, 64-row tile of the chunk).  The group's
-// C.B^T block (64 x j) is computed once and reused by the H/G heads of the group.  The
-// intra-chunk products take fp16 operands (C, B, the decay-weighted C.B^T and x: 11-bit
-// significands; y is heavy-tailed, and bf16's 8 bits leave its largest elements ~10% of the
-// RMS off), the entering-state product bf16 operands (the state's range):
+// chunked SSD, outputs.  CTA = (chunk c, B/C group g, 64-row tile of the chunk), two CTAs per
+// SM.  The group's C.B^T block (64 x j) is formed once (fragments read straight from the fp16
+// image of the conv outputs, which the chunk's CTAs share through L2) and kept in shared memory
+// as fp16; the H/G heads of the group then reuse it:
 //   y_i[p] = sum_{j<=i} (C_i.B_j) exp(Lam_i - Lam_j) dt_j x_j[p]      (intra-chunk, W . X)
 //          + exp(Lam_i) sum_n C_i[n] S_in[p][n]                        (state entering the chunk)
 //          + D x_i[p]
+// The decay-weighted W fragments are built in registers from the fp16 C.B^T, so only x is
+// staged per head.  The intra-chunk products take fp16 operands (C, B, W and x: 11-bit
+// significands; y is heavy-tailed, and bf16's 8 bits leave its largest elements ~10% of the
+// RMS off), the entering-state product bf16 operands (the state's range).
 // ------------------------------------------------------------------------------------------
 static constexpr int kSsdChunk = 256;
 static constexpr int kSsdTi = 64;
 
+VC_DEV uint32_t pack_f16x2(float lo, float hi) { return (uint32_t)f16_bits(lo) | ((uint32_t)f16_bits(hi) << 16); }
+
 struct SsdLayout {
-    int sc, sb, scb, sw, ss, sx;               // row strides (elements); x is stored [j][p]
-    size_t off_c, off_c2, off_b, off_w, off_s, off_cb, off_x, off_l, total;
+    int scb, sx;                 // row strides (elements): C.B^T fp16 [64][scb], x fp16 [j][sx]
+    size_t off_cb, off_x, off_l, total;
 };
 
 __host__ __device__ inline SsdLayout ssd_layout(int N, int P) {
+    (void)N;
     SsdLayout L{};
-    L.sc = N + 8;
-    L.sb = N + 8;
-    L.scb = kSsdChunk + 4;
-    L.sw = kSsdChunk + 8;
-    L.ss = N + 8;
+    L.scb = kSsdChunk + 8;
     L.sx = P + 8;
     auto a16 = [](size_t v) { return (v + 15) / 16 * 16; };
-    const size_t rc = a16((size_t)kSsdTi * L.sc * 2);
-    const size_t rb_b = (size_t)kSsdChunk * L.sb * 2;
-    const size_t rw = a16((size_t)kSsdTi * L.sw * 2);
-    const size_t rs = a16((size_t)P * L.ss * 2);
-    const size_t rb = a16(rb_b > rw + rs ? rb_b : rw + rs);   // B is dead once C.B^T is formed
-    L.off_c = 0;
-    L.off_c2 = rc;
-    L.off_b = 2 * rc;
-    L.off_w = 2 * rc;
-    L.off_s = 2 * rc + rw;
-    L.off_cb = 2 * rc + rb;
-    L.off_x = L.off_cb + a16((size_t)kSsdTi * L.scb * 4);
+    L.off_cb = 0;
+    L.off_x = a16((size_t)kSsdTi * L.scb * 2);
     L.off_l = L.off_x + a16((size_t)kSsdChunk * L.sx * 2);
     L.total = L.off_l + 2 * kSsdChunk * 4;
     return L;
 }
 
-__global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __restrict__ xc,
-                                                             const uint16_t* __restrict__ xc16,
-                                                             const float* __restrict__ dt,
-                                                             const float* __restrict__ lam,
-                                                             const uint16_t* __restrict__ sin16,
-                                                             const float* __restrict__ Dv,
-                                                             int T, int H, int P, int N, int G, int E, int Cx,
-                                                             float* __restrict__ y) {
+__global__ void __launch_bounds__(256, 2) pf_ssd_out_mma_kernel(const float* __restrict__ xc,
+                                                                const uint16_t* __restrict__ xc16,
+                                                                const float* __restrict__ dt,
+                                                                const float* __restrict__ lam,
+                                                                const uint16_t* __restrict__ sin16,
+                                                                const float* __restrict__ Dv, int T, int H, int P,
+                                                                int N, int G, int E, int Cx, float* __restrict__ y) {
     extern __shared__ __align__(16) unsigned char smraw[];
     const int c = blockIdx.x, g = blockIdx.y, it = blockIdx.z;
     const int t0 = c * kSsdChunk, len = min(kSsdChunk, T - t0);
@@ -95,48 +86,19 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
     const int i1 = min(len, i0 + kSsdTi);
     const int jn = i1;                       // frames j < jn are visible to some row of the tile
     const int jn16 = (jn + 15) & ~15;
-    const int jn32 = (jn + 31) & ~31;
     const SsdLayout L = ssd_layout(N, P);
-    uint16_t* Cs = reinterpret_cast<uint16_t*>(smraw + L.off_c);     // C rows, fp16
-    uint16_t* Cb = reinterpret_cast<uint16_t*>(smraw + L.off_c2);    // C rows, bf16
-    uint16_t* Bs = reinterpret_cast<uint16_t*>(smraw + L.off_b);
-    uint16_t* Ws = reinterpret_cast<uint16_t*>(smraw + L.off_w);
-    uint16_t* Sb = reinterpret_cast<uint16_t*>(smraw + L.off_s);
-    float* CBs = reinterpret_cast<float*>(smraw + L.off_cb);
+    uint16_t* CB = reinterpret_cast<uint16_t*>(smraw + L.off_cb);    // C_i.B_j, fp16 [64][scb]
     uint16_t* Xs = reinterpret_cast<uint16_t*>(smraw + L.off_x);     // x rows of the head, fp16 [j][p]
     float* lam_s = reinterpret_cast<float*>(smraw + L.off_l);
     float* dts = lam_s + kSsdChunk;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-    const size_t coff = (size_t)t0 * Cx + E + (size_t)G * N + (size_t)g * N;
-    const size_t boff = (size_t)t0 * Cx + E + (size_t)g * N;
+    const uint16_t* C16 = xc16 + (size_t)t0 * Cx + E + (size_t)G * N + (size_t)g * N;
+    const uint16_t* B16 = xc16 + (size_t)t0 * Cx + E + (size_t)g * N;
+    const float* C32 = xc + (size_t)t0 * Cx + E + (size_t)G * N + (size_t)g * N;
     const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-    const int n8 = N / 8;
+    auto ldg32 = [](const uint16_t* p) { return __ldg(reinterpret_cast<const unsigned int*>(p)); };
 
-    // 1. the group's C rows of the tile (fp16 copies, and bf16 for the entering-state product)
-    //    and B rows 0..jn-1 (fp16), zero padded; 16-byte copies from the fp16 image of xc
-#pragma unroll 4
-    for (int idx = tid; idx < kSsdTi * n8; idx += blockDim.x) {
-        const int ii = idx / n8, c8 = idx - ii * n8;
-        const bool ok = i0 + ii < i1;
-        *reinterpret_cast<uint4*>(Cs + ii * L.sc + c8 * 8) =
-            ok ? *reinterpret_cast<const uint4*>(xc16 + coff + (size_t)(i0 + ii) * Cx + c8 * 8) : z4;
-        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-        if (ok) {
-            v0 = *reinterpret_cast<const float4*>(xc + coff + (size_t)(i0 + ii) * Cx + c8 * 8);
-            v1 = *reinterpret_cast<const float4*>(xc + coff + (size_t)(i0 + ii) * Cx + c8 * 8 + 4);
-        }
-        *reinterpret_cast<uint4*>(Cb + ii * L.sc + c8 * 8) =
-            make_uint4(pack_bf16x2(v0.x, v0.y), pack_bf16x2(v0.z, v0.w), pack_bf16x2(v1.x, v1.y), pack_bf16x2(v1.z, v1.w));
-    }
-#pragma unroll 4
-    for (int idx = tid; idx < jn32 * n8; idx += blockDim.x) {
-        const int j = idx / n8, c8 = idx - j * n8;
-        *reinterpret_cast<uint4*>(Bs + j * L.sb + c8 * 8) =
-            j < jn ? *reinterpret_cast<const uint4*>(xc16 + boff + (size_t)j * Cx + c8 * 8) : z4;
-    }
-    __syncthreads();
-
-    // 2. CB[ii][j] = C_i . B_j: warp w forms columns 32w .. 32w+31 of all 64 rows
+    // 1. CB[ii][j] = C_i . B_j: warp w forms columns 32w .. 32w+31 of all 64 rows
     if (32 * warp < jn) {
         float acc[4][4][4];
 #pragma unroll
@@ -149,16 +111,19 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
             uint32_t af[4][4];
 #pragma unroll
             for (int mt = 0; mt < 4; ++mt) {
-                const uint16_t* r = Cs + (mt * 16 + gq) * L.sc + k0 + 2 * tq;
-                af[mt][0] = lds32(r);
-                af[mt][1] = lds32(r + 8 * L.sc);
-                af[mt][2] = lds32(r + 8);
-                af[mt][3] = lds32(r + 8 * L.sc + 8);
+                const int ra = i0 + mt * 16 + gq, rb = ra + 8;
+                const uint16_t* pa = C16 + (size_t)ra * Cx + k0 + 2 * tq;
+                const uint16_t* pb = C16 + (size_t)rb * Cx + k0 + 2 * tq;
+                af[mt][0] = ra < i1 ? ldg32(pa) : 0u;
+                af[mt][1] = rb < i1 ? ldg32(pb) : 0u;
+                af[mt][2] = ra < i1 ? ldg32(pa + 8) : 0u;
+                af[mt][3] = rb < i1 ? ldg32(pb + 8) : 0u;
             }
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                const uint16_t* r = Bs + (32 * warp + nt * 8 + gq) * L.sb + k0 + 2 * tq;
-                const uint32_t b0 = lds32(r), b1 = lds32(r + 8);
+                const int j = 32 * warp + nt * 8 + gq;
+                const uint16_t* pbj = B16 + (size_t)j * Cx + k0 + 2 * tq;
+                const uint32_t b0 = j < jn ? ldg32(pbj) : 0u, b1 = j < jn ? ldg32(pbj + 8) : 0u;
 #pragma unroll
                 for (int mt = 0; mt < 4; ++mt) mma_f16(acc[mt][nt], af[mt], b0, b1, acc[mt][nt]);
             }
@@ -167,14 +132,13 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
         for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                float* r = CBs + (mt * 16 + gq) * L.scb + 32 * warp + nt * 8 + 2 * tq;
-                *reinterpret_cast<float2*>(r) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
-                *reinterpret_cast<float2*>(r + 8 * L.scb) = make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+                uint16_t* r = CB + (mt * 16 + gq) * L.scb + 32 * warp + nt * 8 + 2 * tq;
+                *reinterpret_cast<uint32_t*>(r) = pack_f16x2(acc[mt][nt][0], acc[mt][nt][1]);
+                *reinterpret_cast<uint32_t*>(r + 8 * L.scb) = pack_f16x2(acc[mt][nt][2], acc[mt][nt][3]);
             }
     }
-    __syncthreads();
 
-    // 3. the heads of the group
+    // 2. the heads of the group
     const int hpg = H / G;
     const int nt8 = P / 8;
     const int wm = warp & 3, wn = warp >> 2;
@@ -182,52 +146,47 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
     const int q0 = wn * half;
     const int qn = min(nt8, q0 + half) - q0;
     const int kend = min(jn16, i0 + wm * 16 + 16);   // rows of this warp see j < i0 + 16 (wm + 1)
+    const int lk = (lane & 7) + 8 * ((lane >> 3) & 1);
+    const int lp = 8 * (lane >> 4);
+    const int p8 = P / 8;
+    const int ia = wm * 16 + gq, ib = ia + 8;          // the lane's two rows within the tile
     for (int hh = 0; hh < hpg; ++hh) {
         const int h = g * hpg + hh;
+        __syncthreads();   // C.B^T ready (first head) / previous head's x consumed
         for (int j = tid; j < jn16; j += blockDim.x) {
             lam_s[j] = j < jn ? lam[(size_t)(t0 + j) * H + h] : 0.0f;
             dts[j] = j < jn ? dt[(size_t)(t0 + j) * H + h] : 0.0f;
         }
-        const float* xh = xc + (size_t)t0 * Cx + (size_t)h * P;
         const uint16_t* xh16 = xc16 + (size_t)t0 * Cx + (size_t)h * P;
-        const int p8 = P / 8;
 #pragma unroll 4
         for (int idx = tid; idx < jn16 * p8; idx += blockDim.x) {
             const int j = idx / p8, c8 = idx - j * p8;
             *reinterpret_cast<uint4*>(Xs + j * L.sx + c8 * 8) =
                 j < jn ? *reinterpret_cast<const uint4*>(xh16 + (size_t)j * Cx + c8 * 8) : z4;
         }
-        const uint16_t* Sh = sin16 + ((size_t)c * H + h) * P * N;
-#pragma unroll 4
-        for (int idx = tid; idx < P * n8; idx += blockDim.x) {
-            const int p = idx / n8, c8 = idx - p * n8;
-            *reinterpret_cast<uint4*>(Sb + p * L.ss + c8 * 8) = *reinterpret_cast<const uint4*>(Sh + (size_t)p * N + c8 * 8);
-        }
         __syncthreads();
-        for (int idx = tid; idx < kSsdTi * jn16; idx += blockDim.x) {
-            const int ii = idx / jn16, j = idx - ii * jn16;
-            const int i = i0 + ii;
-            float v = 0.0f;
-            if (i < i1 && j <= i) v = CBs[ii * L.scb + j] * __expf(lam_s[i] - lam_s[j]) * dts[j];
-            Ws[ii * L.sw + j] = f16_bits(v);
-        }
-        __syncthreads();
+        const float la = lam_s[min(i0 + ia, jn - 1)], lb = lam_s[min(i0 + ib, jn - 1)];
         float acc[8][4], acc2[8][4];
 #pragma unroll
         for (int q = 0; q < 8; ++q)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[q][e] = acc2[q][e] = 0.0f;
-        // x fragments by transposing 8x8 loads of the [j][p] rows: lanes 0-7 rows k0..k0+7,
-        // 8-15 rows k0+8..k0+15 (columns p0..p0+7), 16-31 the same rows at columns p0+8..p0+15
-        const int lk = (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int lp = 8 * (lane >> 4);
         for (int k0 = 0; k0 < kend; k0 += 16) {
+            // W fragments: W[i][j] = CB[i][j] exp(Lam_i - Lam_j) dt_j for j <= i < i1, else 0
             uint32_t af[4];
-            const uint16_t* r = Ws + (wm * 16 + gq) * L.sw + k0 + 2 * tq;
-            af[0] = lds32(r);
-            af[1] = lds32(r + 8 * L.sw);
-            af[2] = lds32(r + 8);
-            af[3] = lds32(r + 8 * L.sw + 8);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int ii = (e & 1) ? ib : ia;
+                const int j = k0 + 2 * tq + 8 * (e >> 1);
+                const float li = (e & 1) ? lb : la;
+                const __half2 cb = *reinterpret_cast<const __half2*>(CB + ii * L.scb + j);
+                const float2 lj = *reinterpret_cast<const float2*>(lam_s + j);
+                const float2 dj = *reinterpret_cast<const float2*>(dts + j);
+                const int i = i0 + ii;
+                const float w0 = (i < i1 && j <= i) ? __low2float(cb) * __expf(li - lj.x) * dj.x : 0.0f;
+                const float w1 = (i < i1 && j + 1 <= i) ? __high2float(cb) * __expf(li - lj.y) * dj.y : 0.0f;
+                af[e] = pack_f16x2(w0, w1);
+            }
 #pragma unroll
             for (int q = 0; q < 8; q += 2)
                 if (q < qn) {
@@ -237,24 +196,30 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
                     if (q + 1 < qn) mma_f16(acc[q + 1], af, xb[2], xb[3], acc[q + 1]);
                 }
         }
+        // C . S_in^T: C rows (bf16 from the fp32 conv outputs), S_in rows p (bf16) from L2
+        const uint16_t* Sh = sin16 + ((size_t)c * H + h) * P * N;
         for (int k0 = 0; k0 < N; k0 += 16) {
             uint32_t af[4];
-            const uint16_t* r = Cb + (wm * 16 + gq) * L.sc + k0 + 2 * tq;
-            af[0] = lds32(r);
-            af[1] = lds32(r + 8 * L.sc);
-            af[2] = lds32(r + 8);
-            af[3] = lds32(r + 8 * L.sc + 8);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int ii = (e & 1) ? ib : ia;
+                const int k = k0 + 2 * tq + 8 * (e >> 1);
+                float2 cv = make_float2(0.0f, 0.0f);
+                if (i0 + ii < i1) cv = __ldg(reinterpret_cast<const float2*>(C32 + (size_t)(i0 + ii) * Cx + k));
+                af[e] = pack_bf16x2(cv.x, cv.y);
+            }
 #pragma unroll
             for (int q = 0; q < 8; ++q)
                 if (q < qn) {
-                    const uint16_t* br = Sb + ((q0 + q) * 8 + gq) * L.ss + k0 + 2 * tq;
-                    mma_bf16(acc2[q], af, lds32(br), lds32(br + 8), acc2[q]);
+                    const uint16_t* br = Sh + (size_t)((q0 + q) * 8 + gq) * N + k0 + 2 * tq;
+                    mma_bf16(acc2[q], af, ldg32(br), ldg32(br + 8), acc2[q]);
                 }
         }
         const float Dh_ = Dv[h];
+        const float* xh = xc + (size_t)t0 * Cx + (size_t)h * P;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-            const int i = i0 + wm * 16 + gq + 8 * r;
+            const int i = i0 + (r ? ib : ia);
             if (i < i1) {
                 const float el = __expf(lam_s[i]);
                 const float* xi = xh + (size_t)i * Cx;
@@ -271,7 +236,6 @@ __global__ void __launch_bounds__(256) pf_ssd_out_mma_kernel(const float* __rest
                     }
             }
         }
-        __syncthreads();
     }
 }
 
