@@ -404,7 +404,14 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
     pf_dt_kernel<<<(unsigned)(((long long)T * H + 255) / 256), 256, 0, s>>>(m.zx, zxw, T, E + Cx, H, Lw.dt_bias, m.dt);
     const size_t st_smem = (size_t)kStJ * (P + N) * 4;
     const dim3 sg(nch, H);
-    if (P <= 80 && P > 64 && N <= 128 && N > 112)
+    const bool st_mma = N % 16 == 0 && N <= 128 && (P == 80 || P == 32);
+    const StateLayout STL = state_layout(N, P);
+    if (st_mma) {
+        auto kst = P == 80 ? pf_ssd_state_mma_kernel<5> : pf_ssd_state_mma_kernel<2>;
+        if ((e = cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STL.total)) != cudaSuccess)
+            return e;
+        kst<<<sg, 256, STL.total, s>>>(m.xc, m.dt, Lw.A_log, T, H, P, N, m.G, E, Cx, m.lam, m.schunk);
+    } else if (P <= 80 && P > 64 && N <= 128 && N > 112)
         pf_ssd_state_kernel<5, 8><<<sg, 256, st_smem, s>>>(m.xc, m.dt, Lw.A_log, T, H, P, N, m.G, E, Cx, m.lam,
                                                              m.schunk);
     else if (P <= 32 && N <= 16)

@@ -240,6 +240,169 @@ __global__ void __launch_bounds__(256, 2) pf_ssd_out_mma_kernel(const float* __r
 }
 
 // ------------------------------------------------------------------------------------------
+// chunked SSD, chunk states on tensor cores:  S_c[p][n] = sum_j (w_j x_j[p]) B_j[n],
+// w_j = exp(Lam_end - Lam_j) dt_j.  The state decode continues from must meet the fp32 bound, so
+// each operand is split into two fp16 halves (v = hi + lo, lo = v - hi) and the product is
+// hi.hi + hi.lo + lo.hi (the dropped lo.lo term is ~2^-22 of the product), accumulated in fp32.
+// CTA = (chunk, head); frames staged 64 at a time; warp w owns state columns 16 w .. 16 w + 15
+// (two n8 tiles) for all P rows (MT m16 tiles).  Both operands are loaded with transposing
+// 8x8 matrix loads from their natural [frame][channel] rows.
+// ------------------------------------------------------------------------------------------
+static constexpr int kStTile = 64;
+
+struct StateLayout {
+    int sx, sb;
+    size_t off_xh, off_xl, off_bh, off_bl, off_w, total;
+};
+
+__host__ __device__ inline StateLayout state_layout(int N, int P) {
+    StateLayout L{};
+    L.sx = P + 8;
+    L.sb = N + 8;
+    auto a16 = [](size_t v) { return (v + 15) / 16 * 16; };
+    const size_t rx = a16((size_t)kStTile * L.sx * 2), rb = a16((size_t)kStTile * L.sb * 2);
+    L.off_xh = 0;
+    L.off_xl = rx;
+    L.off_bh = 2 * rx;
+    L.off_bl = 2 * rx + rb;
+    L.off_w = 2 * rx + 2 * rb;
+    L.total = L.off_w + 2 * kSsdChunk * 4;
+    return L;
+}
+
+VC_DEV void split_f16(float v, uint16_t& hi, uint16_t& lo) {
+    hi = f16_bits(v);
+    const __half h = *reinterpret_cast<const __half*>(&hi);
+    lo = f16_bits(v - __half2float(h));
+}
+
+template <int MT>
+__global__ void __launch_bounds__(256) pf_ssd_state_mma_kernel(const float* __restrict__ xc, const float* __restrict__ dt,
+                                                               const float* __restrict__ A_log, int T, int H, int P,
+                                                               int N, int G, int E, int Cx, float* __restrict__ lam,
+                                                               float* __restrict__ schunk) {
+    extern __shared__ __align__(16) unsigned char smraw[];
+    const int c = blockIdx.x, h = blockIdx.y;
+    const int t0 = c * kSsdChunk, len = min(kSsdChunk, T - t0);
+    const int g = (int)((long long)h * G / H);
+    const StateLayout L = state_layout(N, P);
+    uint16_t* Xh = reinterpret_cast<uint16_t*>(smraw + L.off_xh);
+    uint16_t* Xl = reinterpret_cast<uint16_t*>(smraw + L.off_xl);
+    uint16_t* Bh = reinterpret_cast<uint16_t*>(smraw + L.off_bh);
+    uint16_t* Bl = reinterpret_cast<uint16_t*>(smraw + L.off_bl);
+    float* lam_s = reinterpret_cast<float*>(smraw + L.off_w);
+    float* w = lam_s + kSsdChunk;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    const float A = -expf(A_log[h]);
+    // inclusive scan of A*dt over the chunk (one warp)
+    if (warp == 0) {
+        float run = 0.0f;
+        for (int base = 0; base < len; base += 32) {
+            const int i = base + lane;
+            float v = i < len ? A * dt[(size_t)(t0 + i) * H + h] : 0.0f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            v += run;
+            if (i < len) lam_s[i] = v;
+            run = __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    __syncthreads();
+    const float lend = lam_s[len - 1];
+    for (int i = tid; i < len; i += blockDim.x) {
+        w[i] = expf(lend - lam_s[i]) * dt[(size_t)(t0 + i) * H + h];
+        lam[(size_t)(t0 + i) * H + h] = lam_s[i];
+    }
+    const int npairs = N / 16;   // pairs of n8 tiles
+    float acc[MT][2][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][q][e] = 0.0f;
+    const float* xh = xc + (size_t)t0 * Cx + (size_t)h * P;
+    const float* bg = xc + (size_t)t0 * Cx + E + (size_t)g * N;
+    const int P4 = P / 4, N4 = N / 4;
+    // A fragments (rows p, k = frame) from Xw[j][p]: lanes 0-7 frames 0-7 at p0, 8-15 frames 0-7 at
+    // p0 + 8, 16-23 frames 8-15 at p0, 24-31 frames 8-15 at p0 + 8
+    const int ar = (lane & 7) + 8 * (lane >> 4), ac = 8 * ((lane >> 3) & 1);
+    // B fragments (k = frame, n) from B[j][n]: lanes 0-7 frames 0-7, 8-15 frames 8-15 (n0),
+    // 16-31 the same frames at n0 + 8
+    const int br = (lane & 7) + 8 * ((lane >> 3) & 1), bc = 8 * (lane >> 4);
+    for (int jb = 0; jb < len; jb += kStTile) {
+        const int nj = min(kStTile, len - jb);
+        const int nj16 = (nj + 15) & ~15;
+        __syncthreads();   // w ready (first tile) / previous tile consumed
+        for (int idx = tid; idx < nj16 * P4; idx += blockDim.x) {
+            const int j = idx / P4, q = idx - j * P4;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (j < nj) {
+                v = *reinterpret_cast<const float4*>(xh + (size_t)(jb + j) * Cx + 4 * q);
+                const float wj = w[jb + j];
+                v.x *= wj; v.y *= wj; v.z *= wj; v.w *= wj;
+            }
+            uint16_t hh[4], ll[4];
+            split_f16(v.x, hh[0], ll[0]); split_f16(v.y, hh[1], ll[1]);
+            split_f16(v.z, hh[2], ll[2]); split_f16(v.w, hh[3], ll[3]);
+            *reinterpret_cast<uint2*>(Xh + j * L.sx + 4 * q) =
+                make_uint2(hh[0] | ((uint32_t)hh[1] << 16), hh[2] | ((uint32_t)hh[3] << 16));
+            *reinterpret_cast<uint2*>(Xl + j * L.sx + 4 * q) =
+                make_uint2(ll[0] | ((uint32_t)ll[1] << 16), ll[2] | ((uint32_t)ll[3] << 16));
+        }
+        for (int idx = tid; idx < nj16 * N4; idx += blockDim.x) {
+            const int j = idx / N4, q = idx - j * N4;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (j < nj) v = *reinterpret_cast<const float4*>(bg + (size_t)(jb + j) * Cx + 4 * q);
+            uint16_t hh[4], ll[4];
+            split_f16(v.x, hh[0], ll[0]); split_f16(v.y, hh[1], ll[1]);
+            split_f16(v.z, hh[2], ll[2]); split_f16(v.w, hh[3], ll[3]);
+            *reinterpret_cast<uint2*>(Bh + j * L.sb + 4 * q) =
+                make_uint2(hh[0] | ((uint32_t)hh[1] << 16), hh[2] | ((uint32_t)hh[3] << 16));
+            *reinterpret_cast<uint2*>(Bl + j * L.sb + 4 * q) =
+                make_uint2(ll[0] | ((uint32_t)ll[1] << 16), ll[2] | ((uint32_t)ll[3] << 16));
+        }
+        __syncthreads();
+        if (warp < npairs) {
+            const int pr = warp;
+            for (int k0 = 0; k0 < nj16; k0 += 16) {
+                uint32_t bh[4], bl[4];
+                ldsm_x4_trans(bh, Bh + (k0 + br) * L.sb + 16 * pr + bc);
+                ldsm_x4_trans(bl, Bl + (k0 + br) * L.sb + 16 * pr + bc);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    uint32_t ah[4], al[4];
+                    ldsm_x4_trans(ah, Xh + (k0 + ar) * L.sx + 16 * mt + ac);
+                    ldsm_x4_trans(al, Xl + (k0 + ar) * L.sx + 16 * mt + ac);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        mma_f16(acc[mt][q], ah, bh[2 * q], bh[2 * q + 1], acc[mt][q]);
+                        mma_f16(acc[mt][q], ah, bl[2 * q], bl[2 * q + 1], acc[mt][q]);
+                        mma_f16(acc[mt][q], al, bh[2 * q], bh[2 * q + 1], acc[mt][q]);
+                    }
+                }
+            }
+        }
+    }
+    // write the chunk state (each warp its column pair; N <= 128, so every pair has one owner)
+    if (warp < npairs) {
+        float* S = schunk + ((size_t)c * H + h) * P * N;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int n = 16 * warp + 8 * q + 2 * tq;
+                const int p = 16 * mt + gq;
+                *reinterpret_cast<float2*>(S + (size_t)p * N + n) = make_float2(acc[mt][q][0], acc[mt][q][1]);
+                *reinterpret_cast<float2*>(S + (size_t)(p + 8) * N + n) = make_float2(acc[mt][q][2], acc[mt][q][3]);
+            }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
 // causal GQA attention (flash form): CTA = (64 query frames, q head), 4 warps of 16 rows; keys
 // and values in tiles of 64 frames from the KV cache rows the qkv projection just wrote; online
 // softmax in fp32 (exp2 with the 1/sqrt(Dh) scale folded in), P rounded to bf16 for P.V.
