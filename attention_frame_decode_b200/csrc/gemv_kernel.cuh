@@ -39,9 +39,15 @@ static constexpr int kRingBudget = 210 * 1024; // dynamic shared memory for the 
 // partition helpers (worker w of W owns flat blocks [w*T/W, (w+1)*T/W))
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ long long llmin(long long a, long long b) { return a < b ? a : b; }
-__device__ __forceinline__ long long part_begin(long long w, long long T, long long W) { return w * T / W; }
+// With T (W + 1) < 2^32 (every shape of the backbone) the same integer quotients are taken in
+// 32-bit arithmetic, which costs a fraction of a 64-bit division.
+__device__ __forceinline__ long long part_begin(long long w, long long T, long long W, bool s32) {
+    if (s32) return (long long)((uint32_t)w * (uint32_t)T / (uint32_t)W);
+    return w * T / W;
+}
 // largest worker whose range starts at or before block f (always a non-empty range)
-__device__ __forceinline__ long long part_owner(long long f, long long T, long long W) {
+__device__ __forceinline__ long long part_owner(long long f, long long T, long long W, bool s32) {
+    if (s32) return (long long)(((uint32_t)(f + 1) * (uint32_t)W + (uint32_t)T - 1u) / (uint32_t)T) - 1;
     return ((f + 1) * W + T - 1) / T - 1;
 }
 
@@ -176,7 +182,8 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
     const bool idle = wl >= Wm;
     // block indices fit in 32 bits (at most a few 10^5 blocks per matrix); positions advance
     // incrementally so the hot loop has no integer division
-    const int f0 = idle ? 0 : (int)part_begin(wl, T, Wm), f1 = idle ? 0 : (int)part_begin(wl + 1, T, Wm);
+    const bool s32 = (unsigned long long)T * (unsigned long long)(Wm + 1) < (1ull << 32);
+    const int f0 = idle ? 0 : (int)part_begin(wl, T, Wm, s32), f1 = idle ? 0 : (int)part_begin(wl + 1, T, Wm, s32);
     const int bps = L.bps;
     const int nstages = (f1 - f0 + bps - 1) / bps;
     const int KT = M.KT;
@@ -353,7 +360,8 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
 
     // a unit leaves this worker: finish it here or hand a partial to the last contributor
     auto flush = [&](int u) {
-        const long long lo = part_owner((long long)u * M.KT, T, Wm), hi = part_owner((long long)(u + 1) * M.KT - 1, T, Wm);
+        const long long lo = part_owner((long long)u * M.KT, T, Wm, s32),
+                        hi = part_owner((long long)(u + 1) * M.KT - 1, T, Wm, s32);
         if (lo == hi) {
             epilogue(u, acc);
             return;
@@ -417,7 +425,7 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
             for (int q = 0; q < 2; ++q) {
                 const long long w2 = w0 + q;
                 if (w2 > hi) break;
-                const long long fu = part_begin(w2, T, Wm) / M.KT;
+                const long long fu = part_begin(w2, T, Wm, s32) / M.KT;
                 const float* p = args.partials + ((size_t)(wbase + w2) * 2 + (u == fu ? 0 : 1)) * (R * NT * 128);
 #pragma unroll
                 for (int rj = 0; rj < R * NT; ++rj) x[q][rj] = __ldcg(reinterpret_cast<const float4*>(p + (rj * 32 + lane) * 4));

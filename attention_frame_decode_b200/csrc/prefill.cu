@@ -124,10 +124,12 @@ __global__ void pf_rownorm_kernel(const uint16_t* x, float* r, const float* gamm
 // raw pre-conv rows go to the conv ring (frame t in slot t mod W).
 static constexpr int kConvTF = 64;
 
+template <int WC>   // conv width when fixed at compile time (the backbone's 4), else 0: runtime W <= 8
 __global__ void __launch_bounds__(256) pf_conv_kernel(const uint16_t* __restrict__ zx, int zxw, int T, int E, int Cx,
-                                                      int W, const float* __restrict__ conv_w,
+                                                      int Wr, const float* __restrict__ conv_w,
                                                       const float* __restrict__ conv_b, float* __restrict__ xc,
                                                       uint16_t* __restrict__ xc16, uint16_t* __restrict__ ring) {
+    const int W = WC ? WC : Wr;
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= Cx) return;
     const int t0 = blockIdx.y * kConvTF, t1 = min(T, t0 + kConvTF);
@@ -399,8 +401,11 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(m.ring, 0, (size_t)W * Cx * 2, s)) != cudaSuccess) return e;
     if (W > 8 || m.NG > 32) return cudaErrorNotSupported;
-    pf_conv_kernel<<<dim3((Cx + 255) / 256, (T + kConvTF - 1) / kConvTF), 256, 0, s>>>(m.zx, zxw, T, E, Cx, W, Lw.conv_w,
-                                                                                       Lw.conv_b, m.xc, m.xc16, m.ring);
+    const dim3 cg((Cx + 255) / 256, (T + kConvTF - 1) / kConvTF);
+    if (W == 4)
+        pf_conv_kernel<4><<<cg, 256, 0, s>>>(m.zx, zxw, T, E, Cx, W, Lw.conv_w, Lw.conv_b, m.xc, m.xc16, m.ring);
+    else
+        pf_conv_kernel<0><<<cg, 256, 0, s>>>(m.zx, zxw, T, E, Cx, W, Lw.conv_w, Lw.conv_b, m.xc, m.xc16, m.ring);
     pf_dt_kernel<<<(unsigned)(((long long)T * H + 255) / 256), 256, 0, s>>>(m.zx, zxw, T, E + Cx, H, Lw.dt_bias, m.dt);
     const size_t st_smem = (size_t)kStJ * (P + N) * 4;
     const dim3 sg(nch, H);

@@ -54,8 +54,8 @@ static constexpr int kSsdTi = 64;
 VC_DEV uint32_t pack_f16x2(float lo, float hi) { return (uint32_t)f16_bits(lo) | ((uint32_t)f16_bits(hi) << 16); }
 
 struct SsdLayout {
-    int scb, sx;                 // row strides (elements): C.B^T fp16 [64][scb], x fp16 [j][sx]
-    size_t off_cb, off_x, off_l, total;
+    int scb, sx, sc;             // row strides (elements): C.B^T fp16 [64][scb], x fp16 [j][sx], C bf16 [64][sc]
+    size_t off_cb, off_x, off_c, off_l, total;
 };
 
 __host__ __device__ inline SsdLayout ssd_layout(int N, int P) {
@@ -63,10 +63,12 @@ __host__ __device__ inline SsdLayout ssd_layout(int N, int P) {
     SsdLayout L{};
     L.scb = kSsdChunk + 8;
     L.sx = P + 8;
+    L.sc = N + 8;
     auto a16 = [](size_t v) { return (v + 15) / 16 * 16; };
     L.off_cb = 0;
     L.off_x = a16((size_t)kSsdTi * L.scb * 2);
-    L.off_l = L.off_x + a16((size_t)kSsdChunk * L.sx * 2);
+    L.off_c = L.off_x + a16((size_t)kSsdChunk * L.sx * 2);
+    L.off_l = L.off_c + a16((size_t)kSsdTi * L.sc * 2);
     L.total = L.off_l + 2 * kSsdChunk * 4;
     return L;
 }
@@ -89,6 +91,7 @@ __global__ void __launch_bounds__(256, 2) pf_ssd_out_mma_kernel(const float* __r
     const SsdLayout L = ssd_layout(N, P);
     uint16_t* CB = reinterpret_cast<uint16_t*>(smraw + L.off_cb);    // C_i.B_j, fp16 [64][scb]
     uint16_t* Xs = reinterpret_cast<uint16_t*>(smraw + L.off_x);     // x rows of the head, fp16 [j][p]
+    uint16_t* Cb = reinterpret_cast<uint16_t*>(smraw + L.off_c);     // C rows of the tile, bf16 [64][sc]
     float* lam_s = reinterpret_cast<float*>(smraw + L.off_l);
     float* dts = lam_s + kSsdChunk;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
@@ -98,6 +101,13 @@ __global__ void __launch_bounds__(256, 2) pf_ssd_out_mma_kernel(const float* __r
     const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
     auto ldg32 = [](const uint16_t* p) { return __ldg(reinterpret_cast<const unsigned int*>(p)); };
 
+    // 0. the tile's C rows as bf16, for the entering-state product of every head
+    for (int idx = tid; idx < kSsdTi * (N / 4); idx += blockDim.x) {
+        const int ii = idx / (N / 4), q = idx - ii * (N / 4);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i0 + ii < i1) v = __ldg(reinterpret_cast<const float4*>(C32 + (size_t)(i0 + ii) * Cx + 4 * q));
+        *reinterpret_cast<uint2*>(Cb + ii * L.sc + 4 * q) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+    }
     // 1. CB[ii][j] = C_i . B_j: warp w forms columns 32w .. 32w+31 of all 64 rows
     if (32 * warp < jn) {
         float acc[4][4][4];
@@ -196,18 +206,15 @@ __global__ void __launch_bounds__(256, 2) pf_ssd_out_mma_kernel(const float* __r
                     if (q + 1 < qn) mma_f16(acc[q + 1], af, xb[2], xb[3], acc[q + 1]);
                 }
         }
-        // C . S_in^T: C rows (bf16 from the fp32 conv outputs), S_in rows p (bf16) from L2
+        // C . S_in^T: C rows (bf16, staged once), S_in rows p (bf16) from L2
         const uint16_t* Sh = sin16 + ((size_t)c * H + h) * P * N;
         for (int k0 = 0; k0 < N; k0 += 16) {
             uint32_t af[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int ii = (e & 1) ? ib : ia;
-                const int k = k0 + 2 * tq + 8 * (e >> 1);
-                float2 cv = make_float2(0.0f, 0.0f);
-                if (i0 + ii < i1) cv = __ldg(reinterpret_cast<const float2*>(C32 + (size_t)(i0 + ii) * Cx + k));
-                af[e] = pack_bf16x2(cv.x, cv.y);
-            }
+            const uint16_t* r = Cb + ia * L.sc + k0 + 2 * tq;
+            af[0] = lds32(r);
+            af[1] = lds32(r + 8 * L.sc);
+            af[2] = lds32(r + 8);
+            af[3] = lds32(r + 8 * L.sc + 8);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
                 if (q < qn) {
