@@ -80,8 +80,8 @@ def launches_per_step(cfg):
 # kernel and shape (profiles/gemv_mlp_shapes_bf16_w4.md, profiles/gemm_tc_prefill_4096x15680x4480.md);
 # None where no capture of the current kernel exists.
 TRAFFIC = {
-    "nano_bf16": 141.117440e6 + 4.171776e6,      # gemv bf16 15680 x 4480, B = 1
-    "nano_w4": 38.452480e6 + 0.0,                # gemv W4 g64 15680 x 4480, B = 1
+    "nano_bf16": 141.126400e6 + 4.253184e6,      # gemv bf16 15680 x 4480, B = 1
+    "nano_w4": 38.456576e6 + 0.0,                # gemv W4 g64 15680 x 4480, B = 1
     "nano_prefill": 241.034496e6 + 236.244736e6,  # tcgen05 GEMM 4096 x 15680 x 4480
 }
 
