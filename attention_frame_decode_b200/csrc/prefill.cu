@@ -1,8 +1,8 @@
 // prefill.cu -- opening-context prefill of one session: all T frames layer by layer.
 //
-// "system-prompt prefill, then the user's speech" ("NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM,
-// MLX", "Recipe"): before streaming, the backbone consumes a context of T frames at once.  Per
-// layer:
+// A streaming session takes in its prompt as one block before the caller's speech
+// ("NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM, MLX", "Recipe"): the backbone consumes a context of
+// T frames at once.  Per layer:
 //   pre-RMSNorm rows (act = bf16(r * gamma), inv_rms per row)
 //   Mamba-2 : in_proj GEMM (tcgen05) -> causal conv1d + SiLU over the frames (the last W-1 raw
 //             rows go to the session's conv ring) -> chunked SSD (Dao & Gu, "Transformers are
@@ -14,7 +14,8 @@
 //   attention: qkv GEMM (k, v written to the KV cache rows 0..T-1) -> causal GQA softmax
 //             attention -> o_proj GEMM + residual
 //   MLP      : up GEMM with squared ReLU -> down GEMM + residual
-// The SSD and attention run on fp32 CUDA cores; the projections (>95% of the FLOPs) on tcgen05.
+// The projections (>95% of the FLOPs) run on tcgen05; the chunked SSD and the causal attention on
+// warp-level MMA (prefill_mma.cuh); the scan over chunks, conv, norms in fp32 on CUDA cores.
 // The call (re)initialises the slot: the SSM state ends as the scan's final state, the conv
 // ring holds the last W-1 frames, KV rows 0..T-1 are written and ctx_len[slot] = T.
 #include <string.h>

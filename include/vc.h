@@ -4,7 +4,7 @@
  *
  * What it computes (sources: the pages' titles and sections):
  *   - "NemotronLabs VoiceChat" (SGLang-Omni cookbook), intro and "Request parameters": every
- *     80 ms frame advances the thinker, which emits one text token and one function token
+ *     80 ms frame advances the thinker, which yields a text token and a function token
  *     per frame and always decodes greedily; backbone and KV cache run in bf16
  *     ("Known limitations").
  *   - "NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM, MLX", intro and "Measurements": the LLM is
@@ -179,7 +179,7 @@ vc_status vc_step_host(vc_backbone* h, const void* x_host, int B, const int32_t*
 
 /* Prefill of T frames x bf16 [T][d_model] (device) into session `slot` -- the opening context a
  * streaming session consumes before its frames ("NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM,
- * MLX", Recipe: system-prompt prefill, then the user's speech).  The slot starts empty: whatever
+ * MLX", Recipe: the prompt is taken in as one block before the caller's speech).  The slot starts empty: whatever
  * it held is overwritten.  Mamba-2 layers run the chunked SSD (Dao & Gu, "Transformers are SSMs",
  * chunk 256) over the frames, attention layers causal GQA; the call writes the final SSM state,
  * the conv ring (the last W-1 frames' rows, frame t in slot t mod W, the other slot zero) and
