@@ -1,0 +1,39 @@
+"""The algorithmic byte and FLOP counts bench.py divides by (the roofline's numerator), checked
+against the per-step totals computed by hand from the layer shapes (d 4480; 27 Mamba-2 layers with
+in_proj 22656 x 4480 and out_proj 4480 x 10240; 4 attention layers with qkv 7168 x 4480 and
+o 4480 x 5120; 25 MLP layers 15680 x 4480 and back; two bf16 heads 131072 x 4480)."""
+import pytest
+
+import bench
+import synth
+
+
+def test_linear_weight_count():
+    cfg = synth.CONFIGS["nano_bf16"]
+    n = sum(N * K for l in range(cfg.n_layers) for _, N, K in synth.linear_shapes(cfg, l))
+    assert n == 27 * (22656 * 4480 + 4480 * 10240) + 4 * (7168 * 4480 + 4480 * 5120) + 25 * 2 * 15680 * 4480
+
+
+@pytest.mark.parametrize("name,gb", [("nano_bf16", 17.95), ("nano_w4", 6.69), ("nano_w3", 5.71)])
+def test_step_bytes_batch1_ctx2000(name, gb):
+    cfg = synth.CONFIGS[name]
+    read, write, weights = bench.step_bytes(cfg, 1, 2000)
+    assert abs(read / 1e9 - gb) < 0.02, read
+    # what the step writes: the SSM state, one conv row per Mamba layer, one KV row per attention layer
+    assert write == 27 * 128 * 80 * 128 * 4 + 27 * 12288 * 2 + 4 * 2 * 8 * 128 * 2
+
+
+def test_quantized_matrix_bytes():
+    # W4 g64: 4 bits per weight, then per 64 weights an fp16 scale and a 4-bit zero
+    assert bench.matrix_bytes(synth.FMT_W4, 64, 16, 128) == 16 * 128 / 2 + 16 * 2 * (2 + 0.5)
+    # W8: 8 bits per weight, an fp16 scale per group, no zero
+    assert bench.matrix_bytes(synth.FMT_W8, 128, 16, 256) == 16 * 256 + 16 * 2 * 2
+    assert bench.matrix_bytes(synth.FMT_BF16, 64, 16, 128) == 16 * 128 * 2
+
+
+def test_prefill_flops_4096():
+    proj, attn, ssd = bench.prefill_flops(synth.CONFIGS["nano_prefill"], 4096)
+    assert abs(proj / 1e12 - 63.17) < 0.01
+    # causal attention: QK^T and PV over T(T+1)/2 pairs, 40 q heads of 128, 4 layers
+    assert attn == 4 * 40 * 2 * 2.0 * 128 * 4096 * 4097 / 2
+    assert 0 < ssd < 0.05 * proj
