@@ -209,6 +209,8 @@ CONFIGS = {
     "nano_bf16": nano_config(),
     "nano_w4": nano_config(name="nano_w4", wfmt=FMT_W4, group_size=64),
     "nano_w3": nano_config(name="nano_w3", wfmt=FMT_W3, group_size=64),
+    # W4 backbone with 4-bit vocabulary heads too (the heads are 35% of the W4 step's bytes in bf16)
+    "nano_w4_qheads": nano_config(name="nano_w4_qheads", wfmt=FMT_W4, group_size=64, head_fmt=FMT_W4),
     "nano_w8_b16": nano_config(name="nano_w8_b16", wfmt=FMT_W8, group_size=128, batch=16,
                                ctx_range=(500, 6000), steps=500, kv_capacity=7000),
     "nano_prefill": nano_config(name="nano_prefill", ctx=0, prefill_T=4096, steps=0,

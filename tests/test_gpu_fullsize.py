@@ -28,7 +28,7 @@ def perturbed(x):
     return x
 
 
-@pytest.mark.parametrize("name", ["nano_bf16", "nano_w4", "nano_w3", "nano_w8_b16"])
+@pytest.mark.parametrize("name", ["nano_bf16", "nano_w4", "nano_w3", "nano_w8_b16", "nano_w4_qheads"])
 def test_full_size_decode(cuda, name):
     import torch
     from attention_frame_decode_b200.synthetic import ring_to_history
