@@ -47,6 +47,10 @@ class VcWeights(C.Structure):
                 ("head_func", VcQmat)]
 
 
+class VcTokenEmbeddings(C.Structure):
+    _fields_ = [("emb_text", C.c_void_p), ("emb_func", C.c_void_p)]
+
+
 class VcState(C.Structure):
     _fields_ = [("ssm", C.c_void_p), ("conv", C.c_void_p), ("k", C.c_void_p), ("v", C.c_void_p),
                 ("ctx_len", C.c_void_p), ("status", C.c_void_p)]
@@ -65,6 +69,7 @@ _lib.vc_workspace_bytes.restype = C.c_size_t
 _lib.vc_backbone_create.argtypes = [C.POINTER(VcConfig), C.POINTER(VcWeights), _p, C.c_size_t, _p, C.POINTER(_p)]
 _lib.vc_set_option.argtypes = [_p, _i, _i]
 _lib.vc_step.argtypes = [_p, _p, _i, _p, C.POINTER(VcState), _p, _p, _p]
+_lib.vc_step_fused.argtypes = [_p, _p, C.POINTER(VcTokenEmbeddings), _i, _p, C.POINTER(VcState), _p, _p, _p]
 _lib.vc_step_host.argtypes = [_p, _p, _i, _p, C.POINTER(VcState), _p, _p, _p]
 _lib.vc_prefill.argtypes = [_p, _p, _i, _i, C.POINTER(VcState), _p]
 _lib.vc_debug_set_taps.argtypes = [_p, _p, _p]
@@ -89,13 +94,14 @@ _lib.vc_status_string.restype = C.c_char_p
 _lib.vc_last_cuda_error.argtypes = []
 _lib.vc_last_cuda_error.restype = C.c_char_p
 for _f in ("vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant", "vc_backbone_create",
-           "vc_set_option", "vc_step", "vc_step_host", "vc_prefill", "vc_debug_set_taps", "vc_debug_set_prefill_taps",
-           "vc_debug_mamba_step",
+           "vc_set_option", "vc_step", "vc_step_fused", "vc_step_host", "vc_prefill", "vc_debug_set_taps",
+           "vc_debug_set_prefill_taps", "vc_debug_mamba_step",
            "vc_debug_gemv", "vc_debug_gemm", "vc_debug_mamba_prefill", "vc_debug_gemv_noalloc"):
     getattr(_lib, _f).restype = _i
 
 EXPORTS = ("vc_weight_bytes", "vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant",
-           "vc_workspace_bytes", "vc_backbone_create", "vc_set_option", "vc_step", "vc_step_host", "vc_prefill",
+           "vc_workspace_bytes", "vc_backbone_create", "vc_set_option", "vc_step", "vc_step_fused", "vc_step_host",
+           "vc_prefill",
            "vc_debug_set_taps", "vc_debug_set_prefill_taps", "vc_debug_mamba_step", "vc_gemv_scratch_bytes",
            "vc_debug_gemv", "vc_debug_gemm", "vc_gemv_noalloc_scratch_bytes", "vc_debug_gemv_noalloc",
            "vc_debug_mamba_prefill_scratch_bytes", "vc_debug_mamba_prefill", "vc_destroy",
@@ -322,6 +328,15 @@ class Backbone:
         B = x.shape[0]
         _check(_lib.vc_step(self.h, _ptr(x), B, _ptr(slots), C.byref(state.c), _ptr(tok_text), _ptr(tok_func),
                             _stream(stream)), "vc_step")
+
+    def step_fused(self, speech, emb_text, emb_func, state: State, tok_text, tok_func, slots=None, stream=None):
+        """one frame with its input fused on the device: speech + emb_text[tok_text] + emb_func[tok_func]
+        (the previous frame's tokens, read from and then overwritten in tok_text / tok_func)"""
+        B = speech.shape[0]
+        emb = VcTokenEmbeddings(_ptr(emb_text), _ptr(emb_func))
+        self._emb = (emb_text, emb_func)
+        _check(_lib.vc_step_fused(self.h, _ptr(speech), C.byref(emb), B, _ptr(slots), C.byref(state.c),
+                                  _ptr(tok_text), _ptr(tok_func), _stream(stream)), "vc_step_fused")
 
     def step_host(self, x_host, state: State, tok_text_host, tok_func_host, slots=None, stream=None):
         B = x_host.shape[0]

@@ -119,6 +119,8 @@ struct GraphKey {
     const void* tf;
     const float* th;
     const float* tl;
+    const void* et;   // token embeddings of the fused-input variant (null: plain inputs)
+    const void* ef;
     bool operator<(const GraphKey& o) const {
         return memcmp(this, &o, sizeof(GraphKey)) < 0;
     }
@@ -365,7 +367,7 @@ static GemvMat gm(const vc_qmat& q) {
 
 // the step's launch sequence (recorded into a graph, or launched directly)
 static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32_t* slots, const vc_state* st,
-                               int32_t* tt, int32_t* tf, cudaStream_t s) {
+                               int32_t* tt, int32_t* tf, const vc_token_embeddings* emb, cudaStream_t s) {
     const Dims& D = h->D;
     const Workspace& W = h->ws;
     const int fmt = h->cfg.wfmt, grp = h->cfg.group_size;
@@ -381,6 +383,10 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
     ia.r = W.r; ia.gamma = h->layers[0].norm; ia.act = W.act_a; ia.act_ld = W.lda; ia.act_f16 = act_f16;
     ia.parts = W.parts_r; ia.tap = h->tap_hidden; ia.ctx_len = st->ctx_len; ia.slots = slots; ia.cap = D.cap;
     ia.ok = W.ok; ia.status = st->status;
+    if (emb) {
+        ia.emb_t = (const uint16_t*)emb->emb_text; ia.emb_f = (const uint16_t*)emb->emb_func;
+        ia.tok_t = tt; ia.tok_f = tf; ia.Vt = D.Vt; ia.Vf = D.Vf;
+    }
     if ((e = launch_input(ia, s)) != cudaSuccess) return e;
 
     InScale pre{};
@@ -496,21 +502,22 @@ static vc_status check_step_args(vc_backbone* h, const void* x, int B, const vc_
 }
 
 static vc_status run_step(vc_backbone* h, const void* x, int B, const int32_t* slots, const vc_state* st, int32_t* tt,
-                          int32_t* tf, cudaStream_t s) {
+                          int32_t* tf, cudaStream_t s, const vc_token_embeddings* emb = nullptr) {
     if (!h->use_graph) {
-        cudaError_t e = record_step(h, x, B, slots, st, tt, tf, s);
+        cudaError_t e = record_step(h, x, B, slots, st, tt, tf, emb, s);
         return e == cudaSuccess ? VC_OK : cuda_fail(e, "vc_step launch");
     }
     GraphKey key;
     memset(&key, 0, sizeof(key));
     key.B = B; key.slots = slots; key.st = *st; key.tt = tt; key.tf = tf;
     key.th = h->tap_hidden; key.tl = h->tap_logits;
+    if (emb) { key.et = emb->emb_text; key.ef = emb->emb_func; }
     auto it = h->graphs.find(key);
     if (it == h->graphs.end()) {
         if (h->graphs.size() > 64) clear_graphs(h);
         cudaStream_t cs = h->capture_stream;
         CK(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
-        cudaError_t e = record_step(h, x, B, slots, st, tt, tf, cs);
+        cudaError_t e = record_step(h, x, B, slots, st, tt, tf, emb, cs);
         cudaGraph_t g = nullptr;
         cudaError_t e2 = cudaStreamEndCapture(cs, &g);
         if (e != cudaSuccess) {
@@ -557,6 +564,15 @@ extern "C" vc_status vc_step(vc_backbone* h, const void* x, int B, const int32_t
     if (st != VC_OK) return st;
     if (!aligned16(x)) return VC_ERR_INVALID_ARG;
     return run_step(h, x, B, slots, state, tok_text, tok_func, (cudaStream_t)stream);
+}
+
+extern "C" vc_status vc_step_fused(vc_backbone* h, const void* speech, const vc_token_embeddings* emb, int B,
+                                   const int32_t* slots, const vc_state* state, int32_t* tok_text, int32_t* tok_func,
+                                   vc_stream_t stream) {
+    vc_status st = check_step_args(h, speech, B, state, tok_text, tok_func);
+    if (st != VC_OK) return st;
+    if (!emb || !emb->emb_text || !emb->emb_func || !aligned16(speech)) return VC_ERR_INVALID_ARG;
+    return run_step(h, speech, B, slots, state, tok_text, tok_func, (cudaStream_t)stream, emb);
 }
 
 extern "C" vc_status vc_step_host(vc_backbone* h, const void* x_host, int B, const int32_t* slots,

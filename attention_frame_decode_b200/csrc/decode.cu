@@ -27,18 +27,31 @@ __global__ void input_kernel(const InputArgs a) {
         a.ok[b] = okb;
         if (!okb) atomicOr(a.status, VC_DEV_CAPACITY);
     }
+    const uint16_t* et = nullptr;
+    const uint16_t* ef = nullptr;
+    if (a.emb_t) {
+        const int tt = a.tok_t[b], tf = a.tok_f[b];
+        if (tt >= 0 && tt < a.Vt) et = a.emb_t + (size_t)tt * a.d;
+        if (tf >= 0 && tf < a.Vf) ef = a.emb_f + (size_t)tf * a.d;
+    }
     for (int k = threadIdx.x; k < a.d; k += blockDim.x) {
-        const float v = bf16_bits_to_f(a.x[(size_t)b * a.d + k]);
+        float v = bf16_bits_to_f(a.x[(size_t)b * a.d + k]);
+        if (a.emb_t) {
+            if (et) v += bf16_bits_to_f(et[k]);
+            if (ef) v += bf16_bits_to_f(ef[k]);
+            v = bf16_bits_to_f(act_bits<false>(v));   // the fused input is a bf16 embedding
+        }
         a.r[(size_t)b * a.d + k] = v;
         const float an = v * a.gamma[k];
         a.act[(size_t)b * a.act_ld + k] = a.act_f16 ? act_bits<true>(an) : act_bits<false>(an);
         if (a.tap) a.tap[(size_t)b * a.d + k] = v;
     }
+    __syncthreads();   // r of this row complete (written by all threads of the CTA)
     for (int u = threadIdx.x; u < a.n_units; u += blockDim.x) {
         float ss = 0.0f;
         const int k1 = min(a.d, (u + 1) * a.unit_rows);
         for (int k = u * a.unit_rows; k < k1; ++k) {
-            const float v = bf16_bits_to_f(a.x[(size_t)b * a.d + k]);
+            const float v = a.r[(size_t)b * a.d + k];
             ss += v * v;
         }
         a.parts[(size_t)b * a.n_units + u] = ss;

@@ -7,7 +7,14 @@
 namespace vc {
 
 struct InputArgs {
-    const uint16_t* x;      // [B][d] bf16 frame inputs
+    const uint16_t* x;      // [B][d] bf16 frame inputs (with emb_t/emb_f: the speech embeddings)
+    // optional fusion of the previous frame's tokens: x + emb_t[tok_t[b]] + emb_f[tok_f[b]] (a token
+    // outside [0, V) adds nothing), summed in fp32 and rounded once to bf16
+    const uint16_t* emb_t;  // [Vt][d] bf16 or null
+    const uint16_t* emb_f;  // [Vf][d] bf16 or null
+    const int* tok_t;       // [B] previous text tokens (the step's own output buffer)
+    const int* tok_f;       // [B] previous function tokens
+    int Vt, Vf;
     int B, d, unit_rows, n_units;
     float* r;               // [B][d] residual stream (fp32)
     const float* gamma;     // first layer's pre-norm gamma

@@ -171,6 +171,27 @@ vc_status vc_set_option(vc_backbone* h, int option, int value);
 vc_status vc_step(vc_backbone* h, const void* x, int B, const int32_t* slots, const vc_state* state,
                   int32_t* tok_text, int32_t* tok_func, vc_stream_t stream);
 
+/* Token embeddings for the fused-input step (device, caller-owned): bf16 [vocab_text][d_model]
+ * and [vocab_func][d_model]. */
+typedef struct {
+    const void* emb_text;
+    const void* emb_func;
+} vc_token_embeddings;
+
+/* One frame whose input is fused on the device from this frame's speech embedding and the
+ * tokens the previous frame emitted -- the user and agent channels summed into one input per
+ * frame ("NVIDIA NemotronLabs VoiceChat 11B" blog, "Key design decisions" 3; the fused per-frame
+ * embedding of "NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM, MLX", Recipe) -- so that a session
+ * runs frame after frame without a host round trip.  For each row b:
+ *   x[b] = bf16( speech[b] + emb_text[tok_text[b]] + emb_func[tok_func[b]] )
+ * summed in fp32 in that order and rounded once; a token outside [0, vocab) (e.g. -1 before the
+ * first frame, or from a skipped session) adds nothing.  tok_text / tok_func (device, int32 [B])
+ * hold the previous tokens on entry and this frame's tokens on return (the same buffers feed the
+ * next call).  speech: bf16 [B][d_model] (device).  Otherwise as vc_step. */
+vc_status vc_step_fused(vc_backbone* h, const void* speech, const vc_token_embeddings* emb, int B,
+                        const int32_t* slots, const vc_state* state, int32_t* tok_text, int32_t* tok_func,
+                        vc_stream_t stream);
+
 /* The same frame with host buffers: copies x (host, ideally pinned) to the device, runs the
  * step and copies the tokens back into tok_text/tok_func (host), all on `stream`; the caller
  * synchronizes the stream before reading the tokens. */

@@ -84,6 +84,9 @@ def lib():
         L.or_prefill.restype = C.c_int
         L.or_mamba_mixer.argtypes = [C.POINTER(OrConfig), C.POINTER(OrLayer), C.c_int, p, p, p, C.c_int, p, p]
         L.or_mamba_mixer.restype = None
+        L.or_fuse_inputs.argtypes = [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_int,
+                                     C.c_void_p, C.c_void_p, C.c_void_p]
+        L.or_fuse_inputs.restype = None
         L.or_round_bf16.argtypes = [C.c_double]
         L.or_round_bf16.restype = C.c_double
         L.or_round_fp16.argtypes = [C.c_double]
@@ -148,6 +151,21 @@ def quantize(fmt: int, group: int, w: np.ndarray) -> Mat:
 def bf16_mat(wbits: np.ndarray) -> Mat:
     wbits = np.ascontiguousarray(wbits, np.uint16)
     return Mat(BF16, 64, wbits.shape[0], wbits.shape[1], wbits)
+
+
+def fuse_inputs(speech_bits, emb_text_bits, emb_func_bits, tok_text, tok_func):
+    """bf16 bits of speech + emb_text[tok_text] + emb_func[tok_func] per row (exact sum, one RNE
+    rounding; tokens outside the vocabulary add nothing)"""
+    sp = np.ascontiguousarray(speech_bits, np.uint16)
+    et = np.ascontiguousarray(emb_text_bits, np.uint16)
+    ef = np.ascontiguousarray(emb_func_bits, np.uint16)
+    tt = np.ascontiguousarray(tok_text, np.int32)
+    tf = np.ascontiguousarray(tok_func, np.int32)
+    B, d = sp.shape
+    out = np.empty_like(sp)
+    lib().or_fuse_inputs(B, d, sp.ctypes.data, et.ctypes.data, et.shape[0], ef.ctypes.data, ef.shape[0],
+                         tt.ctypes.data, tf.ctypes.data, out.ctypes.data)
+    return out
 
 
 def round_bf16(v: float) -> float:

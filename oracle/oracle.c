@@ -637,3 +637,29 @@ int or_prefill(const or_config* cfg, const or_weights* w, or_state* st, int slot
     free(r); free(U); free(Y); free(Y2); free(V2);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* fused per-frame input (the previous frame's tokens fed back)             */
+/* ------------------------------------------------------------------------ */
+
+static uint16_t bf16_bits_of(double v) {
+    /* v is already a bf16 value: its float image has 16 zero low bits */
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+}
+
+void or_fuse_inputs(int B, int d, const uint16_t* speech, const uint16_t* emb_text, int Vt,
+                    const uint16_t* emb_func, int Vf, const int32_t* tok_text, const int32_t* tok_func,
+                    uint16_t* out) {
+    for (int b = 0; b < B; ++b) {
+        const int tt = tok_text[b], tf = tok_func[b];
+        for (int k = 0; k < d; ++k) {
+            double v = bf16_val(speech[(long)b * d + k]);
+            if (tt >= 0 && tt < Vt) v += bf16_val(emb_text[(long)tt * d + k]);
+            if (tf >= 0 && tf < Vf) v += bf16_val(emb_func[(long)tf * d + k]);
+            out[(long)b * d + k] = bf16_bits_of(or_round_bf16(v));
+        }
+    }
+}

@@ -126,6 +126,15 @@ int or_prefill(const or_config* cfg, const or_weights* w, or_state* st, int slot
 void or_mamba_mixer(const or_config* cfg, const or_layer* L, int T, const double* zxbcdt, double* ssm,
                     double* conv, int ssd_chunk, double* y_out, double* v_out);
 
+/* Fused per-frame input of a session ("NVIDIA NemotronLabs VoiceChat 11B" blog, "Key design
+ * decisions" 3: the user's channel and the agent's channels are summed into one input per frame):
+ * out[b] = bf16( speech[b] + emb_text[tok_text[b]] + emb_func[tok_func[b]] ), the sum exact (in
+ * double) and rounded once to nearest-even bf16; a token outside [0, V) adds nothing.
+ * speech/out: bf16 bits [B][d]; emb_text [Vt][d], emb_func [Vf][d] bf16 bits. */
+void or_fuse_inputs(int B, int d, const uint16_t* speech, const uint16_t* emb_text, int Vt,
+                    const uint16_t* emb_func, int Vf, const int32_t* tok_text, const int32_t* tok_func,
+                    uint16_t* out);
+
 /* Rounding helpers exposed for tests: RNE to bf16 / fp16 value, in double. */
 double or_round_bf16(double v);
 double or_round_fp16(double v);

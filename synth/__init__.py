@@ -222,6 +222,7 @@ CONFIGS = {
 # ----------------------------------------------------------------------------------------------
 K_NORM, K_IN, K_OUT, K_CONVW, K_CONVB, K_ALOG, K_D, K_DTB, K_GNORM, K_QKV, K_O, K_UP, K_DOWN = range(13)
 TID_FINAL_NORM, TID_HEAD_TEXT, TID_HEAD_FUNC = 1, 2, 3
+TID_EMB_TEXT, TID_EMB_FUNC = 4, 5
 
 
 def layer_tid(layer, kind):
@@ -281,6 +282,12 @@ def frame_inputs(cfg: Config, seed: int, step: int, B: int | None = None):
     """fused per-frame input embeddings x[B][d] (bf16 bits) for decode step ``step``."""
     B = cfg.batch if B is None else B
     return normal_bf16(seed + 1, 100 + step, (B, cfg.d_model))
+
+
+def token_embeddings(cfg: Config, seed: int):
+    """bf16 bits of the text and function token embedding tables, N(0, 0.5): [Vt][d], [Vf][d]."""
+    return (normal_bf16(seed, TID_EMB_TEXT, (cfg.vocab_text, cfg.d_model), 0.0, 0.5),
+            normal_bf16(seed, TID_EMB_FUNC, (cfg.vocab_func, cfg.d_model), 0.0, 0.5))
 
 
 def prefill_inputs(cfg: Config, seed: int, T: int):

@@ -378,3 +378,41 @@ def test_scalar_ssm_hand_example():
     y, _ = model.mamba_mixer(0, zx, s, np.zeros((1, cfg.conv_dim)), 0)
     assert np.allclose(y[:, 0], g["y"], rtol=0, atol=5e-12)
     assert abs(s[0, 0, 0] - g["S_final"][0]) < 5e-12
+
+
+# ------------------------------------------------------------------------------------------------
+# fused per-frame input: speech + previous text token's embedding + previous function token's
+# ------------------------------------------------------------------------------------------------
+
+def _bf16_bits(v):
+    return synth.f32_to_bf16(np.asarray(v, np.float32))
+
+
+def test_fuse_inputs_no_tokens_is_the_speech_embedding():
+    cfg = synth.tiny_config()
+    et, ef = synth.token_embeddings(cfg, 0)
+    sp = synth.frame_inputs(cfg, 0, 3, 2)
+    out = oracle.fuse_inputs(sp, et, ef, [-1, cfg.vocab_text], [-1, -7])   # outside the vocabulary
+    assert np.array_equal(out, sp)
+
+
+def test_fuse_inputs_picks_the_token_rows():
+    cfg = synth.tiny_config()
+    et, ef = synth.token_embeddings(cfg, 0)
+    zero = np.zeros((1, cfg.d_model), np.uint16)
+    assert np.array_equal(oracle.fuse_inputs(zero, et, np.zeros_like(ef), [17], [4])[0], et[17])
+    assert np.array_equal(oracle.fuse_inputs(zero, np.zeros_like(et), ef, [17], [4])[0], ef[4])
+
+
+def test_fuse_inputs_rounds_the_exact_sum_once():
+    # 1 + 2^-8 + 2^-9 lies above the midpoint 1 + 2^-8 of bf16 neighbours 1 and 1 + 2^-7, so one
+    # rounding of the exact sum gives 1 + 2^-7; rounding after each addition would give 1 (the
+    # first partial sum is a tie, to even).  1 + 2^-8 alone is that tie: 1.
+    d = 4
+    sp = np.tile(_bf16_bits([1.0]), (1, d))
+    et = np.tile(_bf16_bits([2.0 ** -8]), (1, d))
+    ef = np.tile(_bf16_bits([2.0 ** -9]), (1, d))
+    out = synth.bf16_to_f32(oracle.fuse_inputs(sp, et, ef, [0], [0]))
+    assert np.all(out == 1.0 + 2.0 ** -7)
+    out = synth.bf16_to_f32(oracle.fuse_inputs(sp, et, ef, [0], [-1]))
+    assert np.all(out == 1.0)
