@@ -318,3 +318,52 @@ def test_prefill_rejects_bad_arguments(cuda):
     with pytest.raises(vc.VcError) as e:
         bb.prefill(x[:8], 1, st)
     assert e.value.code == vc.VC_ERR_INVALID_ARG
+
+
+def test_prefill_on_a_second_stream_while_another_session_steps(cuda):
+    """A new session's opening context is prefilled into slot 1 on one stream while the session in
+    slot 0 steps frame by frame on another; both end as the oracle's do."""
+    import torch
+    from attention_frame_decode_b200.synthetic import build_model, ring_to_history
+    cfg = synth.tiny_config()
+    seed, T, cap = 4, 300, 400
+    dm = build_model(cfg, seed)
+    bb = dm.backbone(1, cap, 2)
+    st = dm.new_state(2, cap)
+    om = oracle.Model(cfg, seed)
+    ost = om.new_state(2, cap)
+    xp = synth.prefill_inputs(cfg, seed, T)
+    xpd = torch.from_numpy(xp).cuda().view(torch.bfloat16)
+    xs = [synth.frame_inputs(cfg, seed, t, 1) for t in range(8)]
+    xsd = [torch.from_numpy(x).cuda().view(torch.bfloat16) for x in xs]
+    tt = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    tf = torch.zeros_like(tt)
+    slot0 = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    s_pf, s_dec = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s_pf):
+        bb.prefill(xpd, 1, st, stream=s_pf)
+    toks = []
+    with torch.cuda.stream(s_dec):
+        for x in xsd:
+            bb.step(x, st, tt, tf, slots=slot0, stream=s_dec)
+            toks.append((tt.clone(), tf.clone()))
+    torch.cuda.synchronize()
+    assert om.prefill(ost, 1, xp, oracle.MIRROR, ssd_chunk=256)["rc"] == 0
+    for i, x in enumerate(xs):
+        ro = om.step(ost, x, oracle.MIRROR, slots=[0], taps=True)
+        for hsel, key, V in ((0, "tok_text", cfg.vocab_text), (1, "tok_func", cfg.vocab_func)):
+            top2 = np.sort(ro["logits"][hsel, 0, :V])[-2:]
+            if top2[1] - top2[0] > MARGIN:
+                assert int(toks[i][hsel].cpu()[0]) == int(ro[key][0]), (i, key)
+    assert st.ctx_len.cpu().numpy().tolist() == [8, T]
+    assert int(st.status.cpu()[0]) == 0
+    for m in range(cfg.n_mamba):
+        for slot, t in ((0, 8), (1, T)):
+            assert rel_heads(st.ssm[m, slot].cpu().numpy(), ost.ssm[m, slot]) < HID_TOL
+            ring = st.conv[m, slot].float().cpu().numpy()
+            assert rel_stored(ring_to_history(ring, t, cfg.conv_width), ost.conv[m, slot]) < HID_TOL
+    for a in range(cfg.n_attn):
+        for slot, t in ((0, 8), (1, T)):
+            assert rel_stored(st.k[a, slot, :, :t].float().cpu().numpy(), ost.k[a, slot, :, :t]) < HID_TOL
+            assert rel_stored(st.v[a, slot, :, :t].float().cpu().numpy(), ost.v[a, slot, :, :t]) < HID_TOL
