@@ -206,7 +206,9 @@ vc_status vc_step_host(vc_backbone* h, const void* x_host, int B, const int32_t*
  * the conv ring (the last W-1 frames' rows, frame t in slot t mod W, the other slot zero) and
  * KV rows 0..T-1 of the slot and sets ctx_len[slot] = T.  No tokens are produced.
  * 1 <= T <= kv_capacity (else VC_ERR_CAPACITY / VC_ERR_INVALID_ARG, nothing launched).  Uses the
- * backbone's workspace (prefill scratch sized for kv_capacity frames); asynchronous on stream. */
+ * backbone's workspace (prefill scratch sized for kv_capacity frames); asynchronous on stream.
+ * It may run concurrently with vc_step calls of other slots on other streams (they use disjoint
+ * parts of the workspace); two vc_prefill calls on one backbone must not overlap in time. */
 vc_status vc_prefill(vc_backbone* h, const void* x, int T, int slot, const vc_state* state, vc_stream_t stream);
 
 /* test/debug taps for the next vc_step calls (device fp32 buffers or NULL):
