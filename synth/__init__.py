@@ -213,6 +213,9 @@ CONFIGS = {
     "nano_w4_qheads": nano_config(name="nano_w4_qheads", wfmt=FMT_W4, group_size=64, head_fmt=FMT_W4),
     "nano_w8_b16": nano_config(name="nano_w8_b16", wfmt=FMT_W8, group_size=128, batch=16,
                                ctx_range=(500, 6000), steps=500, kv_capacity=7000),
+    # the W4 backbone serving 16 sessions of ragged contexts (C2's weights with C3's batch)
+    "nano_w4_b16": nano_config(name="nano_w4_b16", wfmt=FMT_W4, group_size=64, batch=16,
+                               ctx_range=(500, 6000), steps=500, kv_capacity=7000),
     "nano_prefill": nano_config(name="nano_prefill", ctx=0, prefill_T=4096, steps=0,
                                 kv_capacity=4096 + 64, random_state=False),
 }

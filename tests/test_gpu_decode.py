@@ -192,16 +192,41 @@ def test_nano_layer(cuda, pattern, wfmt, group):
     assert int(run.st.ctx_len.cpu()[0]) == 2002
 
 
-@pytest.mark.parametrize("B", [3, 16])
-def test_nano_batch_ragged_contexts(cuda, B):
-    cfg = nano_layer_cfg("M*-", synth.FMT_W8, 128)
+@pytest.mark.parametrize("B,wfmt,group", [(3, synth.FMT_W8, 128), (16, synth.FMT_W8, 128), (16, synth.FMT_W4, 64),
+                                           (12, synth.FMT_W3, 64)])
+def test_nano_batch_ragged_contexts(cuda, B, wfmt, group):
+    """16 sessions at ragged contexts (the two-tile GEMV for 9..16 rows).  With 16 rows x 2 heads
+    some top-2 margins sit just above 1e-3 inside the rounding noise of fp16-dequantized weights,
+    so tokens are compared where the margin also exceeds twice the logit change that 1-ulp flips
+    in ~1% of the frame inputs cause in the oracle itself (as in the full-size tests)."""
+    cfg = nano_layer_cfg("M*-", wfmt, group)
     ctx = synth.uniform_i32(7, 0, (B,), 0, 300)
     ctx[0] = 0
     ctx[-1] = 63
     run = Run(cfg, 4, B, 512, ctx_lens=ctx)
+    compared = 0
     for t in range(2):
+        ost_floor = run.ost.clone()
+        x = synth.frame_inputs(cfg, 4, t, B)
         ro = run.step(t)
-        check_step(run, ro)
+        xp = x.copy()
+        xp[:, ::97] ^= 1
+        rp = run.om.step(ost_floor, xp, oracle.MIRROR, taps=True)
+        hid = run.hid.cpu().numpy()
+        lg = run.lg.cpu().numpy()
+        for layer in range(cfg.n_layers + 1):
+            assert rel(hid[layer], ro["hidden"][layer]) < HID_TOL, (t, layer)
+        for b in range(B):
+            for hsel, (tg, to, V) in enumerate(((run.tt, ro["tok_text"], cfg.vocab_text),
+                                                (run.tf, ro["tok_func"], cfg.vocab_func))):
+                lo = ro["logits"][hsel, b, :V]
+                assert rel(lg[hsel, b, :V], lo) < HID_TOL
+                noise = float(np.max(np.abs(rp["logits"][hsel, b, :V] - lo)))
+                top2 = np.sort(lo)[-2:]
+                if top2[1] - top2[0] > max(MARGIN, 2.0 * noise):
+                    compared += 1
+                    assert int(tg.cpu().numpy()[b]) == int(to[b]), (t, b, hsel)
+    assert compared >= B // 2
     assert np.array_equal(run.st.ctx_len.cpu().numpy()[:B], ctx + 2)
 
 
