@@ -326,7 +326,9 @@ def run_prefill_bench(args, cfg, world, rank, local):
         cpu = {"value": v, "unit": "frames/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"prefill of the first {Ts} frames of the same context on the same model, {dt:.1f} s"}
     if rank == 0:
-        n_launch = 2 + sum({"M": 9, "*": 5, "-": 5}[k] for k in cfg.pattern)
+        # per layer: pre-norm, two unpacks (side stream) and two GEMMs, plus conv, dt, chunk
+        # states, scan, SSD outputs and gated norm (Mamba-2) or flash attention; one final kernel
+        n_launch = 1 + sum({"M": 11, "*": 6, "-": 5}[k] for k in cfg.pattern)
         line = {
             "metric": PREFILL_METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
