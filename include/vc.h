@@ -200,8 +200,8 @@ vc_status vc_step_host(vc_backbone* h, const void* x_host, int B, const int32_t*
 
 /* Prefill of T frames x bf16 [T][d_model] (device) into session `slot` -- the opening context a
  * streaming session consumes before its frames ("NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM,
- * MLX", Recipe: the prompt is taken in as one block before the caller's speech).  The slot starts empty: whatever
- * it held is overwritten.  Mamba-2 layers run the chunked SSD (Dao & Gu, "Transformers are SSMs",
+ * MLX", Recipe: the prompt is taken in as one block before the caller's speech).  The slot
+ * starts empty: whatever it held is overwritten.  Mamba-2 layers run the chunked SSD (Dao & Gu, "Transformers are SSMs",
  * chunk 256) over the frames, attention layers causal GQA; the call writes the final SSM state,
  * the conv ring (the last W-1 frames' rows, frame t in slot t mod W, the other slot zero) and
  * KV rows 0..T-1 of the slot and sets ctx_len[slot] = T.  No tokens are produced.
