@@ -416,3 +416,42 @@ def test_fuse_inputs_rounds_the_exact_sum_once():
     assert np.all(out == 1.0 + 2.0 ** -7)
     out = synth.bf16_to_f32(oracle.fuse_inputs(sp, et, ef, [0], [-1]))
     assert np.all(out == 1.0)
+
+
+# ------------------------------------------------------------------------------------------------
+# mirror mode: the storage points really round, and only by a rounding's worth
+# ------------------------------------------------------------------------------------------------
+
+def _is_bf16(a):
+    a = np.asarray(a, np.float64)
+    back = synth.bf16_to_f32(synth.f32_to_bf16(a.astype(np.float32))).astype(np.float64)
+    return bool(np.array_equal(a, back))
+
+
+@pytest.mark.parametrize("how", ["steps", "prefill"])
+def test_mirror_mode_stores_bf16_values(how):
+    """In mirror mode the conv history (the stored in_proj xBC values) and the KV cache hold bf16
+    values only; in exact mode they do not.  Each layer's update of the residual differs from the
+    exact mode's by less than 2% of its RMS (a few bf16 roundings of its inputs) and by more than
+    nothing (the roundings happen)."""
+    cfg = small_cfg(pattern="M*-M")
+    model = oracle.Model(cfg, seed=12)
+    T = 6
+    sm, se = model.new_state(1, cfg.kv_capacity), model.new_state(1, cfg.kv_capacity)
+    if how == "steps":
+        for t in range(T):
+            x = synth.frame_inputs(cfg, 12, t, 1)
+            rm = model.step(sm, x, oracle.MIRROR, taps=True)["hidden"][:, 0]
+            re = model.step(se, x, oracle.EXACT, taps=True)["hidden"][:, 0]
+    else:
+        xb = synth.prefill_inputs(cfg, 12, T)
+        rm = model.prefill(sm, 0, xb, oracle.MIRROR, ssd_chunk=4, taps=True)["hidden"][:, -1]
+        re = model.prefill(se, 0, xb, oracle.EXACT, ssd_chunk=4, taps=True)["hidden"][:, -1]
+    for st, want in ((sm, True), (se, False)):
+        assert _is_bf16(st.conv) == want
+        assert _is_bf16(st.k[:, :, :, :T]) == want
+        assert _is_bf16(st.v[:, :, :, :T]) == want
+    # first layer only: later layers see inputs that already differ
+    dm, de = rm[1] - rm[0], re[1] - re[0]
+    err = rel_err(dm, de)
+    assert 0.0 < err < 2e-2
