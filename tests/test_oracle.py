@@ -10,8 +10,11 @@
   4. chunked SSD == sequential recurrence for several chunk lengths, ragged T
      and a non-zero initial state.
   5. closed forms: memoryless limit, pure decay with x = 0 and softplus(0) = ln 2,
-     relu^2 of negative pre-activations, argmax ties, the hand-worked scalar
-     SSM recurrence in tests/golden/ssm_scalar.txt.
+     relu^2 of negative pre-activations, RMSNorm of a constant vector, argmax ties,
+     the hand-worked scalar SSM recurrence in tests/golden/ssm_scalar.txt.
+  6. fused input: one rounding of the exact sum, token rows, no-token case.
+  7. mirror mode: the stored values (conv history, K/V) are bf16 values, and the
+     roundings move a layer's update by less than 2% of its RMS.
 """
 import math
 import os
@@ -328,6 +331,32 @@ def test_relu2_kills_negative_preactivations():
     x = synth.f32_to_bf16(np.abs(synth.normal_f32(7, 7, (1, cfg.d_model))) + 0.5)
     r = model.step(st, x, oracle.EXACT, taps=True)
     assert np.array_equal(r["hidden"][1], r["hidden"][0])
+
+
+def test_rmsnorm_of_a_constant_vector():
+    """A residual that is the constant c everywhere normalizes to gamma c / sqrt(c^2 + eps) (its
+    mean square is c^2).  The MLP layer is made inert (every up pre-activation negative), and the
+    text head's rows 0..d-1 are the unit vectors, so its logits read the final norm's output."""
+    cfg = small_cfg(pattern="-")
+    d = cfg.d_model
+    model = oracle.Model(cfg, seed=13)
+    up = model.mats[(0, synth.K_UP)]
+    wneg = -np.abs(synth.bf16_to_f32(up.q)).astype(np.float32) - 0.01
+    model.mats[(0, synth.K_UP)] = oracle.bf16_mat(synth.f32_to_bf16(wneg))
+    model.layers[0].up = model.mats[(0, synth.K_UP)].c()
+    eye = np.zeros((cfg.vocab_text, d), np.float32)
+    eye[np.arange(d), np.arange(d)] = 1.0
+    model.head_text = oracle.bf16_mat(synth.f32_to_bf16(eye))
+    model.weights.head_text = model.head_text.c()
+    gamma = model.final_norm.astype(np.float64)
+    for c in (0.75, 3.0, 1e-3):
+        x = synth.f32_to_bf16(np.full((1, d), c, np.float32))
+        cb = float(synth.bf16_to_f32(x)[0, 0])
+        r = model.step(model.new_state(1, cfg.kv_capacity), x, oracle.EXACT, taps=True)
+        assert np.array_equal(r["hidden"][1], r["hidden"][0])
+        expect = gamma * cb / math.sqrt(cb * cb + cfg.eps)
+        assert np.allclose(r["logits"][0, 0, :d], expect, rtol=1e-13, atol=0)
+        assert np.all(r["logits"][0, 0, d:cfg.vocab_text] == 0.0)
 
 
 def test_argmax_lowest_index_on_ties():
