@@ -322,8 +322,9 @@ extern "C" vc_status vc_backbone_create(const vc_config* cfg, const vc_weights* 
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->prefill_side, cudaStreamNonBlocking);
     for (int i = 0; i < 5 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&h->pf_ev[i], cudaEventDisableTiming);
     if (e != cudaSuccess) {
-        delete h;
-        return cuda_fail(e, "vc_backbone_create");
+        const vc_status st = cuda_fail(e, "vc_backbone_create");
+        vc_destroy(h);   // releases whichever streams and events were created
+        return st;
     }
     *out = h;
     return VC_OK;
