@@ -159,49 +159,74 @@ class ClockSampler:
 # CPU oracle (cpu_baseline leg and --impl reference)
 # ------------------------------------------------------------------------------------------------
 
-def oracle_rate(cfg, n_steps, seed=0):
-    """time n_steps of the oracle on this host (all cores) from the same pre-filled state."""
+def oracle_run(cfg, max_steps, seed=0, warmup=0, budget_s=None):
+    """time up to max_steps frame-steps of the oracle on this host (all cores) from the same
+    pre-filled state, after `warmup` untimed ones; with a budget, the timing stops after the step
+    that crosses it.  Returns (frame-steps/s, seconds timed, steps timed)."""
     import oracle
     B = cfg.batch
     model = oracle.Model(cfg, seed)
     st = model.new_state(B, cfg.kv_capacity)
     if cfg.random_state:
         st.fill_random(seed, synth.context_lengths(cfg, seed, B))
-    t0 = time.perf_counter()
-    for s in range(n_steps):
+    for s in range(warmup):
         model.step(st, synth.frame_inputs(cfg, seed, s, B), oracle.MIRROR)
+    n = 0
+    t0 = time.perf_counter()
+    while n < max_steps:
+        model.step(st, synth.frame_inputs(cfg, seed, warmup + n, B), oracle.MIRROR)
+        n += 1
+        if budget_s is not None and time.perf_counter() - t0 >= budget_s:
+            break
     dt = time.perf_counter() - t0
-    return B * n_steps / dt, dt
+    return B * n / dt, dt, n
+
+
+def oracle_rate(cfg, n_steps, seed=0):
+    """time n_steps of the oracle on this host (all cores) from the same pre-filled state."""
+    rate, dt, _ = oracle_run(cfg, n_steps, seed)
+    return rate, dt
 
 
 def cpu_threads():
     return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
 
+REF_BUDGET_S = 30.0   # seconds of oracle work the reference arm times, so that its run ends in minutes
+REF_PREFILL_FRAMES = 16
+
+
 def run_reference(args, cfg, rank):
+    """The reference arm: the oracle on this host's cores, on this workload.  At most one untimed
+    warm-up step, then up to --steps timed steps, each a bounded sample of the workload (decode: one
+    frame-step of the whole batch, continuing from the same pre-filled state; prefill: the oracle's
+    prefill of the context's first 16 frames into an empty slot); the timing stops after the step
+    that crosses REF_BUDGET_S, and the line reports the steps it timed."""
     if rank != 0:
         return
+    warm = min(args.warmup, 1)
     if cfg.prefill_T:
-        Ts = 16
-        value, dt = prefill_oracle_rate(cfg, Ts)
-        sample = f"prefill of the first {Ts} frames of the {cfg.prefill_T}-frame context per timed run"
+        Ts = REF_PREFILL_FRAMES
+        value, dt, n = prefill_oracle_run(cfg, Ts, args.steps, warmup=warm, budget_s=REF_BUDGET_S)
+        sample = (f"each step: the oracle's prefill of the first {Ts} frames of the {cfg.prefill_T}-frame "
+                  f"context; {n} step(s) timed, {dt:.1f} s")
         line = {"impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "frames/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * dt,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": {"workload": cfg.name, "frames": cfg.prefill_T, "batch": 1},
+                "n_gpus": args.gpus, "steps": n, "steps_requested": args.steps, "warmup": warm,
+                "ms_per_step": 1000.0 * dt / n, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic", "config": {"workload": cfg.name, "frames": cfg.prefill_T,
+                                                                "batch": 1},
                 "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cpu_threads(), "kind": "oracle",
                                  "sample": sample},
                 "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
-    n = max(1, min(args.steps, 2 if cfg.d_model > 1000 else 64))
-    for _ in range(max(0, min(args.warmup, 1))):
-        pass
-    value, dt = oracle_rate(cfg, n)
-    sample = f"{n} frame-step(s) x batch {cfg.batch} of {cfg.name} per timed run"
+    room = cfg.kv_capacity - int(synth.context_lengths(cfg, 0, cfg.batch).max()) - warm   # frames the cache holds
+    value, dt, n = oracle_run(cfg, max(1, min(args.steps, room)), warmup=warm, budget_s=REF_BUDGET_S)
+    sample = (f"each step: one frame-step of the batch of {cfg.batch} of {cfg.name}, continuing from the workload's starting "
+              f"state; {n} step(s) timed, {dt:.1f} s")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "frame-steps/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * dt / n, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "steps": n, "steps_requested": args.steps, "warmup": warm, "ms_per_step": 1000.0 * dt / n,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "batch": cfg.batch, "ctx": cfg.ctx},
             "cpu_baseline": {"value": value, "unit": "frame-steps/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
@@ -233,15 +258,30 @@ def prefill_flops(cfg, T):
     return proj, attn, ssd
 
 
-def prefill_oracle_rate(cfg, T, seed=0):
+def prefill_oracle_run(cfg, T, max_runs, seed=0, warmup=0, budget_s=None):
+    """time up to max_runs oracle prefills of the context's first T frames, each into an empty
+    slot, after `warmup` untimed ones; with a budget, the timing stops after the run that crosses
+    it.  Returns (frames/s, seconds timed, runs timed)."""
     import oracle
     model = oracle.Model(cfg, seed)
-    st = model.new_state(1, max(T, 1) + 8)
     x = synth.prefill_inputs(cfg, seed, T)
-    t0 = time.perf_counter()
-    model.prefill(st, 0, x, oracle.MIRROR, ssd_chunk=256)
-    dt = time.perf_counter() - t0
-    return T / dt, dt
+    for _ in range(warmup):
+        model.prefill(model.new_state(1, max(T, 1) + 8), 0, x, oracle.MIRROR, ssd_chunk=256)
+    n, dt = 0, 0.0
+    while n < max_runs:
+        st = model.new_state(1, max(T, 1) + 8)
+        t0 = time.perf_counter()
+        model.prefill(st, 0, x, oracle.MIRROR, ssd_chunk=256)
+        dt += time.perf_counter() - t0
+        n += 1
+        if budget_s is not None and dt >= budget_s:
+            break
+    return T * n / dt, dt, n
+
+
+def prefill_oracle_rate(cfg, T, seed=0):
+    rate, dt, _ = prefill_oracle_run(cfg, T, 1, seed)
+    return rate, dt
 
 
 def run_prefill_bench(args, cfg, world, rank, local):

@@ -1,7 +1,8 @@
 """The algorithmic byte and FLOP counts bench.py divides by (the roofline's numerator), checked
 against the per-step totals computed by hand from the layer shapes (d 4480; 27 Mamba-2 layers with
 in_proj 22656 x 4480 and out_proj 4480 x 10240; 4 attention layers with qkv 7168 x 4480 and
-o 4480 x 5120; 25 MLP layers 15680 x 4480 and back; two bf16 heads 131072 x 4480)."""
+o 4480 x 5120; 25 MLP layers 15680 x 4480 and back; two bf16 heads 131072 x 4480).  Also the
+reference arm's JSON line, run on the host for the tiny workload."""
 import pytest
 
 import bench
@@ -37,3 +38,25 @@ def test_prefill_flops_4096():
     # causal attention: QK^T and PV over T(T+1)/2 pairs, 40 q heads of 128, 4 layers
     assert attn == 4 * 40 * 2 * 2.0 * 128 * 4096 * 4097 / 2
     assert 0 < ssd < 0.05 * proj
+
+
+def test_reference_arm_line_on_the_tiny_workload():
+    """`bench.py --impl reference` times the oracle on the host (no GPU, no torch.cuda) and prints
+    one JSON line with the base keys, the steps it timed and its own cpu_baseline and e2e."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "tiny_w8", "--steps", "5",
+                          "--warmup", "3"], cwd=root, capture_output=True, text=True, timeout=300, check=True)
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "frame-steps/s" and d["higher_is_better"] is True
+    assert d["steps"] == 5 and d["steps_requested"] == 5 and d["warmup"] == 1
+    assert d["value"] > 0 and abs(d["ms_per_step"] - 1000.0 / d["value"]) < 1e-6 * d["ms_per_step"]
+    assert d["config"]["workload"] == "tiny"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "frame-steps/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
