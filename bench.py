@@ -182,12 +182,6 @@ def oracle_run(cfg, max_steps, seed=0, warmup=0, budget_s=None):
     return B * n / dt, dt, n
 
 
-def oracle_rate(cfg, n_steps, seed=0):
-    """time n_steps of the oracle on this host (all cores) from the same pre-filled state."""
-    rate, dt, _ = oracle_run(cfg, n_steps, seed)
-    return rate, dt
-
-
 def cpu_threads():
     return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
@@ -532,8 +526,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_or = 2 if cfg.d_model > 1000 else 64
-        v, dt = oracle_rate(cfg, n_or)
+        # a bounded sample: frame-steps from the same pre-filled state until 15 s of work, 64 at most
+        v, dt, n_or = oracle_run(cfg, 64, budget_s=15.0)
         cpu = {"value": v, "unit": "frame-steps/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{n_or} frame-step(s) of the same workload (batch {B}) from the same pre-filled state, "
                          f"{dt:.1f} s"}
