@@ -31,7 +31,8 @@
 /* ------------------------------------------------------------------------ */
 
 /* round v to a binary float with `sig` significant bits, round-half-to-even,
- * whose smallest quantum is 2^qmin (gradual underflow) */
+ * whose smallest quantum is 2^qmin (gradual underflow).  Pinned by ties to
+ * even, an fp16 subnormal tie and numpy's float16 conversion. */
 static double round_sig(double v, int sig, int qmin) {
     if (v == 0.0 || !isfinite(v)) return v;
     int e;
@@ -103,7 +104,10 @@ static uint32_t get_bits(const uint32_t* row, long idx, int bits) {
  * with s := 1 when the fp16 scale would be 0 (constant or all-zero group).
  * Dequantization is w^ = s * (q - z) (z = 0 for W8).  GPTQ's calibration
  * (error feedback from activations, "Recipe" on the GPTQ 3-bit MLX page) is not
- * reproduced: with synthetic weights there is no calibration data.         */
+ * reproduced: with synthetic weights there is no calibration data.
+ * Pinned by: constructed weights s (q - z) quantize back to (q, s, z) exactly,
+ * a hand-worked example (tests/golden/quant_example.txt), and the RTN error
+ * bound (half a step, one step at a clamped group extreme).                 */
 void or_quantize(int fmt, int group, int N, int K, const float* w, uint32_t* q, uint16_t* scales,
                  uint32_t* zeros) {
     const int bits = fmt_bits(fmt);
@@ -181,7 +185,8 @@ void or_codes(const or_mat* W, int32_t* codes, int32_t* zeros, double* scales) {
         codes_row(W, n, codes + (long)n * W->K, zeros + (long)n * ng, scales + (long)n * ng);
 }
 
-/* row n of the dequantized weight, w^ = s * (q - z), exact in double */
+/* row n of the dequantized weight, w^ = s * (q - z), exact in double (pinned
+ * against the independently decoded codes times scales) */
 static void deq_row(const or_mat* W, int n, double* row, int32_t* tmp_codes, int32_t* tmp_z, double* tmp_s) {
     if (W->fmt == OR_BF16) {
         const uint16_t* r = (const uint16_t*)W->q + (long)n * W->K;
@@ -208,7 +213,8 @@ void or_dequant(const or_mat* W, double* out) {
     }
 }
 
-/* Y[b][n] = sum_k W^[n][k] U[b][k] for b < B (rows of U are inputs). */
+/* Y[b][n] = sum_k W^[n][k] U[b][k] for b < B (rows of U are inputs).  Pinned
+ * by equality with a dense product on the dequantized matrix. */
 static void matmul_rows(const or_mat* W, int B, const double* U, double* Y) {
     const int ng = W->fmt == OR_BF16 ? 1 : n_groups(W);
 #pragma omp parallel
@@ -276,7 +282,9 @@ static double rnd(int mode, double v) { return mode == OR_MIRROR ? or_round_bf16
 
 /* Causal depthwise conv1d + SiLU of one frame over the history ring.
  * xc[c] = silu(b[c] + sum_{k<W-1} w[c][k] * hist[k][c] + w[c][W-1] * xBC[c]);
- * the history then drops its oldest row and appends xBC. */
+ * the history then drops its oldest row and appends xBC.  Pinned by the
+ * brute-force full causal convolution over the zero-padded sequence, and by the
+ * memoryless-limit and hand-worked scalar cases. */
 static void conv_step(const dims* m, const or_layer* L, double* hist, const double* xBC, double* xc) {
     for (int c = 0; c < m->Cx; ++c) {
         double acc = (double)L->conv_b[c];
@@ -399,7 +407,9 @@ void or_mamba_mixer(const or_config* cfg, const or_layer* L, int T, const double
     free(xc_all);
 }
 
-/* gated RMSNorm (P4): groups of E/NG channels; returns the out_proj input */
+/* gated RMSNorm (P4): groups of E/NG channels; returns the out_proj input.
+ * Pinned end to end by the brute-force full-sequence check (one and two
+ * groups). */
 static void gated_norm_row(const dims* m, const or_layer* L, const double* v, int mode, double* u) {
     int gs = m->E / m->NG;
     for (int q = 0; q < m->NG; ++q) {

@@ -106,8 +106,11 @@ void or_matvec(const or_mat* W, const double* u, double* y);
 /* One decode step for B sessions.  x: bf16 bits [B][d]; slots: [B] or NULL (=0..B-1).
  * Outputs: tok_text/tok_func [B]; optional taps: hidden [n_layers+1][B][d]
  * (residual stream after each layer, entry 0 = input), logits [2][B][V]
- * (text then function), final_act [B][d] (normed input of the heads).
- * Returns 0, or 1 if a session's cache is full (that session is skipped). */
+ * (text then function).
+ * Returns 0, or 1 if a session's cache is full (that session is skipped).
+ * Pinned by: T steps == the brute-force full-sequence evaluation (every weight
+ * format, one and two norm groups), ctx = 0 attention == v, the closed forms of
+ * the test suite, and the mirror-mode storage points holding bf16 values. */
 int or_step(const or_config* cfg, const or_weights* w, or_state* st, int B, const uint16_t* x,
             const int32_t* slots, int mode, int32_t* tok_text, int32_t* tok_func, double* hidden,
             double* logits);
@@ -115,14 +118,19 @@ int or_step(const or_config* cfg, const or_weights* w, or_state* st, int B, cons
 /* Prefill of T frames into one zero-initialised slot, layer by layer.
  * ssd_chunk = 0: Mamba-2 layers use the sequential recurrence;
  * ssd_chunk = Q > 0: they use the chunked SSD algorithm with chunk length Q.
- * hidden (optional): [n_layers+1][T][d].  Sets ctx_len[slot] = T. */
+ * hidden (optional): [n_layers+1][T][d].  Sets ctx_len[slot] = T.
+ * Pinned by: the final SSM state, conv history and K/V equal T decode steps from
+ * an empty slot. */
 int or_prefill(const or_config* cfg, const or_weights* w, or_state* st, int slot, int T,
                const uint16_t* x, int mode, int ssd_chunk, double* hidden);
 
 /* Isolated Mamba-2 mixer over T frames for one session (used by the kernel-level
  * checks): input zxbcdt [T][E+Cx+H] (double), state in/out ssm [H][P][N] and
  * conv history [W-1][Cx]; outputs the gated-norm input v [T][E] (= y*silu(z))
- * and ysum [T][E] (= y before gating).  ssd_chunk as in or_prefill. */
+ * and y [T][E] (= y before gating).  ssd_chunk as in or_prefill.
+ * Pinned by: chunked == sequential (Q in 1, 3, 16, 64, 70, 256; ragged T; a
+ * non-zero initial state), the memoryless limit, pure decay at x = 0, and the
+ * hand-worked scalar recurrence (tests/golden/ssm_scalar.txt). */
 void or_mamba_mixer(const or_config* cfg, const or_layer* L, int T, const double* zxbcdt, double* ssm,
                     double* conv, int ssd_chunk, double* y_out, double* v_out);
 
@@ -130,7 +138,9 @@ void or_mamba_mixer(const or_config* cfg, const or_layer* L, int T, const double
  * decisions" 3: the user's channel and the agent's channels are summed into one input per frame):
  * out[b] = bf16( speech[b] + emb_text[tok_text[b]] + emb_func[tok_func[b]] ), the sum exact (in
  * double) and rounded once to nearest-even bf16; a token outside [0, V) adds nothing.
- * speech/out: bf16 bits [B][d]; emb_text [Vt][d], emb_func [Vf][d] bf16 bits. */
+ * speech/out: bf16 bits [B][d]; emb_text [Vt][d], emb_func [Vf][d] bf16 bits.
+ * Pinned by: no token gives the speech row itself, a zero speech row gives the
+ * token's row, and a worked sum whose one rounding differs from two. */
 void or_fuse_inputs(int B, int d, const uint16_t* speech, const uint16_t* emb_text, int Vt,
                     const uint16_t* emb_func, int Vf, const int32_t* tok_text, const int32_t* tok_func,
                     uint16_t* out);
