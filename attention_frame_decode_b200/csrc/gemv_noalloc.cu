@@ -42,9 +42,8 @@ static __device__ __align__(256) unsigned char g_gemv_scratch[kScratchBytes];
 std::mutex g_setup_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Set-up, once per device, with that device current: the device address of g_gemv_scratch.
-// The first vc_debug_gemv_noalloc call on a device does it; make that first call before any
-// stream capture begins.
+// Set-up, once per device, with that device current: the device address of g_gemv_scratch,
+// looked up by the first vc_debug_gemv_noalloc call on that device and kept.
 vc_status scratch_for_current_device(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

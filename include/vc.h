@@ -269,7 +269,7 @@ vc_status vc_debug_gemm(const void* A, int lda, int M, const void* W, int ldw, i
  * library (4 MiB of partial sums, 65536 arrival counters that are zero at load and that every
  * call leaves zero), and the launch uses at most 32 SMs' worth of CTAs.  A weight with more than
  * 65536 row units (16*R rows each) returns VC_ERR_CAPACITY.  The first call on a device looks
- * up the array's device address for that device; make it before any stream capture begins.
+ * up the array's device address for that device and keeps it.
  * All calls on a device share the array: calls that overlap in time race and give wrong
  * results, so callers order them.  Allocates nothing. */
 size_t vc_gemv_noalloc_scratch_bytes(void);
