@@ -318,6 +318,21 @@ def test_prefill_rejects_bad_arguments(cuda):
     with pytest.raises(vc.VcError) as e:
         bb.prefill(x[:8], 1, st)
     assert e.value.code == vc.VC_ERR_INVALID_ARG
+    # empty inputs: no frames to prefill, no sessions to step; and more sessions than max_batch
+    with pytest.raises(vc.VcError) as e:
+        bb.prefill(x[:0], 0, st)
+    assert e.value.code == vc.VC_ERR_INVALID_ARG
+    tt = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    tf = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    with pytest.raises(vc.VcError) as e:
+        bb.step(x[:0], st, tt, tf)
+    assert e.value.code == vc.VC_ERR_INVALID_ARG
+    with pytest.raises(vc.VcError) as e:
+        bb.step(x[:2], st, tt, tf)
+    assert e.value.code == vc.VC_ERR_INVALID_ARG
+    # every rejection came before any launch: the session is untouched
+    torch.cuda.synchronize()
+    assert int(st.ctx_len[0]) == 0 and int(st.status[0]) == 0
 
 
 def test_prefill_on_a_second_stream_while_another_session_steps(cuda):
