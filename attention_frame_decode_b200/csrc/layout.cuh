@@ -3,7 +3,8 @@
 // The matrix is cut into units of 16*R rows and k-steps of KS = max(64, group) columns.
 // A "block" (unit u, k-step kt) holds R*SUB tiles of 16 rows x 64 columns (SUB = KS/64)
 // followed by one metadata record per 16-row slab (its fp16 scales and, for W4 and W3, its
-// zeros in 4-bit fields, for this k-step's quantization group).  Blocks are stored unit-major, k-step-minor:
+// zeros in 4-bit fields, for this k-step's quantization group).  Blocks are stored
+// unit-major, k-step-minor:
 //       offset(u, kt) = (u * KT + kt) * block_bytes
 // so any contiguous range of the flattened (u, kt) index is one contiguous byte range:
 // a warp streams its share of the matrix with 1-D bulk copies and no gather.
