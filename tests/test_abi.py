@@ -1,8 +1,12 @@
 """The C-ABI library loads on a machine without a GPU and exports every function vc.h declares;
-host-side argument validation (no device work) rejects bad shapes before any launch."""
+host-side argument validation (no device work) rejects bad shapes before any launch; vc.h
+compiles as plain C99, and the binding's ctypes structures have the sizes and member offsets the
+C compiler gives the header's structs."""
 import ctypes
 import os
 import re
+import shutil
+import subprocess
 
 import pytest
 
@@ -62,3 +66,28 @@ def test_create_rejects_bad_arguments_without_a_gpu():
     assert vc.lib().vc_step(None, None, 1, None, None, None, None, None) == vc.VC_ERR_INVALID_ARG
     assert vc.lib().vc_prefill(None, None, 4, 0, None, None) == vc.VC_ERR_INVALID_ARG
     assert vc.lib().vc_status_string(vc.VC_ERR_CAPACITY) == b"capacity exceeded"
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs a host C compiler")
+def test_header_is_c99_and_binding_structs_match_it(tmp_path):
+    import attention_frame_decode_b200 as vc
+    exe = str(tmp_path / "abi_layout")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-o", exe,
+                    os.path.join(ROOT, "tests", "host", "abi_layout.c")], check=True, capture_output=True,
+                   timeout=300)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True, timeout=60).stdout
+    py = {"vc_config": vc.VcConfig, "vc_qmat": vc.VcQmat, "vc_layer_weights": vc.VcLayerWeights,
+          "vc_weights": vc.VcWeights, "vc_state": vc.VcState, "vc_token_embeddings": vc.VcTokenEmbeddings}
+    seen = set()
+    for line in out.splitlines():
+        name, value = line.split()
+        if "." in name:
+            struct, member = name.split(".")
+            assert getattr(py[struct], member).offset == int(value), name
+            seen.add(struct + "." + member)
+        else:
+            assert ctypes.sizeof(py[name]) == int(value), name
+    # every member of every binding structure was checked
+    for struct, cls in py.items():
+        for field in cls._fields_:
+            assert struct + "." + field[0] in seen, (struct, field[0])
