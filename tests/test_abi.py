@@ -1,7 +1,8 @@
 """The C-ABI library loads on a machine without a GPU and exports every function vc.h declares;
 host-side argument validation (no device work) rejects bad shapes before any launch; vc.h
-compiles as plain C99, and the binding's ctypes structures have the sizes and member offsets the
-C compiler gives the header's structs."""
+compiles as plain C99, the binding's ctypes structures have the sizes and member offsets the C
+compiler gives the header's structs, and every bound call's argument and return types agree with
+its prototype."""
 import ctypes
 import os
 import re
@@ -91,3 +92,57 @@ def test_header_is_c99_and_binding_structs_match_it(tmp_path):
     for struct, cls in py.items():
         for field in cls._fields_:
             assert struct + "." + field[0] in seen, (struct, field[0])
+
+
+def _prototypes():
+    src = open(os.path.join(ROOT, "include", "vc.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"#[^\n]*", "", src)
+    protos = {}
+    for m in re.finditer(r"([A-Za-z_][\w\s\*]*?)\b(vc_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", src):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        args = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+        protos[name] = (ret, args)
+    return protos
+
+
+def _c_kind(decl):
+    if "*" in decl or decl.startswith("vc_stream_t"):
+        return "ptr"
+    if decl.startswith("size_t"):
+        return "size"
+    if decl.startswith("float"):
+        return "float"
+    if re.match(r"(const\s+)?(int|int32_t|vc_status|vc_wfmt)\b", decl):
+        return "int"
+    raise AssertionError(decl)
+
+
+def _ct_kind(t):
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "ptr"
+    if t is ctypes.c_size_t:
+        return "size"
+    if t is ctypes.c_float:
+        return "float"
+    if t is ctypes.c_int:
+        return "int"
+    raise AssertionError(t)
+
+
+def test_binding_signatures_match_the_header():
+    """each exported call's ctypes argument and return types agree with its vc.h prototype
+    (pointer, int, size_t, float), so no argument is marshalled at the wrong width"""
+    import attention_frame_decode_b200 as vc
+    protos = _prototypes()
+    for name in vc.EXPORTS:
+        ret, args = protos[name]
+        fn = getattr(vc.lib(), name)
+        assert fn.argtypes is not None, name
+        assert [_c_kind(a) for a in args] == [_ct_kind(t) for t in fn.argtypes], name
+        if ret == "void":
+            assert fn.restype is None, name
+        elif ret.startswith("const char"):
+            assert fn.restype is ctypes.c_char_p, name
+        else:
+            assert _c_kind(ret) == _ct_kind(fn.restype), name
