@@ -12,8 +12,9 @@
  *     size 64 (3 or 4 bits); the LLM step is memory-bandwidth bound; the speech side's fused
  *     per-frame input embedding is the LLM's input ("Recipe").
  *   - "Nemotron Voicechat on DGX Spark" intro: GPTQ W8 weights for the same backbone.
- *   - "NVIDIA NemotronLabs VoiceChat 11B" (blog), "Key design decisions" 2-3: alternating
- *     Mamba and attention layers; user and agent channels summed into one input per frame.
+ *   - "NVIDIA NemotronLabs VoiceChat 11B" (blog), "Key design decisions" 2-3: the backbone
+ *     interleaves Mamba layers with attention layers; user and agent channels are summed into
+ *     one input per frame.
  * The pages print no layer equations.  The plainest reading is used: a pre-RMSNorm residual
  * stack of Mamba-2 blocks (Dao & Gu, "Transformers are SSMs"), GQA attention without
  * positional encoding and squared-ReLU MLPs; two vocabulary heads after a final RMSNorm.

@@ -8,12 +8,12 @@
  * its own quantizer.
  *
  * Sources of the arithmetic (page titles and sections):
- *  - "NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM, MLX": the LLM inside is
- *    Nemotron-Nano-9B-v2, a 56-layer hybrid of Mamba-2 and attention,
- *    GPTQ-quantized at group size 64; its per-frame step is bandwidth bound.
- *  - "NemotronLabs VoiceChat" (SGLang-Omni cookbook): the thinker emits one
- *    text and one function token per 80 ms frame, always greedy; backbone and
- *    KV cache in bf16.
+ *  - "NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM, MLX", introduction: the
+ *    backbone is Nemotron-Nano-9B-v2 (56 layers mixing Mamba-2 and attention)
+ *    with GPTQ weights in groups of 64; its per-frame step is bandwidth bound.
+ *  - "NemotronLabs VoiceChat" (SGLang-Omni cookbook), overview: each 80 ms
+ *    frame, the thinker decodes a text token and a function token greedily;
+ *    backbone and KV cache in bf16.
  *  - The pages name the layer kinds but print no equations.  The plainest
  *    reading is used: the Mamba-2 layer of Dao & Gu, "Transformers are SSMs"
  *    (arXiv:2405.21060): causal depthwise conv1d over a ring of past inputs,
