@@ -82,3 +82,18 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] == 4
+
+
+def test_clock_record_summary():
+    """the clocks object of the JSON line: median SM clock, the highest max clock seen, and every
+    throttle reason that was active in any sample"""
+    s = bench.ClockSampler()
+    s.samples = [["1965", "1965", "700.1", "Not Active", "Not Active", "Not Active", "Not Active"],
+                 ["1800", "1965", "990.0", "Not Active", "Not Active", "Not Active", "Active"],
+                 ["1900", "1965", "980.5", "Not Active", "Not Active", "Not Active", "Not Active"],
+                 ["[N/A]", "1965", "[N/A]", "Not Active", "Not Active", "Not Active", "Not Active"]]
+    c = s.stop()
+    assert c["sm_mhz"] == 1900.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"] and c["samples"] == 4
+    s2 = bench.ClockSampler()
+    assert s2.stop()["reasons"] == ["no samples"]
