@@ -2,7 +2,8 @@
 against the per-step totals computed by hand from the layer shapes (d 4480; 27 Mamba-2 layers with
 in_proj 22656 x 4480 and out_proj 4480 x 10240; 4 attention layers with qkv 7168 x 4480 and
 o 4480 x 5120; 25 MLP layers 15680 x 4480 and back; two bf16 heads 131072 x 4480).  Also the
-reference arm's JSON line, run on the host for the tiny workload."""
+reference arm's JSON line, run on the host for the tiny workload (alone and under torchrun with two
+ranks), and the summary of the clock record."""
 import pytest
 
 import bench
