@@ -15,6 +15,8 @@
   6. fused input: one rounding of the exact sum, token rows, no-token case.
   7. mirror mode: the stored values (conv history, K/V) are bf16 values, and the
      roundings move a layer's update by less than 2% of its RMS.
+  8. sessions: batched rows through a slot map equal solo sessions; a full cache skips
+     its session and touches nothing of it.
 """
 import math
 import os
@@ -407,6 +409,56 @@ def test_scalar_ssm_hand_example():
     y, _ = model.mamba_mixer(0, zx, s, np.zeros((1, cfg.conv_dim)), 0)
     assert np.allclose(y[:, 0], g["y"], rtol=0, atol=5e-12)
     assert abs(s[0, 0, 0] - g["S_final"][0]) < 5e-12
+
+
+# ------------------------------------------------------------------------------------------------
+# sessions: slots and the full-cache rule
+# ------------------------------------------------------------------------------------------------
+
+def test_batched_slots_equal_solo_sessions():
+    """B sessions stepped together, row b writing slot slots[b], end exactly as each session
+    stepped alone: no row reads another row's state, and the slot map is applied everywhere."""
+    cfg = small_cfg(pattern="M*-M")
+    model = oracle.Model(cfg, seed=14)
+    slots = np.array([2, 0, 1], np.int32)
+    sb = model.new_state(3, cfg.kv_capacity)
+    solo = [model.new_state(1, cfg.kv_capacity) for _ in range(3)]
+    for t in range(5):
+        x = synth.frame_inputs(cfg, 14, t, 3)
+        rb = model.step(sb, x, oracle.EXACT, slots=slots, taps=True)
+        for b in range(3):
+            r1 = model.step(solo[slots[b]], x[b:b + 1], oracle.EXACT, taps=True)
+            assert rb["tok_text"][b] == r1["tok_text"][0] and rb["tok_func"][b] == r1["tok_func"][0]
+            assert np.array_equal(rb["hidden"][:, b], r1["hidden"][:, 0])
+    for s in range(3):
+        assert np.array_equal(sb.ssm[:, s], solo[s].ssm[:, 0])
+        assert np.array_equal(sb.conv[:, s], solo[s].conv[:, 0])
+        assert np.array_equal(sb.k[:, s], solo[s].k[:, 0]) and np.array_equal(sb.v[:, s], solo[s].v[:, 0])
+        assert sb.ctx_len[s] == solo[s].ctx_len[0] == 5
+
+
+def test_full_cache_session_is_skipped():
+    """A session whose cache holds kv_capacity frames is skipped: tokens -1, its state and
+    ctx_len untouched, the call reports it; the other session steps as it would alone."""
+    cfg = small_cfg(pattern="M*-M", kv_capacity=6)
+    model = oracle.Model(cfg, seed=15)
+    st = model.new_state(2, cfg.kv_capacity)
+    st.fill_random(15, np.array([6, 0], np.int32))
+    before = st.clone()
+    alone = model.new_state(1, cfg.kv_capacity)
+    for name in ("ssm", "conv", "k", "v"):           # session 1's starting state, on its own
+        getattr(alone, name)[:, 0] = getattr(before, name)[:, 1]
+    x = synth.frame_inputs(cfg, 15, 0, 2)
+    r = model.step(st, x, oracle.EXACT)
+    r1 = model.step(alone, x[1:2], oracle.EXACT)
+    assert r["rc"] == 1
+    assert r["tok_text"][0] == -1 and r["tok_func"][0] == -1
+    assert r["tok_text"][1] == r1["tok_text"][0] and r["tok_func"][1] == r1["tok_func"][0]
+    for name in ("ssm", "conv", "k", "v"):
+        assert np.array_equal(getattr(st, name)[:, 0], getattr(before, name)[:, 0]), name
+    assert st.ctx_len[0] == 6 and st.ctx_len[1] == 1
+    for name in ("ssm", "conv", "k", "v"):
+        assert np.array_equal(getattr(st, name)[:, 1], getattr(alone, name)[:, 0]), name
 
 
 # ------------------------------------------------------------------------------------------------
