@@ -1,8 +1,8 @@
 """The C-ABI library loads on a machine without a GPU and exports every function vc.h declares;
 host-side argument validation (no device work) rejects bad shapes before any launch; vc.h
 compiles as plain C99, the binding's ctypes structures have the sizes and member offsets the C
-compiler gives the header's structs, and every bound call's argument and return types agree with
-its prototype."""
+compiler gives the header's structs, every bound call's argument and return types agree with its
+prototype, and a plain C program links the library and calls it."""
 import ctypes
 import os
 import re
@@ -146,3 +146,23 @@ def test_binding_signatures_match_the_header():
             assert fn.restype is ctypes.c_char_p, name
         else:
             assert _c_kind(ret) == _ct_kind(fn.restype), name
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs a host C compiler")
+def test_plain_c_client_links_and_calls_the_library(tmp_path):
+    """a C99 program that includes only vc.h links libvc.so and gets sizes and host-side
+    rejections from it (no Python, no torch, no device)"""
+    import attention_frame_decode_b200 as vc
+    libdir = os.path.dirname(vc.LIB_PATH)
+    exe = str(tmp_path / "abi_from_c")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-o", exe,
+                    os.path.join(ROOT, "tests", "host", "abi_from_c.c"), "-L" + libdir, "-lvc",
+                    "-Wl,-rpath," + libdir], check=True, capture_output=True, timeout=300)
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stdout
+    lines = out.stdout.splitlines()
+    assert lines[-1] == "ok"
+    ws = int(lines[0].split()[1])
+    import synth
+    cfg = synth.tiny_config()
+    assert ws == vc.workspace_bytes(vc.make_config(cfg, 1, 128, 1))
