@@ -2,12 +2,14 @@
 host-side argument validation (no device work) rejects bad shapes before any launch; vc.h
 compiles as plain C99, the binding's ctypes structures have the sizes and member offsets the C
 compiler gives the header's structs, every bound call's argument and return types agree with its
-prototype, and a plain C program links the library and calls it."""
+prototype, a plain C program links the library and calls it, and the package refuses to import
+without the library."""
 import ctypes
 import os
 import re
 import shutil
 import subprocess
+import sys
 
 import pytest
 
@@ -166,3 +168,15 @@ def test_plain_c_client_links_and_calls_the_library(tmp_path):
     import synth
     cfg = synth.tiny_config()
     assert ws == vc.workspace_bytes(vc.make_config(cfg, 1, 128, 1))
+
+
+def test_package_refuses_to_import_without_the_library(tmp_path):
+    """no fallback: a copy of the package without libvc.so raises ImportError on import"""
+    pkg = tmp_path / "attention_frame_decode_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "attention_frame_decode_b200", "__init__.py"), pkg / "__init__.py")
+    code = "import attention_frame_decode_b200"
+    out = subprocess.run([sys.executable, "-c", code], cwd=str(tmp_path), capture_output=True, text=True,
+                         timeout=120)
+    assert out.returncode != 0
+    assert "ImportError" in out.stderr and "libvc.so not found" in out.stderr
