@@ -98,3 +98,12 @@ def test_clock_record_summary():
     assert c["reasons"] == ["sw_power_cap"] and c["samples"] == 4
     s2 = bench.ClockSampler()
     assert s2.stop()["reasons"] == ["no samples"]
+
+
+def test_decode_launch_count():
+    """kernels per decode step: the input kernel, in_proj GEMV + Mamba-2 step + out_proj GEMV per
+    Mamba-2 layer (27), QKV GEMV + attention + o_proj GEMV per attention layer (4), up and down
+    GEMVs per MLP layer (25), and the heads: 1 + 81 + 12 + 50 + 1 (the same counts per kernel as
+    the ncu launch lists of the step)"""
+    assert bench.launches_per_step(synth.CONFIGS["nano_bf16"]) == 145
+    assert bench.launches_per_step(synth.CONFIGS["tiny_w8"]) == 1 + 3 + 2 + 3 + 2 + 1
