@@ -183,7 +183,9 @@ def oracle_run(cfg, max_steps, seed=0, warmup=0, budget_s=None):
 
 
 def cpu_threads():
-    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    """threads the oracle actually runs on (its OpenMP team size)"""
+    import oracle
+    return oracle.threads()
 
 
 REF_BUDGET_S = 30.0   # seconds of oracle work the reference arm times, so that its run ends in minutes

@@ -91,6 +91,8 @@ def lib():
         L.or_round_bf16.restype = C.c_double
         L.or_round_fp16.argtypes = [C.c_double]
         L.or_round_fp16.restype = C.c_double
+        L.or_threads.argtypes = []
+        L.or_threads.restype = C.c_int
         _lib = L
     return _lib
 
@@ -174,6 +176,11 @@ def round_bf16(v: float) -> float:
 
 def round_fp16(v: float) -> float:
     return lib().or_round_fp16(float(v))
+
+
+def threads() -> int:
+    """threads the oracle's parallel loops run on"""
+    return int(lib().or_threads())
 
 
 # ------------------------------------------------------------------------------------------------

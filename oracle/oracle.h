@@ -149,6 +149,9 @@ void or_fuse_inputs(int B, int d, const uint16_t* speech, const uint16_t* emb_te
 double or_round_bf16(double v);
 double or_round_fp16(double v);
 
+/* threads the oracle's parallel loops use (1 without OpenMP) */
+int or_threads(void);
+
 #ifdef __cplusplus
 }
 #endif
