@@ -216,14 +216,18 @@ def run_reference(args, cfg, rank):
                 "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
-    room = cfg.kv_capacity - int(synth.context_lengths(cfg, 0, cfg.batch).max()) - warm   # frames the cache holds
+    ctx0 = synth.context_lengths(cfg, 0, cfg.batch)
+    room = cfg.kv_capacity - int(ctx0.max()) - warm   # frames the cache holds
     value, dt, n = oracle_run(cfg, max(1, min(args.steps, room)), warmup=warm, budget_s=REF_BUDGET_S)
     sample = (f"each step: one frame-step of the batch of {cfg.batch} of {cfg.name}, continuing from the workload's starting "
               f"state; {n} step(s) timed, {dt:.1f} s")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "frame-steps/s", "n_gpus": args.gpus,
             "steps": n, "steps_requested": args.steps, "warmup": warm, "ms_per_step": 1000.0 * dt / n,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "batch": cfg.batch, "ctx": cfg.ctx},
+            "config": {"workload": cfg.name, "batch": cfg.batch,
+                       "ctx_start": int(ctx0.max()) if cfg.batch == 1 else [int(ctx0.min()), int(ctx0.max())],
+                       "layers": cfg.n_layers, "weights": synth.FMT_NAMES[cfg.wfmt], "group": cfg.group_size,
+                       "heads": synth.FMT_NAMES[cfg.head_fmt]},
             "cpu_baseline": {"value": value, "unit": "frame-steps/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "frame-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
