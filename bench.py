@@ -210,7 +210,8 @@ def run_reference(args, cfg, rank):
                 "n_gpus": args.gpus, "steps": n, "steps_requested": args.steps, "warmup": warm,
                 "ms_per_step": 1000.0 * dt / n, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic", "config": {"workload": cfg.name, "frames": cfg.prefill_T,
-                                                                "batch": 1},
+                                                                "batch": 1, "layers": cfg.n_layers,
+                                                                "ssd_chunk": 256},
                 "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cpu_threads(), "kind": "oracle",
                                  "sample": sample},
                 "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
