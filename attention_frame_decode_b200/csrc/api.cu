@@ -281,6 +281,9 @@ extern "C" vc_status vc_backbone_create(const vc_config* cfg, const vc_weights* 
     Dims D;
     if (!dims_from_cfg(cfg, D)) return VC_ERR_INVALID_ARG;
     if (!fmt_ok(cfg->wfmt, cfg->group_size) || !fmt_ok(cfg->head_fmt, cfg->group_size)) return VC_ERR_INVALID_ARG;
+    // shapes the decode kernels do not cover are refused here rather than at the first step
+    if ((D.na && !attn_decode_supported(D.Hq, D.Hk, D.Dh)) || (D.nm && !mamba_step_supported(D.P, D.N)))
+        return VC_ERR_UNSUPPORTED;
     if (!weights || !weights->layers || !weights->final_norm || !workspace || !aligned16(workspace))
         return VC_ERR_INVALID_ARG;
     if (workspace_bytes < vc_workspace_bytes(cfg)) return VC_ERR_INVALID_ARG;

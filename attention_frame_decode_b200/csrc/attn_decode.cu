@@ -205,6 +205,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_decode_kernel(const AttnArg
     }
 }
 
+bool attn_decode_supported(int Hq, int Hk, int Dh) {
+    return Hk > 0 && Hq % Hk == 0 && Hq / Hk <= kMaxGQ && Dh > 0 && Dh <= kAttnThreads && kAttnThreads % Dh == 0;
+}
+
 cudaError_t launch_attn_decode(const AttnArgs& a, int pdl, cudaStream_t s) {
     const int GQ = a.Hq / a.Hk;
     if (GQ > kMaxGQ || a.Dh > kAttnThreads || kAttnThreads % a.Dh) return cudaErrorInvalidValue;

@@ -194,6 +194,8 @@ __global__ void __launch_bounds__(kMambaThreads) mamba_step_kernel(const MambaSt
     }
 }
 
+bool mamba_step_supported(int P, int N) { return P > 0 && N > 0 && P / 2 + 2 * N <= 2 * kMambaThreads; }
+
 cudaError_t launch_mamba_step(const MambaStepArgs& a, int pdl, cudaStream_t s) {
     const int Ph = a.P / 2;
     if (Ph + 2 * a.N > 2 * kMambaThreads) return cudaErrorInvalidValue;

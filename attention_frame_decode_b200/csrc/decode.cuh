@@ -67,4 +67,8 @@ cudaError_t launch_input(const InputArgs& a, cudaStream_t s);
 cudaError_t launch_mamba_step(const MambaStepArgs& a, int pdl, cudaStream_t s);
 cudaError_t launch_attn_decode(const AttnArgs& a, int pdl, cudaStream_t s);
 
+// shapes the two mixer kernels cover (their launch functions refuse the others)
+bool mamba_step_supported(int P, int N);
+bool attn_decode_supported(int Hq, int Hk, int Dh);
+
 }  // namespace vc

@@ -154,7 +154,9 @@ size_t vc_workspace_bytes(const vc_config* cfg);
 
 /* Validates cfg and weights, carves the workspace (device, vc_workspace_bytes, zeroed here on
  * `stream`) and returns a handle.  Weight and workspace memory must stay valid until
- * vc_destroy.  Nothing is launched except the workspace clear. */
+ * vc_destroy.  Nothing is launched except the workspace clear.  VC_ERR_UNSUPPORTED (before any
+ * CUDA call) for shapes the decode kernels do not cover: an attention head dim that does not
+ * divide 256, or a Mamba-2 head with P/2 + 2N > 512. */
 vc_status vc_backbone_create(const vc_config* cfg, const vc_weights* weights, void* workspace,
                              size_t workspace_bytes, vc_stream_t stream, vc_backbone** out);
 

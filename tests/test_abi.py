@@ -71,6 +71,26 @@ def test_create_rejects_bad_arguments_without_a_gpu():
     assert vc.lib().vc_status_string(vc.VC_ERR_CAPACITY) == b"capacity exceeded"
 
 
+def test_create_refuses_shapes_the_decode_kernels_do_not_cover():
+    """valid configurations outside what the mixer kernels handle are refused with
+    VC_ERR_UNSUPPORTED at create time, before any CUDA call (here: no GPU at all)"""
+    import attention_frame_decode_b200 as vc
+    import synth
+    h = ctypes.c_void_p()
+
+    def create(cfg):
+        c = vc.make_config(cfg, 1, 128, 1)
+        return vc.lib().vc_backbone_create(ctypes.byref(c), None, None, 0, None, ctypes.byref(h))
+
+    assert create(synth.tiny_config()) == vc.VC_ERR_INVALID_ARG             # supported; NULL weights
+    assert create(synth.tiny_config(attn_head_dim=48)) == vc.VC_ERR_UNSUPPORTED   # 256 % 48 != 0
+    assert create(synth.tiny_config(attn_head_dim=32)) == vc.VC_ERR_INVALID_ARG
+    big_state = synth.tiny_config(pattern="M-", ssm_heads=64, ssm_head_dim=2, ssm_state=256)
+    assert create(big_state) == vc.VC_ERR_UNSUPPORTED                        # P/2 + 2N = 513
+    assert create(big_state.replace(ssm_state=252)) == vc.VC_ERR_INVALID_ARG  # 505: supported
+    assert not h.value
+
+
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="needs a host C compiler")
 def test_header_is_c99_and_binding_structs_match_it(tmp_path):
     import attention_frame_decode_b200 as vc
