@@ -5,7 +5,7 @@
 // resident together share a few W column tiles, each streamed from HBM once, while the
 // activation rows stay in L2).  Per CTA:
 //   warp 0 (one thread): TMA producer over a 4-stage ring of 64-wide k-blocks (128-byte swizzle,
-//           no multicast), across tile boundaries;
+//           each CTA loads its own tiles), across tile boundaries;
 //   warp 1: allocates 512 TMEM columns = two 128 x 256 fp32 accumulators; one thread issues
 //           tcgen05.mma (M=128, N=256, K=16, 4 per k-block) into accumulator (tile & 1),
 //           commits each stage back to the producer and each finished tile to the epilogue;
