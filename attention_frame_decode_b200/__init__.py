@@ -73,7 +73,8 @@ _lib.vc_step_fused.argtypes = [_p, _p, C.POINTER(VcTokenEmbeddings), _i, _p, C.P
 _lib.vc_step_host.argtypes = [_p, _p, _i, _p, C.POINTER(VcState), _p, _p, _p]
 _lib.vc_prefill.argtypes = [_p, _p, _i, _i, C.POINTER(VcState), _p]
 _lib.vc_debug_set_taps.argtypes = [_p, _p, _p]
-_lib.vc_debug_set_prefill_taps.argtypes = [_p, _p]
+_lib.vc_debug_set_prefill_taps.argtypes = [_p, _p, _p]
+_lib.vc_debug_set_zx_taps.argtypes = [_p, _p]
 _lib.vc_debug_mamba_step.argtypes = [C.POINTER(VcConfig), C.POINTER(VcLayerWeights), _p, _i, _p, _p, _p, _p, _p, _p,
                                       _p, _p]
 _lib.vc_gemv_scratch_bytes.argtypes = []
@@ -95,14 +96,15 @@ _lib.vc_last_cuda_error.argtypes = []
 _lib.vc_last_cuda_error.restype = C.c_char_p
 for _f in ("vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant", "vc_backbone_create",
            "vc_set_option", "vc_step", "vc_step_fused", "vc_step_host", "vc_prefill", "vc_debug_set_taps",
-           "vc_debug_set_prefill_taps", "vc_debug_mamba_step",
+           "vc_debug_set_prefill_taps", "vc_debug_set_zx_taps", "vc_debug_mamba_step",
            "vc_debug_gemv", "vc_debug_gemm", "vc_debug_mamba_prefill", "vc_debug_gemv_noalloc"):
     getattr(_lib, _f).restype = _i
 
 EXPORTS = ("vc_weight_bytes", "vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant",
            "vc_workspace_bytes", "vc_backbone_create", "vc_set_option", "vc_step", "vc_step_fused", "vc_step_host",
            "vc_prefill",
-           "vc_debug_set_taps", "vc_debug_set_prefill_taps", "vc_debug_mamba_step", "vc_gemv_scratch_bytes",
+           "vc_debug_set_taps", "vc_debug_set_prefill_taps", "vc_debug_set_zx_taps", "vc_debug_mamba_step",
+           "vc_gemv_scratch_bytes",
            "vc_debug_gemv", "vc_debug_gemm", "vc_gemv_noalloc_scratch_bytes", "vc_debug_gemv_noalloc",
            "vc_debug_mamba_prefill_scratch_bytes", "vc_debug_mamba_prefill", "vc_destroy",
            "vc_status_string", "vc_last_cuda_error")
@@ -320,9 +322,15 @@ class Backbone:
         self._taps = (hidden, logits)
         _check(_lib.vc_debug_set_taps(self.h, _ptr(hidden), _ptr(logits)), "vc_debug_set_taps")
 
-    def set_prefill_taps(self, hidden=None):
-        self._ptaps = hidden
-        _check(_lib.vc_debug_set_prefill_taps(self.h, _ptr(hidden)), "vc_debug_set_prefill_taps")
+    def set_zx_taps(self, zx=None):
+        """fp32 [n_mamba][B][E+Cx+H]: each Mamba-2 layer's in_proj output before its bf16 rounding"""
+        self._ztaps = zx
+        _check(_lib.vc_debug_set_zx_taps(self.h, _ptr(zx)), "vc_debug_set_zx_taps")
+
+    def set_prefill_taps(self, hidden=None, zx=None):
+        """hidden fp32 [n_layers+1][T][d]; zx bf16 [n_mamba][T][E+Cx+H] (each Mamba-2 layer's in_proj output)"""
+        self._ptaps = (hidden, zx)
+        _check(_lib.vc_debug_set_prefill_taps(self.h, _ptr(hidden), _ptr(zx)), "vc_debug_set_prefill_taps")
 
     def step(self, x, state: State, tok_text, tok_func, slots=None, stream=None):
         B = x.shape[0]

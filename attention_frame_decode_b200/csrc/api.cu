@@ -119,6 +119,7 @@ struct GraphKey {
     const void* tf;
     const float* th;
     const float* tl;
+    const float* tz;
     const void* et;   // token embeddings of the fused-input variant (null: plain inputs)
     const void* ef;
     bool operator<(const GraphKey& o) const {
@@ -138,6 +139,8 @@ struct vc_backbone {
     float* tap_hidden = nullptr;
     float* tap_logits = nullptr;
     float* tap_prefill = nullptr;
+    float* tap_zx = nullptr;
+    uint16_t* tap_prefill_zx = nullptr;
     struct Graph {
         cudaGraph_t graph;
         cudaGraphExec_t exec;
@@ -350,9 +353,17 @@ extern "C" vc_status vc_set_option(vc_backbone* h, int option, int value) {
     return VC_OK;
 }
 
-extern "C" vc_status vc_debug_set_prefill_taps(vc_backbone* h, float* hidden) {
+extern "C" vc_status vc_debug_set_prefill_taps(vc_backbone* h, float* hidden, void* zx) {
     if (!h) return VC_ERR_INVALID_ARG;
     h->tap_prefill = hidden;
+    h->tap_prefill_zx = (uint16_t*)zx;
+    return VC_OK;
+}
+
+extern "C" vc_status vc_debug_set_zx_taps(vc_backbone* h, float* zx) {
+    if (!h) return VC_ERR_INVALID_ARG;
+    h->tap_zx = zx;
+    clear_graphs(h);
     return VC_OK;
 }
 
@@ -423,6 +434,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
             GemvArgs a = base;
             a.mat[0] = gm(Lw.in_proj); a.act = W.act_a; a.act_ld = W.lda; a.insc = pre;
             a.out = W.zx; a.out_ld = D.zx_rows; a.out_f16 = 0;
+            if (h->tap_zx) { a.tap = h->tap_zx + (size_t)mi * B * D.zx_rows; a.tap_ld = D.zx_rows; }
             gl.epi = EPI_STORE;
             if ((e = launch_gemv(gl, a, s)) != cudaSuccess) return e;
 
@@ -514,7 +526,7 @@ static vc_status run_step(vc_backbone* h, const void* x, int B, const int32_t* s
     GraphKey key;
     memset(&key, 0, sizeof(key));
     key.B = B; key.slots = slots; key.st = *st; key.tt = tt; key.tf = tf;
-    key.th = h->tap_hidden; key.tl = h->tap_logits;
+    key.th = h->tap_hidden; key.tl = h->tap_logits; key.tz = h->tap_zx;
     if (emb) { key.et = emb->emb_text; key.ef = emb->emb_func; }
     auto it = h->graphs.find(key);
     if (it == h->graphs.end()) {
@@ -610,6 +622,7 @@ extern "C" vc_status vc_prefill(vc_backbone* h, const void* x, int T, int slot, 
     c.ssm = state->ssm; c.conv = (uint16_t*)state->conv; c.k = (uint16_t*)state->k; c.v = (uint16_t*)state->v;
     c.ctx_len = state->ctx_len; c.status = state->status;
     c.tap = h->tap_prefill;
+    c.tap_zx = h->tap_prefill_zx;
     c.side = h->prefill_side;
     for (int i = 0; i < 5; ++i) c.ev[i] = h->pf_ev[i];
     cudaError_t e = run_prefill(c, (const uint16_t*)x, T, slot, (cudaStream_t)stream);

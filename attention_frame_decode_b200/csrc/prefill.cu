@@ -526,6 +526,9 @@ cudaError_t run_prefill(const PrefillCtx& c, const uint16_t* x, int T, int slot,
             // the GEMM's GE_ROWSCALE outputs are the bf16 in_proj values (the decode path's zx)
             if ((e = gemm(GE_ROWSCALE, b.act_d, b.ld_d, T, Lw.in_proj, b.inv, b.zx, zxw, nullptr, 0))) return e;
             m.zx = b.zx;
+            if (c.tap_zx && (e = cudaMemcpyAsync(c.tap_zx + (size_t)mi * T * zxw, b.zx, (size_t)T * zxw * 2,
+                                                 cudaMemcpyDeviceToDevice, s)))
+                return e;
             if ((e = prefill_mixer(m, s))) return e;
             if ((e = gemm(GE_RESID, b.act_big, b.ld_big, T, Lw.out_proj, nullptr, nullptr, 0, b.r, d))) return e;
             mi++;

@@ -20,6 +20,7 @@ struct PrefillCtx {
     int32_t* ctx_len;
     int32_t* status;
     float* tap;   // test tap or null: residual stream [L+1][T][d] (entry 0 = input, l+1 after layer l)
+    uint16_t* tap_zx;   // test tap or null: bf16 in_proj outputs [n_mamba][T][E+Cx+H]
     cudaStream_t side;   // weight unpacking, one GEMM ahead of the caller's stream
     cudaEvent_t ev[5];   // unpacked[2], gemm done[2], call start
 };

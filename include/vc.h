@@ -219,10 +219,16 @@ vc_status vc_prefill(vc_backbone* h, const void* x, int T, int slot, const vc_st
  * logits [2][B][max(vocab_text, vocab_func)] (text, function). */
 vc_status vc_debug_set_taps(vc_backbone* h, float* hidden, float* logits);
 
-/* test/debug tap for the next vc_prefill calls (device fp32 buffer or NULL): hidden
- * [n_layers+1][T][d], the residual stream of every prefilled frame after each layer (entry 0 =
- * input), for the T of that call; the caller sizes it. */
-vc_status vc_debug_set_prefill_taps(vc_backbone* h, float* hidden);
+/* test/debug tap for the next vc_step calls (device fp32 buffer or NULL): zx
+ * [n_mamba][B][E+Cx+H], the in_proj output of each Mamba-2 layer before its bf16 storage rounding
+ * (the mixer consumes the bf16 rounding, to nearest even, of these values). */
+vc_status vc_debug_set_zx_taps(vc_backbone* h, float* zx);
+
+/* test/debug taps for the next vc_prefill calls (device buffers or NULL), for the T of that call;
+ * the caller sizes them: hidden fp32 [n_layers+1][T][d], the residual stream of every prefilled
+ * frame after each layer (entry 0 = input); zx bf16 [n_mamba][T][E+Cx+H], each Mamba-2 layer's
+ * in_proj output as its mixer consumes it. */
+vc_status vc_debug_set_prefill_taps(vc_backbone* h, float* hidden, void* zx);
 
 /* test/debug: one Mamba-2 mixer step (the kernel vc_step runs for a Mamba-2 layer) on given
  * inputs.  zx: bf16 [B][E+Cx+H] in_proj outputs; ssm/conv: this layer's state slices

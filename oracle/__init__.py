@@ -79,6 +79,14 @@ def lib():
         L.or_step.argtypes = [C.POINTER(OrConfig), C.POINTER(OrWeights), C.POINTER(OrState), C.c_int, p, p, C.c_int,
                               p, p, p, p]
         L.or_step.restype = C.c_int
+        L.or_layer_step.argtypes = [C.POINTER(OrConfig), C.POINTER(OrWeights), C.POINTER(OrState), C.c_int, C.c_int,
+                                    p, p, C.c_int, p]
+        L.or_layer_step.restype = C.c_int
+        L.or_prefill_layer.argtypes = [C.POINTER(OrConfig), C.POINTER(OrWeights), C.POINTER(OrState), C.c_int, C.c_int,
+                                       C.c_int, p, C.c_int, C.c_int, p]
+        L.or_prefill_layer.restype = C.c_int
+        L.or_heads.argtypes = [C.POINTER(OrConfig), C.POINTER(OrWeights), C.c_int, p, C.c_int, p, p, p]
+        L.or_heads.restype = None
         L.or_prefill.argtypes = [C.POINTER(OrConfig), C.POINTER(OrWeights), C.POINTER(OrState), C.c_int, C.c_int, p,
                                  C.c_int, C.c_int, p]
         L.or_prefill.restype = C.c_int
@@ -260,6 +268,29 @@ class Model:
                            mode, tt.ctypes.data, tf.ctypes.data, _ptr(hidden), _ptr(logits))
         return dict(rc=rc, tok_text=tt, tok_func=tf, hidden=hidden, logits=logits)
 
+    def layer_step(self, st: "State", layer: int, r_in: np.ndarray, mode: int = MIRROR, slots=None):
+        """One layer teacher-forced from the residual stream r_in [B][d] entering it; updates that
+        layer's state in st (ctx_len is not advanced) and returns (rc, r_out [B][d])."""
+        r_in = np.ascontiguousarray(r_in, np.float64)
+        B = r_in.shape[0]
+        r_out = np.empty_like(r_in)
+        sl = None if slots is None else np.ascontiguousarray(slots, np.int32)
+        rc = lib().or_layer_step(C.byref(self.ocfg), C.byref(self.weights), C.byref(st.c), layer, B,
+                                 r_in.ctypes.data, _ptr(sl), mode, r_out.ctypes.data)
+        return rc, r_out
+
+    def heads(self, r: np.ndarray, mode: int = MIRROR):
+        """Final norm, both heads and the greedy tokens from the residual r [B][d] leaving the last layer."""
+        r = np.ascontiguousarray(r, np.float64)
+        B = r.shape[0]
+        tt = np.empty((B,), np.int32)
+        tf = np.empty((B,), np.int32)
+        V = max(self.cfg.vocab_text, self.cfg.vocab_func)
+        logits = np.zeros((2, B, V), np.float64)
+        lib().or_heads(C.byref(self.ocfg), C.byref(self.weights), B, r.ctypes.data, mode, tt.ctypes.data,
+                       tf.ctypes.data, logits.ctypes.data)
+        return dict(tok_text=tt, tok_func=tf, logits=logits)
+
     def prefill(self, st: "State", slot: int, x_bits: np.ndarray, mode: int = MIRROR, ssd_chunk: int = 0,
                 taps: bool = False):
         x_bits = np.ascontiguousarray(x_bits, np.uint16)
@@ -268,6 +299,17 @@ class Model:
         rc = lib().or_prefill(C.byref(self.ocfg), C.byref(self.weights), C.byref(st.c), slot, T, x_bits.ctypes.data,
                               mode, ssd_chunk, _ptr(hidden))
         return dict(rc=rc, hidden=hidden)
+
+    def prefill_layer(self, st: "State", slot: int, layer: int, r_in: np.ndarray, mode: int = MIRROR,
+                      ssd_chunk: int = 0):
+        """One prefill layer teacher-forced from the residual r_in [T][d] of the frames entering it;
+        updates that layer's state of the slot (ctx_len not advanced); returns (rc, r_out [T][d])."""
+        r_in = np.ascontiguousarray(r_in, np.float64)
+        T = r_in.shape[0]
+        r_out = np.empty_like(r_in)
+        rc = lib().or_prefill_layer(C.byref(self.ocfg), C.byref(self.weights), C.byref(st.c), slot, layer, T,
+                                    r_in.ctypes.data, mode, ssd_chunk, r_out.ctypes.data)
+        return rc, r_out
 
     def mamba_mixer(self, layer: int, zxbcdt: np.ndarray, ssm: np.ndarray, conv: np.ndarray, ssd_chunk: int = 0):
         """Isolated Mamba-2 mixer over T frames; ssm [H][P][N] and conv [W-1][Cx] are updated in place."""

@@ -470,6 +470,98 @@ static long kv_slot_size(const dims* m, int cap) { return (long)m->Hk * cap * m-
 /* decode step                                                              */
 /* ------------------------------------------------------------------------ */
 
+/* One layer of the decode step for nl live rows (residual r [nl][d] updated in place; U, Y, Y2
+ * and xc are scratch).  sl[i] is row i's state slot; mi / ai index the layer among the Mamba-2 /
+ * attention layers.  Storage points of mirror mode: P1 (u), P2 (in_proj output), P4 (gated-norm
+ * output), P5 (q, k, v), P6 (attention output), P7 (MLP hidden). */
+static void layer_forward(const dims* mp, const or_layer* L, char kind, int mi, int ai, or_state* st, int nl,
+                          const int* sl, int mode, double* r, double* U, double* Y, double* Y2, double* xc) {
+    const dims m = *mp;
+    const int d = m.d, cap = st->kv_capacity;
+    for (int i = 0; i < nl; ++i) prenorm_row(r + (long)i * d, L->norm, d, m.eps, mode, U + (long)i * d);
+    if (kind == 'M') {
+        const long R = m.E + m.Cx + m.H;
+        matmul_rows(&L->in_proj, nl, U, Y);
+        for (int i = 0; i < nl; ++i) {
+            double* zx = Y + (long)i * R;
+            for (long c = 0; c < R; ++c) zx[c] = rnd(mode, zx[c]); /* P2 */
+            int s = sl[i];
+            double* S = st->ssm + ((long)mi * st->n_slots + s) * ssm_slot_size(&m);
+            double* hist = st->conv + ((long)mi * st->n_slots + s) * conv_slot_size(&m);
+            conv_step(&m, L, hist, zx + m.E, xc);
+            double* yv = Y2 + (long)i * m.E;
+            ssm_step(&m, L, S, xc, zx + m.E + m.Cx, yv);
+            for (int c = 0; c < m.E; ++c) yv[c] *= silu(zx[c]);
+            gated_norm_row(&m, L, yv, mode, U + (long)i * m.E);
+        }
+        matmul_rows(&L->out_proj, nl, U, Y);
+        for (long k = 0; k < (long)nl * d; ++k) r[k] += Y[k];
+    } else if (kind == '*') {
+        const long R = (long)(m.Hq + 2 * m.Hk) * m.Dh;
+        matmul_rows(&L->qkv, nl, U, Y);
+        for (int i = 0; i < nl; ++i) {
+            double* qkv = Y + (long)i * R;
+            for (long c = 0; c < R; ++c) qkv[c] = rnd(mode, qkv[c]); /* P5 */
+            int s = sl[i];
+            int t = st->ctx_len[s];
+            double* Kc = st->k + ((long)ai * st->n_slots + s) * kv_slot_size(&m, cap);
+            double* Vc = st->v + ((long)ai * st->n_slots + s) * kv_slot_size(&m, cap);
+            for (int j = 0; j < m.Hk; ++j)
+                for (int e = 0; e < m.Dh; ++e) {
+                    Kc[((long)j * cap + t) * m.Dh + e] = qkv[(long)m.Hq * m.Dh + (long)j * m.Dh + e];
+                    Vc[((long)j * cap + t) * m.Dh + e] = qkv[(long)(m.Hq + m.Hk) * m.Dh + (long)j * m.Dh + e];
+                }
+            attend(&m, qkv, Kc, Vc, cap, t, mode, U + (long)i * m.Hq * m.Dh); /* P6 */
+        }
+        matmul_rows(&L->o, nl, U, Y);
+        for (long k = 0; k < (long)nl * d; ++k) r[k] += Y[k];
+    } else {
+        matmul_rows(&L->up, nl, U, Y);
+        for (long k = 0; k < (long)nl * m.F; ++k) {
+            double h = Y[k] > 0.0 ? Y[k] : 0.0;
+            U[k] = rnd(mode, h * h); /* P7 */
+        }
+        matmul_rows(&L->down, nl, U, Y);
+        for (long k = 0; k < (long)nl * d; ++k) r[k] += Y[k];
+    }
+}
+
+/* final norm (P8), the text and function heads, greedy argmax (lowest index on ties) for nl live
+ * rows; out_row[i] is the output row of live row i.  U is scratch [nl][d]. */
+static void heads_forward(const dims* mp, const or_weights* w, int nl, const int* out_row, int B, int mode,
+                          const double* r, double* U, int32_t* tok_text, int32_t* tok_func, double* logits) {
+    const dims m = *mp;
+    const int d = m.d;
+    for (int i = 0; i < nl; ++i) prenorm_row(r + (long)i * d, w->final_norm, d, m.eps, mode, U + (long)i * d);
+    for (int hsel = 0; hsel < 2; ++hsel) {
+        const or_mat* Wh = hsel == 0 ? &w->head_text : &w->head_func;
+        int V = Wh->N;
+        double* lg = malloc(sizeof(double) * (long)nl * V);
+        matmul_rows(Wh, nl, U, lg);
+        for (int i = 0; i < nl; ++i) {
+            const double* li = lg + (long)i * V;
+            int best = 0;
+            for (int v = 1; v < V; ++v)
+                if (li[v] > li[best]) best = v;
+            (hsel == 0 ? tok_text : tok_func)[out_row[i]] = best;
+            if (logits) {
+                int Vmax = m.Vt > m.Vf ? m.Vt : m.Vf;
+                memcpy(logits + ((long)hsel * B + out_row[i]) * Vmax, li, sizeof(double) * V);
+            }
+        }
+        free(lg);
+    }
+}
+
+static long scratch_width(const dims* m) {
+    long maxw = m->E + m->Cx + m->H;
+    if ((long)(m->Hq + 2 * m->Hk) * m->Dh > maxw) maxw = (long)(m->Hq + 2 * m->Hk) * m->Dh;
+    if (m->F > maxw) maxw = m->F;
+    if (m->E > maxw) maxw = m->E;
+    if (m->d > maxw) maxw = m->d;
+    return maxw;
+}
+
 int or_step(const or_config* cfg, const or_weights* w, or_state* st, int B, const uint16_t* x,
             const int32_t* slots, int mode, int32_t* tok_text, int32_t* tok_func, double* hidden,
             double* logits) {
@@ -478,6 +570,7 @@ int or_step(const or_config* cfg, const or_weights* w, or_state* st, int B, cons
     int ret = 0;
     int* live = malloc(sizeof(int) * B);
     int* slot = malloc(sizeof(int) * B);
+    int* sl = malloc(sizeof(int) * B);
     int nl = 0;
     for (int b = 0; b < B; ++b) {
         slot[b] = slots ? slots[b] : b;
@@ -485,14 +578,11 @@ int or_step(const or_config* cfg, const or_weights* w, or_state* st, int B, cons
             ret = 1;
             tok_text[b] = tok_func[b] = -1;
         } else {
+            sl[nl] = slot[b];
             live[nl++] = b;
         }
     }
-    long maxw = m.E + m.Cx + m.H;
-    if ((long)(m.Hq + 2 * m.Hk) * m.Dh > maxw) maxw = (long)(m.Hq + 2 * m.Hk) * m.Dh;
-    if (m.F > maxw) maxw = m.F;
-    if (m.E > maxw) maxw = m.E;
-    if (d > maxw) maxw = d;
+    const long maxw = scratch_width(&m);
     double* r = calloc((long)nl * d, sizeof(double));
     double* U = malloc(sizeof(double) * nl * maxw);
     double* Y = malloc(sizeof(double) * nl * maxw);
@@ -506,89 +596,110 @@ int or_step(const or_config* cfg, const or_weights* w, or_state* st, int B, cons
 
     int mi = 0, ai = 0;
     for (int l = 0; l < m.L; ++l) {
-        const or_layer* L = &w->layers[l];
         char kind = cfg->pattern[l];
-        for (int i = 0; i < nl; ++i) prenorm_row(r + (long)i * d, L->norm, d, m.eps, mode, U + (long)i * d);
-        if (kind == 'M') {
-            const long R = m.E + m.Cx + m.H;
-            matmul_rows(&L->in_proj, nl, U, Y);
-            for (int i = 0; i < nl; ++i) {
-                double* zx = Y + (long)i * R;
-                for (long c = 0; c < R; ++c) zx[c] = rnd(mode, zx[c]); /* P2 */
-                int s = slot[live[i]];
-                double* S = st->ssm + ((long)mi * st->n_slots + s) * ssm_slot_size(&m);
-                double* hist = st->conv + ((long)mi * st->n_slots + s) * conv_slot_size(&m);
-                conv_step(&m, L, hist, zx + m.E, xc);
-                double* yv = Y2 + (long)i * m.E;
-                ssm_step(&m, L, S, xc, zx + m.E + m.Cx, yv);
-                for (int c = 0; c < m.E; ++c) yv[c] *= silu(zx[c]);
-                gated_norm_row(&m, L, yv, mode, U + (long)i * m.E);
-            }
-            matmul_rows(&L->out_proj, nl, U, Y);
-            for (long k = 0; k < (long)nl * d; ++k) r[k] += Y[k];
-            mi++;
-        } else if (kind == '*') {
-            const long R = (long)(m.Hq + 2 * m.Hk) * m.Dh;
-            matmul_rows(&L->qkv, nl, U, Y);
-            for (int i = 0; i < nl; ++i) {
-                double* qkv = Y + (long)i * R;
-                for (long c = 0; c < R; ++c) qkv[c] = rnd(mode, qkv[c]); /* P5 */
-                int s = slot[live[i]];
-                int t = st->ctx_len[s];
-                double* Kc = st->k + ((long)ai * st->n_slots + s) * kv_slot_size(&m, cap);
-                double* Vc = st->v + ((long)ai * st->n_slots + s) * kv_slot_size(&m, cap);
-                for (int j = 0; j < m.Hk; ++j)
-                    for (int e = 0; e < m.Dh; ++e) {
-                        Kc[((long)j * cap + t) * m.Dh + e] = qkv[(long)m.Hq * m.Dh + (long)j * m.Dh + e];
-                        Vc[((long)j * cap + t) * m.Dh + e] = qkv[(long)(m.Hq + m.Hk) * m.Dh + (long)j * m.Dh + e];
-                    }
-                attend(&m, qkv, Kc, Vc, cap, t, mode, U + (long)i * m.Hq * m.Dh); /* P6 */
-            }
-            matmul_rows(&L->o, nl, U, Y);
-            for (long k = 0; k < (long)nl * d; ++k) r[k] += Y[k];
-            ai++;
-        } else {
-            matmul_rows(&L->up, nl, U, Y);
-            for (long k = 0; k < (long)nl * m.F; ++k) {
-                double h = Y[k] > 0.0 ? Y[k] : 0.0;
-                U[k] = rnd(mode, h * h); /* P7 */
-            }
-            matmul_rows(&L->down, nl, U, Y);
-            for (long k = 0; k < (long)nl * d; ++k) r[k] += Y[k];
-        }
+        layer_forward(&m, &w->layers[l], kind, mi, ai, st, nl, sl, mode, r, U, Y, Y2, xc);
+        if (kind == 'M') mi++;
+        if (kind == '*') ai++;
         if (hidden)
             for (int i = 0; i < nl; ++i)
                 memcpy(hidden + ((long)(l + 1) * B + live[i]) * d, r + (long)i * d, sizeof(double) * d);
     }
-
-    /* final norm (P8), the text and function heads, greedy argmax (lowest index on ties) */
-    for (int i = 0; i < nl; ++i) prenorm_row(r + (long)i * d, w->final_norm, d, m.eps, mode, U + (long)i * d);
-    for (int hsel = 0; hsel < 2; ++hsel) {
-        const or_mat* Wh = hsel == 0 ? &w->head_text : &w->head_func;
-        int V = Wh->N;
-        double* lg = malloc(sizeof(double) * (long)nl * V);
-        matmul_rows(Wh, nl, U, lg);
-        for (int i = 0; i < nl; ++i) {
-            const double* li = lg + (long)i * V;
-            int best = 0;
-            for (int v = 1; v < V; ++v)
-                if (li[v] > li[best]) best = v;
-            (hsel == 0 ? tok_text : tok_func)[live[i]] = best;
-            if (logits) {
-                int Vmax = m.Vt > m.Vf ? m.Vt : m.Vf;
-                memcpy(logits + ((long)hsel * B + live[i]) * Vmax, li, sizeof(double) * V);
-            }
-        }
-        free(lg);
-    }
+    heads_forward(&m, w, nl, live, B, mode, r, U, tok_text, tok_func, logits);
     for (int i = 0; i < nl; ++i) st->ctx_len[slot[live[i]]] += 1;
-    free(r); free(U); free(Y); free(Y2); free(xc); free(live); free(slot);
+    free(r); free(U); free(Y); free(Y2); free(xc); free(live); free(slot); free(sl);
     return ret;
+}
+
+int or_layer_step(const or_config* cfg, const or_weights* w, or_state* st, int layer, int B,
+                  const double* r_in, const int32_t* slots, int mode, double* r_out) {
+    dims m = get_dims(cfg);
+    if (layer < 0 || layer >= m.L || B < 1) return 2;
+    const int d = m.d;
+    int mi = 0, ai = 0;
+    for (int l = 0; l < layer; ++l) {
+        if (cfg->pattern[l] == 'M') mi++;
+        if (cfg->pattern[l] == '*') ai++;
+    }
+    int* sl = malloc(sizeof(int) * B);
+    for (int b = 0; b < B; ++b) sl[b] = slots ? slots[b] : b;
+    for (int b = 0; b < B; ++b)
+        if (cfg->pattern[layer] == '*' && st->ctx_len[sl[b]] >= st->kv_capacity) {
+            free(sl);
+            return 1;
+        }
+    const long maxw = scratch_width(&m);
+    double* U = malloc(sizeof(double) * B * maxw);
+    double* Y = malloc(sizeof(double) * B * maxw);
+    double* Y2 = malloc(sizeof(double) * B * maxw);
+    double* xc = malloc(sizeof(double) * m.Cx);
+    memcpy(r_out, r_in, sizeof(double) * (long)B * d);
+    layer_forward(&m, &w->layers[layer], cfg->pattern[layer], mi, ai, st, B, sl, mode, r_out, U, Y, Y2, xc);
+    free(U); free(Y); free(Y2); free(xc); free(sl);
+    return 0;
+}
+
+void or_heads(const or_config* cfg, const or_weights* w, int B, const double* r, int mode, int32_t* tok_text,
+              int32_t* tok_func, double* logits) {
+    dims m = get_dims(cfg);
+    int* rows = malloc(sizeof(int) * B);
+    for (int b = 0; b < B; ++b) rows[b] = b;
+    double* U = malloc(sizeof(double) * (long)B * m.d);
+    heads_forward(&m, w, B, rows, B, mode, r, U, tok_text, tok_func, logits);
+    free(U); free(rows);
 }
 
 /* ------------------------------------------------------------------------ */
 /* prefill (layer by layer over all T frames)                                */
 /* ------------------------------------------------------------------------ */
+
+/* One layer of the prefill over T frames of one slot whose first frame is frame t0 (residual r
+ * [T][d] updated in place; U, Y, Y2, V2 are scratch).  Same storage points as the step. */
+static void prefill_layer_forward(const dims* mp, const or_config* cfg, const or_layer* L, char kind, int mi,
+                                  int ai, or_state* st, int slot, int t0, int T, int mode, int ssd_chunk,
+                                  double* r, double* U, double* Y, double* Y2, double* V2) {
+    const dims m = *mp;
+    const int d = m.d, cap = st->kv_capacity;
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) prenorm_row(r + (long)t * d, L->norm, d, m.eps, mode, U + (long)t * d);
+    if (kind == 'M') {
+        const long R = m.E + m.Cx + m.H;
+        matmul_rows(&L->in_proj, T, U, Y);
+        for (long k = 0; k < (long)T * R; ++k) Y[k] = rnd(mode, Y[k]); /* P2 */
+        double* S = st->ssm + ((long)mi * st->n_slots + slot) * ssm_slot_size(&m);
+        double* hist = st->conv + ((long)mi * st->n_slots + slot) * conv_slot_size(&m);
+        or_mamba_mixer(cfg, L, T, Y, S, hist, ssd_chunk, Y2, V2);
+#pragma omp parallel for schedule(static)
+        for (int t = 0; t < T; ++t) gated_norm_row(&m, L, V2 + (long)t * m.E, mode, U + (long)t * m.E);
+        matmul_rows(&L->out_proj, T, U, Y);
+        for (long k = 0; k < (long)T * d; ++k) r[k] += Y[k];
+    } else if (kind == '*') {
+        const long R = (long)(m.Hq + 2 * m.Hk) * m.Dh;
+        matmul_rows(&L->qkv, T, U, Y);
+        for (long k = 0; k < (long)T * R; ++k) Y[k] = rnd(mode, Y[k]); /* P5 */
+        double* Kc = st->k + ((long)ai * st->n_slots + slot) * kv_slot_size(&m, cap);
+        double* Vc = st->v + ((long)ai * st->n_slots + slot) * kv_slot_size(&m, cap);
+        for (int t = 0; t < T; ++t)
+            for (int j = 0; j < m.Hk; ++j)
+                for (int e = 0; e < m.Dh; ++e) {
+                    Kc[((long)j * cap + t0 + t) * m.Dh + e] = Y[(long)t * R + (long)m.Hq * m.Dh + (long)j * m.Dh + e];
+                    Vc[((long)j * cap + t0 + t) * m.Dh + e] =
+                        Y[(long)t * R + (long)(m.Hq + m.Hk) * m.Dh + (long)j * m.Dh + e];
+                }
+#pragma omp parallel for schedule(dynamic, 4)
+        for (int t = 0; t < T; ++t)
+            attend(&m, Y + (long)t * R, Kc, Vc, cap, t0 + t, mode, U + (long)t * m.Hq * m.Dh); /* P6 */
+        matmul_rows(&L->o, T, U, Y);
+        for (long k = 0; k < (long)T * d; ++k) r[k] += Y[k];
+    } else {
+        matmul_rows(&L->up, T, U, Y);
+        for (long k = 0; k < (long)T * m.F; ++k) {
+            double h = Y[k] > 0.0 ? Y[k] : 0.0;
+            U[k] = rnd(mode, h * h); /* P7 */
+        }
+        matmul_rows(&L->down, T, U, Y);
+        for (long k = 0; k < (long)T * d; ++k) r[k] += Y[k];
+    }
+}
 
 int or_prefill(const or_config* cfg, const or_weights* w, or_state* st, int slot, int T,
                const uint16_t* x, int mode, int ssd_chunk, double* hidden) {
@@ -596,10 +707,7 @@ int or_prefill(const or_config* cfg, const or_weights* w, or_state* st, int slot
     const int d = m.d, cap = st->kv_capacity;
     const int t0 = st->ctx_len[slot];
     if (t0 + T > cap) return 1;
-    long maxw = m.E + m.Cx + m.H;
-    if ((long)(m.Hq + 2 * m.Hk) * m.Dh > maxw) maxw = (long)(m.Hq + 2 * m.Hk) * m.Dh;
-    if (m.F > maxw) maxw = m.F;
-    if (d > maxw) maxw = d;
+    const long maxw = scratch_width(&m);
     double* r = malloc(sizeof(double) * (long)T * d);
     double* U = malloc(sizeof(double) * (long)T * maxw);
     double* Y = malloc(sizeof(double) * (long)T * maxw);
@@ -609,54 +717,38 @@ int or_prefill(const or_config* cfg, const or_weights* w, or_state* st, int slot
     if (hidden) memcpy(hidden, r, sizeof(double) * (long)T * d);
     int mi = 0, ai = 0;
     for (int l = 0; l < m.L; ++l) {
-        const or_layer* L = &w->layers[l];
         char kind = cfg->pattern[l];
-#pragma omp parallel for schedule(static)
-        for (int t = 0; t < T; ++t) prenorm_row(r + (long)t * d, L->norm, d, m.eps, mode, U + (long)t * d);
-        if (kind == 'M') {
-            const long R = m.E + m.Cx + m.H;
-            matmul_rows(&L->in_proj, T, U, Y);
-            for (long k = 0; k < (long)T * R; ++k) Y[k] = rnd(mode, Y[k]); /* P2 */
-            double* S = st->ssm + ((long)mi * st->n_slots + slot) * ssm_slot_size(&m);
-            double* hist = st->conv + ((long)mi * st->n_slots + slot) * conv_slot_size(&m);
-            or_mamba_mixer(cfg, L, T, Y, S, hist, ssd_chunk, Y2, V2);
-#pragma omp parallel for schedule(static)
-            for (int t = 0; t < T; ++t) gated_norm_row(&m, L, V2 + (long)t * m.E, mode, U + (long)t * m.E);
-            matmul_rows(&L->out_proj, T, U, Y);
-            for (long k = 0; k < (long)T * d; ++k) r[k] += Y[k];
-            mi++;
-        } else if (kind == '*') {
-            const long R = (long)(m.Hq + 2 * m.Hk) * m.Dh;
-            matmul_rows(&L->qkv, T, U, Y);
-            for (long k = 0; k < (long)T * R; ++k) Y[k] = rnd(mode, Y[k]); /* P5 */
-            double* Kc = st->k + ((long)ai * st->n_slots + slot) * kv_slot_size(&m, cap);
-            double* Vc = st->v + ((long)ai * st->n_slots + slot) * kv_slot_size(&m, cap);
-            for (int t = 0; t < T; ++t)
-                for (int j = 0; j < m.Hk; ++j)
-                    for (int e = 0; e < m.Dh; ++e) {
-                        Kc[((long)j * cap + t0 + t) * m.Dh + e] = Y[(long)t * R + (long)m.Hq * m.Dh + (long)j * m.Dh + e];
-                        Vc[((long)j * cap + t0 + t) * m.Dh + e] =
-                            Y[(long)t * R + (long)(m.Hq + m.Hk) * m.Dh + (long)j * m.Dh + e];
-                    }
-#pragma omp parallel for schedule(dynamic, 4)
-            for (int t = 0; t < T; ++t)
-                attend(&m, Y + (long)t * R, Kc, Vc, cap, t0 + t, mode, U + (long)t * m.Hq * m.Dh); /* P6 */
-            matmul_rows(&L->o, T, U, Y);
-            for (long k = 0; k < (long)T * d; ++k) r[k] += Y[k];
-            ai++;
-        } else {
-            matmul_rows(&L->up, T, U, Y);
-            for (long k = 0; k < (long)T * m.F; ++k) {
-                double h = Y[k] > 0.0 ? Y[k] : 0.0;
-                U[k] = rnd(mode, h * h); /* P7 */
-            }
-            matmul_rows(&L->down, T, U, Y);
-            for (long k = 0; k < (long)T * d; ++k) r[k] += Y[k];
-        }
+        prefill_layer_forward(&m, cfg, &w->layers[l], kind, mi, ai, st, slot, t0, T, mode, ssd_chunk, r, U, Y, Y2,
+                              V2);
+        if (kind == 'M') mi++;
+        if (kind == '*') ai++;
         if (hidden) memcpy(hidden + (long)(l + 1) * T * d, r, sizeof(double) * (long)T * d);
     }
     st->ctx_len[slot] = t0 + T;
     free(r); free(U); free(Y); free(Y2); free(V2);
+    return 0;
+}
+
+int or_prefill_layer(const or_config* cfg, const or_weights* w, or_state* st, int slot, int layer, int T,
+                     const double* r_in, int mode, int ssd_chunk, double* r_out) {
+    dims m = get_dims(cfg);
+    if (layer < 0 || layer >= m.L || T < 1) return 2;
+    const int t0 = st->ctx_len[slot];
+    if (t0 + T > st->kv_capacity) return 1;
+    int mi = 0, ai = 0;
+    for (int l = 0; l < layer; ++l) {
+        if (cfg->pattern[l] == 'M') mi++;
+        if (cfg->pattern[l] == '*') ai++;
+    }
+    const long maxw = scratch_width(&m);
+    double* U = malloc(sizeof(double) * (long)T * maxw);
+    double* Y = malloc(sizeof(double) * (long)T * maxw);
+    double* Y2 = malloc(sizeof(double) * (long)T * m.E);
+    double* V2 = malloc(sizeof(double) * (long)T * m.E);
+    memcpy(r_out, r_in, sizeof(double) * (long)T * m.d);
+    prefill_layer_forward(&m, cfg, &w->layers[layer], cfg->pattern[layer], mi, ai, st, slot, t0, T, mode, ssd_chunk,
+                          r_out, U, Y, Y2, V2);
+    free(U); free(Y); free(Y2); free(V2);
     return 0;
 }
 

@@ -115,6 +115,22 @@ int or_step(const or_config* cfg, const or_weights* w, or_state* st, int B, cons
             const int32_t* slots, int mode, int32_t* tok_text, int32_t* tok_func, double* hidden,
             double* logits);
 
+/* One layer of the decode step, teacher-forced: the residual stream entering layer `layer` is
+ * given (r_in [B][d], double) instead of being computed from the frame input.  Runs that layer
+ * exactly as or_step does (same storage points), updating the layer's own state in st (its SSM
+ * state and conv history, or its K/V row at position ctx_len), and writes the residual leaving the
+ * layer to r_out [B][d].  ctx_len is not advanced.  slots as in or_step.
+ * Returns 0; 1 if an attention layer meets a full cache; 2 for a bad layer index.
+ * Pinned by: chaining it over every layer, then or_heads, equals or_step bit for bit, and by an
+ * independent numpy restatement of one layer of each kind with the mirror-mode roundings. */
+int or_layer_step(const or_config* cfg, const or_weights* w, or_state* st, int layer, int B,
+                  const double* r_in, const int32_t* slots, int mode, double* r_out);
+
+/* The final norm, both vocabulary heads and the greedy tokens of B rows, teacher-forced from the
+ * residual stream r [B][d] leaving the last layer.  logits (optional) [2][B][max(Vt, Vf)]. */
+void or_heads(const or_config* cfg, const or_weights* w, int B, const double* r, int mode, int32_t* tok_text,
+              int32_t* tok_func, double* logits);
+
 /* Prefill of T frames into one zero-initialised slot, layer by layer.
  * ssd_chunk = 0: Mamba-2 layers use the sequential recurrence;
  * ssd_chunk = Q > 0: they use the chunked SSD algorithm with chunk length Q.
@@ -123,6 +139,14 @@ int or_step(const or_config* cfg, const or_weights* w, or_state* st, int B, cons
  * an empty slot. */
 int or_prefill(const or_config* cfg, const or_weights* w, or_state* st, int slot, int T,
                const uint16_t* x, int mode, int ssd_chunk, double* hidden);
+
+/* One layer of or_prefill, teacher-forced: r_in [T][d] is the residual stream of the T frames
+ * entering layer `layer`; runs that layer as or_prefill does (frames ctx_len[slot] ..
+ * ctx_len[slot]+T-1 of the slot), updates the layer's state in st and writes the residual leaving
+ * the layer to r_out [T][d].  ctx_len is not advanced.  Returns 0, 1 if the frames do not fit the
+ * cache, 2 for a bad layer index.  Pinned by: chaining it over every layer equals or_prefill. */
+int or_prefill_layer(const or_config* cfg, const or_weights* w, or_state* st, int slot, int layer, int T,
+                     const double* r_in, int mode, int ssd_chunk, double* r_out);
 
 /* Isolated Mamba-2 mixer over T frames for one session (used by the kernel-level
  * checks): input zxbcdt [T][E+Cx+H] (double), state in/out ssm [H][P][N] and

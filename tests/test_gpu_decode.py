@@ -302,3 +302,85 @@ def test_mamba_step_kernel_state(cuda, T):
     ss = (v[0].reshape(cfg.ssm_heads * 2, -1) ** 2).sum(axis=1)
     assert rel(parts.cpu().numpy()[0], ss) < 1e-4
     assert int(status.cpu()[0]) == 0
+
+
+# ------------------------------------------------------------------------------------------------
+# greedy decoding picks the lowest index on exact ties (planted duplicate head rows)
+# ------------------------------------------------------------------------------------------------
+
+def _planted_rows(win, V):
+    """lower-index destinations for copies of head row `win`: its partner in the same 16-row slab
+    (rows g and g+8 share a lane and its accumulator) and a row of an earlier unit"""
+    partner = win - 8 if win % 16 >= 8 else win + 8
+    far = win - 1000 if win >= 1000 else (win + 1000) % V
+    return [r for r in (partner, far) if r != win]
+
+
+@pytest.mark.parametrize("B", [1, 16])
+@pytest.mark.parametrize("head_fmt", [synth.FMT_BF16, synth.FMT_W4])
+def test_planted_ties_pick_the_lowest_index(cuda, B, head_fmt):
+    """Both vocabulary heads get copies of session 0's winning row planted at other indices, so
+    the GPU's logits hold exact ties at the maximum.  Every session's token must be the lowest
+    index whose logit equals the maximum (read back from the logits tap), session 0's must be a
+    planted tie, and the oracle, teacher-forced from the GPU's final residual, picks the same."""
+    import torch
+    from attention_frame_decode_b200.synthetic import build_model
+    cfg = nano_layer_cfg("-", synth.FMT_W4, 64, head_fmt=head_fmt)
+    seed = 3
+    dm = build_model(cfg, seed)
+    x = torch.from_numpy(synth.frame_inputs(cfg, seed, 0, B)).cuda().view(torch.bfloat16)
+    V = max(cfg.vocab_text, cfg.vocab_func)
+
+    def run(bb):
+        st = dm.new_state(B, 64)
+        hid = torch.zeros((2, B, cfg.d_model), dtype=torch.float32, device="cuda")
+        lg = torch.zeros((2, B, V), dtype=torch.float32, device="cuda")
+        bb.set_taps(hid, lg)
+        tt = torch.zeros((B,), dtype=torch.int32, device="cuda")
+        tf = torch.zeros_like(tt)
+        bb.step(x, st, tt, tf)
+        torch.cuda.synchronize()
+        return hid.cpu().numpy(), lg.cpu().numpy(), (tt.cpu().numpy(), tf.cpu().numpy())
+
+    _, lg0, _ = run(dm.backbone(B, 64, B))
+    heads = {}
+    for hsel, (which, tid, Vh) in enumerate((("text", synth.TID_HEAD_TEXT, cfg.vocab_text),
+                                             ("func", synth.TID_HEAD_FUNC, cfg.vocab_func))):
+        w = synth.head_bf16(cfg, seed, tid) if head_fmt == synth.FMT_BF16 else synth.head_f32(cfg, seed, tid)
+        win = int(np.argmax(lg0[hsel, 0, :Vh]))
+        for r in _planted_rows(win, Vh):
+            w[r] = w[win]
+        dm.set_head(which, w)
+        heads[hsel] = (win, _planted_rows(win, Vh))
+    hid, lg, toks = run(dm.backbone(B, 64, B))
+    for hsel, Vh in ((0, cfg.vocab_text), (1, cfg.vocab_func)):
+        for b in range(B):
+            l = lg[hsel, b, :Vh]
+            tied = np.flatnonzero(l == l.max())
+            assert int(toks[hsel][b]) == int(tied[0]), (hsel, b, tied)
+        win, planted = heads[hsel]
+        l0 = lg[hsel, 0, :Vh]
+        tied0 = set(np.flatnonzero(l0 == l0.max()).tolist())
+        assert len(tied0 & set([win] + planted)) >= 2, (hsel, win, planted, tied0)
+    # the oracle with the same planted heads, from the GPU's final residual: exact ties, lowest index
+    om_heads = oracle.Model(cfg, seed)
+    for hsel, (which, tid, Vh) in enumerate((("text", synth.TID_HEAD_TEXT, cfg.vocab_text),
+                                             ("func", synth.TID_HEAD_FUNC, cfg.vocab_func))):
+        m = om_heads.head_text if hsel == 0 else om_heads.head_func
+        w = synth.head_bf16(cfg, seed, tid) if head_fmt == synth.FMT_BF16 else synth.head_f32(cfg, seed, tid)
+        win, planted = heads[hsel]
+        for r in planted:
+            w[r] = w[win]
+        nm = oracle.bf16_mat(w) if head_fmt == synth.FMT_BF16 else oracle.quantize(head_fmt, cfg.group_size, w)
+        if hsel == 0:
+            om_heads.head_text = nm
+        else:
+            om_heads.head_func = nm
+    om_heads.weights = oracle.OrWeights(om_heads.layers, oracle._ptr(om_heads.final_norm), om_heads.head_text.c(),
+                                        om_heads.head_func.c())
+    rh = om_heads.heads(hid[1].astype(np.float64), oracle.MIRROR)
+    for hsel, Vh in ((0, cfg.vocab_text), (1, cfg.vocab_func)):
+        l0 = lg[hsel, 0, :Vh]
+        below = l0[l0 < l0.max()]
+        if below.size == 0 or l0.max() - below.max() > MARGIN:     # the tied group is decidable
+            assert int((rh["tok_text"], rh["tok_func"])[hsel][0]) == int(toks[hsel][0]), hsel

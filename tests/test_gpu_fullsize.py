@@ -1,155 +1,222 @@
 """Parity at the full Nemotron-Nano-9B-v2 shape (56 layers, vocab 131072) for every decode
-workload, in the launch configuration the benchmark times (CUDA graph + programmatic
-dependent launch).
+workload, in the launch configuration the benchmark times.
 
-Reading of the 2e-2 bound through 56 layers: the stack itself amplifies rounding noise.  In
-the oracle alone, flipping the last mantissa bit of 1% of the bf16 frame inputs moves the
-residual stream after layer 56 by ~4% (max-abs / RMS) and the oracle's mirror and exact modes
-differ by as much.  Any implementation that is not bit-identical to the oracle therefore drifts
-to that floor.  The bound applied here is, per layer, max(2e-2, 2 x floor) where floor is the
-oracle's own response to that 1-ulp input perturbation, measured in the same test; the 2e-2
-bound without a floor applies to single layers (test_gpu_decode.py::test_nano_layer).  Greedy
-tokens must match wherever the oracle's top-2 margin exceeds both 1e-3 and twice the largest
-logit change that perturbation causes in the oracle itself.
+Teacher forcing: a 56-layer stack amplifies rounding (in the oracle alone, 1-ulp flips in 1% of
+the bf16 frame inputs move the residual after layer 56 by ~4%), so a free-running comparison of
+two implementations that are not bit-identical measures the stack's chaos, not the kernels.  The
+parity checks therefore give each layer of the oracle the residual stream the GPU fed that layer
+(the GPU's tap of the layer input) and the same pre-step state, and compare the layer's output:
+  * residual stream leaving every layer: max |gpu - oracle| <= 2e-2 * RMS(oracle), and the
+    layer's update (output minus input) within 2e-2 of its own RMS;
+  * logits from the GPU's final residual: 2e-2 * RMS; greedy tokens identical wherever the
+    oracle's top-2 margin exceeds 1e-3;
+  * SSM state of every Mamba-2 layer: the oracle's mixer run on the GPU's own bf16 in_proj output
+    from the same pre-step state, max |gpu - oracle| <= 1e-4 * RMS; the conv ring row the step
+    wrote equals that bf16 input bit for bit; the appended K/V rows within 2e-2 * RMS.
+The free-running comparison of the whole step is printed for information only.
 """
 import numpy as np
 import pytest
 
 import oracle
 import synth
-from tests.test_gpu_decode import HID_TOL, MARGIN, Run, rel
+from tests.test_gpu_decode import HID_TOL, MARGIN, SSM_TOL, Run, rel
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 
-def perturbed(x):
-    x = x.copy()
-    x[:, ::97] ^= 1      # last mantissa bit of ~1% of the inputs
-    return x
+def bf16_round(a):
+    """fp32 values -> the bf16 values (as float64) a round-to-nearest-even store keeps"""
+    return synth.bf16_to_f32(synth.f32_to_bf16(np.asarray(a, np.float32))).astype(np.float64)
+
+
+def teacher_forced_check(run, x, ctx, hid, lg, zx):
+    """the checks listed in the module docstring, for one GPU step whose taps are given; run.ost
+    must hold the pre-step state (it is advanced layer by layer here)"""
+    cfg, B = run.cfg, run.B
+    W = cfg.conv_width
+    ost_pre = run.ost.clone()
+    worst = 0.0
+    mi = 0
+    for l in range(cfg.n_layers):
+        rin = hid[l].astype(np.float64)
+        rc, ro = run.om.layer_step(run.ost, l, rin, oracle.MIRROR)
+        assert rc == 0
+        err = rel(hid[l + 1], ro)
+        upd = rel(hid[l + 1] - rin, ro - rin)
+        worst = max(worst, err)
+        assert err <= HID_TOL and upd <= HID_TOL, (l, cfg.pattern[l], err, upd)
+        if cfg.pattern[l] == "M":
+            zb = bf16_round(zx[mi])                                  # the mixer's bf16 inputs
+            E, Cx = cfg.d_inner, cfg.conv_dim
+            ssm_gpu = run.st.ssm[mi, :B].cpu().numpy()
+            ring = run.st.conv[mi, :B].float().cpu().numpy()
+            for b in range(B):
+                S = ost_pre.ssm[mi, b].copy()
+                hist = ost_pre.conv[mi, b].copy()
+                run.om.mamba_mixer(l, zb[b][None, :], S, hist, 0)
+                assert rel(ssm_gpu[b], S) <= SSM_TOL, (l, b, rel(ssm_gpu[b], S))
+                assert np.array_equal(ring[b, int(ctx[b]) % W].astype(np.float64), zb[b, E:E + Cx]), (l, b)
+            mi += 1
+    run.ost.ctx_len[:B] += 1
+    # the appended K/V rows against the teacher-forced oracle's
+    k = run.st.k.float().cpu().numpy()
+    v = run.st.v.float().cpu().numpy()
+    for b in range(B):
+        c = int(ctx[b])
+        assert rel(k[:, b, :, c], run.ost.k[:, b, :, c]) <= HID_TOL
+        assert rel(v[:, b, :, c], run.ost.v[:, b, :, c]) <= HID_TOL
+    # heads from the GPU's final residual
+    rh = run.om.heads(hid[cfg.n_layers].astype(np.float64), oracle.MIRROR)
+    compared = 0
+    for b in range(B):
+        for hsel, (tg, V) in enumerate(((run.tt, cfg.vocab_text), (run.tf, cfg.vocab_func))):
+            lo = rh["logits"][hsel, b, :V]
+            assert rel(lg[hsel, b, :V], lo) <= HID_TOL
+            top2 = np.sort(lo)[-2:]
+            if top2[1] - top2[0] > MARGIN:
+                compared += 1
+                assert int(tg.cpu().numpy()[b]) == int((rh["tok_text"], rh["tok_func"])[hsel][b]), (b, hsel)
+    assert compared >= B
+    return worst, ost_pre
 
 
 @pytest.mark.parametrize("name", ["nano_bf16", "nano_w4", "nano_w3", "nano_w8_b16", "nano_w4_qheads"])
 def test_full_size_decode(cuda, name):
     import torch
-    from attention_frame_decode_b200.synthetic import ring_to_history
     cfg = synth.CONFIGS[name]
     B = cfg.batch
     ctx = synth.context_lengths(cfg, 0, B)
     run = Run(cfg, 0, B, cfg.kv_capacity, ctx_lens=ctx)
-    ost_floor = run.ost.clone()
+    zx_t = torch.zeros((cfg.n_mamba, B, cfg.in_proj_rows), dtype=torch.float32, device="cuda")
+    run.bb.set_zx_taps(zx_t)
     x = synth.frame_inputs(cfg, 0, 0, B)
-    ro = run.step(0)
-    rp = run.om.step(ost_floor, perturbed(x), oracle.MIRROR, taps=True)
-
-    hid = run.hid.cpu().numpy()
-    lg = run.lg.cpu().numpy()
-    floors, errs = [], []
-    for l in range(cfg.n_layers + 1):
-        floor = rel(rp["hidden"][l], ro["hidden"][l])
-        err = rel(hid[l], ro["hidden"][l])
-        floors.append(floor)
-        errs.append(err)
-        assert err <= max(HID_TOL, 2.0 * floor), (l, err, floor)
-    print(f"{name}: layer-56 error {errs[-1]:.4f} vs perturbation floor {floors[-1]:.4f}")
-    compared = 0
-    for b in range(B):
-        for hsel, (tg, to, tp, V) in enumerate(((run.tt, ro["tok_text"], rp["tok_text"], cfg.vocab_text),
-                                                (run.tf, ro["tok_func"], rp["tok_func"], cfg.vocab_func))):
-            lo = ro["logits"][hsel, b, :V]
-            lfl = rel(rp["logits"][hsel, b, :V], lo)
-            assert rel(lg[hsel, b, :V], lo) <= max(HID_TOL, 2.0 * lfl)
-            # decidable: the margin exceeds both 1e-3 and twice the largest logit change the
-            # 1-ulp input perturbation causes in the oracle itself
-            noise = float(np.max(np.abs(rp["logits"][hsel, b, :V] - lo)))
-            top2 = np.sort(lo)[-2:]
-            if top2[1] - top2[0] > max(MARGIN, 2.0 * noise):
-                compared += 1
-                assert int(tg.cpu().numpy()[b]) == int(to[b])
-    if B > 1:
-        assert compared >= B // 2
+    run.bb.step(torch.from_numpy(x).cuda().view(torch.bfloat16), run.st, run.tt, run.tf)
+    torch.cuda.synchronize()
     assert int(run.st.status.cpu()[0]) == 0
     assert np.array_equal(run.st.ctx_len.cpu().numpy()[:B], ctx + 1)
-    # state after the frame: SSM (end to end), conv ring rows, the appended KV row
-    ssm = run.st.ssm.cpu().numpy()
-    ssm_floor = rel(ost_floor.ssm[:, :B], run.ost.ssm[:, :B])
-    assert rel(ssm[:, :B], run.ost.ssm[:, :B]) <= max(1e-4, 2.0 * ssm_floor)
-    conv = run.st.conv.float().cpu().numpy()
-    for b in range(B):
-        h = ring_to_history(conv[0, b], int(ctx[b]) + 1, cfg.conv_width)
-        assert rel(h, run.ost.conv[0, b]) < HID_TOL
-    k = run.st.k.float().cpu().numpy()
-    kf = rel(ost_floor.k[-1, 0, :, int(ctx[0])], run.ost.k[-1, 0, :, int(ctx[0])])
-    for b in range(B):
-        c = int(ctx[b])
-        assert rel(k[:, b, :, c], run.ost.k[:, b, :, c]) <= max(HID_TOL, 2.0 * kf)
+    hid = run.hid.cpu().numpy()
+    lg = run.lg.cpu().numpy()
+    worst, ost_pre = teacher_forced_check(run, x, ctx, hid, lg, zx_t.cpu().numpy())
+    # information only: the whole step free-running against the oracle's own stack
+    ro = run.om.step(ost_pre, x, oracle.MIRROR, taps=True)
+    print(f"{name}: teacher-forced worst layer error {worst:.2e}; free-running layer-56 error "
+          f"{rel(hid[-1], ro['hidden'][-1]):.3f}")
     del run
     torch.cuda.empty_cache()
 
 
-def test_full_size_prefill_equals_frame_by_frame_decode(cuda):
-    """The 4096-frame prefill of the Nano bf16 backbone (the benchmark's prefill workload) against
-    the same frames decoded one by one, both on the GPU: the oracle cannot run this size, so the
-    property checked is that the chunked path (tensor-core GEMMs, chunked SSD, flash attention)
-    and the recurrent path leave the same session state.  Bound: max(2e-2, 2 x floor) per state,
-    floor = the frame-by-frame path against itself with 1-ulp flips in ~1% of the inputs (the
-    stack's own rounding sensitivity); tokens of the next frame compared where decidable."""
+def _prefill_with_taps(cfg, T):
     import torch
-    from attention_frame_decode_b200.synthetic import build_model, ring_to_history
-    from tests.test_gpu_prefill import rel_heads, rel_stored
+    from attention_frame_decode_b200.synthetic import build_model
+    dm = build_model(cfg, 0)
+    bb = dm.backbone(1, cfg.kv_capacity, 1)
+    st = dm.new_state(1, cfg.kv_capacity)
+    x = synth.prefill_inputs(cfg, 0, T)
+    hid = torch.zeros((cfg.n_layers + 1, T, cfg.d_model), dtype=torch.float32, device="cuda")
+    zx = torch.zeros((cfg.n_mamba, T, cfg.in_proj_rows), dtype=torch.bfloat16, device="cuda")
+    bb.set_prefill_taps(hid, zx)
+    bb.prefill(torch.from_numpy(x).cuda().view(torch.bfloat16), 0, st)
+    torch.cuda.synchronize()
+    assert int(st.status.cpu()[0]) == 0 and int(st.ctx_len.cpu()[0]) == T
+    out = dict(hid=hid.cpu().numpy(), zx=synth.bf16_to_f32(zx.view(torch.int16).cpu().numpy().view(np.uint16)),
+               ssm=st.ssm[:, 0].cpu().numpy(), conv=st.conv[:, 0].float().cpu().numpy(),
+               k=st.k[:, 0, :, :, :].float().cpu().numpy()[:, :, :T], v=st.v[:, 0].float().cpu().numpy()[:, :, :T])
+    del bb, st, dm, hid, zx
+    torch.cuda.empty_cache()
+    return out
+
+
+def _mixer_check(om, cfg, l, zx_l, T, ssm_gpu, conv_gpu):
+    """the oracle's mixer on the GPU's own bf16 in_proj outputs of layer l from the zero state:
+    final SSM state within 1e-4 of RMS per head, conv ring bit-exact; returns the oracle's v"""
+    from attention_frame_decode_b200.synthetic import ring_to_history
+    from tests.test_gpu_prefill import rel_heads
+    S = np.zeros((cfg.ssm_heads, cfg.ssm_head_dim, cfg.ssm_state))
+    hist = np.zeros((cfg.conv_width - 1, cfg.conv_dim))
+    y, v = om.mamba_mixer(l, zx_l.astype(np.float64), S, hist, 0)
+    err = rel_heads(ssm_gpu, S)
+    assert err <= SSM_TOL, (l, err)
+    assert np.array_equal(ring_to_history(conv_gpu, T, cfg.conv_width).astype(np.float64), hist), l
+    return v, err
+
+
+def test_full_stack_prefill_teacher_forced(cuda):
+    """The 56-layer Nano bf16 prefill of T = 513 frames (chunks of 256, 256 and a ragged 1) against
+    the oracle's prefill, layer by layer from the GPU's taps of each layer's input: residual
+    stream of every frame and each layer's update within 2e-2 of RMS; every Mamba-2 layer's final
+    SSM state within 1e-4 (per head) of the oracle's mixer run on the GPU's own bf16 in_proj
+    outputs, conv ring bit-exact; K/V rows of every attention layer within 2e-2 of RMS (one bf16
+    rounding either way not counted)."""
+    from tests.test_gpu_prefill import rel_stored
+    cfg = synth.CONFIGS["nano_prefill"]
+    T = 513
+    g = _prefill_with_taps(cfg, T)
+    om = oracle.Model(cfg, 0)
+    ost = om.new_state(1, cfg.kv_capacity)
+    mi = ai = 0
+    worst = 0.0
+    for l in range(cfg.n_layers):
+        rin = g["hid"][l].astype(np.float64)
+        rc, ro = om.prefill_layer(ost, 0, l, rin, oracle.MIRROR)
+        assert rc == 0
+        err, upd = rel(g["hid"][l + 1], ro), rel(g["hid"][l + 1] - rin, ro - rin)
+        worst = max(worst, err)
+        assert err <= HID_TOL and upd <= HID_TOL, (l, cfg.pattern[l], err, upd)
+        if cfg.pattern[l] == "M":
+            _mixer_check(om, cfg, l, g["zx"][mi], T, g["ssm"][mi], g["conv"][mi])
+            mi += 1
+        elif cfg.pattern[l] == "*":
+            for name in ("k", "v"):
+                assert rel_stored(g[name][ai], getattr(ost, name)[ai, 0, :, :T]) <= HID_TOL, (l, name)
+            ai += 1
+    print(f"prefill T={T}: teacher-forced worst layer error {worst:.2e}")
+
+
+def test_full_size_prefill_sampled(cuda):
+    """The benchmark's prefill workload (4096 frames, 16 chunks of 256) on sampled outputs the
+    oracle can compute: every Mamba-2 layer's mixer on the GPU's own bf16 in_proj outputs over all
+    4096 frames (final state within 1e-4 per head, conv ring bit-exact) and that layer's output at
+    16 sampled frames (gated norm and out_proj of the oracle's mixer output on the GPU's layer
+    input) within 2e-2; every MLP layer teacher-forced at the sampled frames; every attention
+    layer teacher-forced over all 4096 frames (outputs and K/V within 2e-2)."""
+    from tests import mirror_layer as ml
+    from tests.test_gpu_prefill import rel_stored
     cfg = synth.CONFIGS["nano_prefill"]
     T = cfg.prefill_T
-    dm = build_model(cfg, 0)
-    bb = dm.backbone(3, cfg.kv_capacity, 3)
-    st = dm.new_state(3, cfg.kv_capacity)
-    x = synth.prefill_inputs(cfg, 0, T)
-    xd = torch.from_numpy(x).cuda().view(torch.bfloat16)
-    xp = torch.from_numpy(perturbed(x)).cuda().view(torch.bfloat16)
-    bb.prefill(xd, 0, st)                                   # slot 0: prefill
-    tt = torch.zeros((2,), dtype=torch.int32, device="cuda")
-    tf = torch.zeros_like(tt)
-    slots = torch.tensor([1, 2], dtype=torch.int32, device="cuda")
-    for t in range(T):                                      # slots 1, 2: frame by frame (2 = perturbed)
-        bb.step(torch.stack([xd[t], xp[t]]), st, tt, tf, slots=slots)
-    torch.cuda.synchronize()
-    assert int(st.status.cpu()[0]) == 0
-    assert st.ctx_len.cpu().numpy().tolist() == [T, T, T]
-    worst = {}
-    for m in range(cfg.n_mamba):
-        s = st.ssm[m].cpu().numpy()
-        err, floor = rel_heads(s[0], s[1]), rel_heads(s[2], s[1])
-        worst[f"ssm{m}"] = (err, floor)
-        assert err <= max(HID_TOL, 2.0 * floor), (m, err, floor)
-        ring = st.conv[m].float().cpu().numpy()
-        h = [ring_to_history(ring[i], T, cfg.conv_width) for i in range(3)]
-        err, floor = rel_stored(h[0], h[1]), rel_stored(h[2], h[1])
-        assert err <= max(HID_TOL, 2.0 * floor), (m, err, floor)
-    for a in range(cfg.n_attn):
-        for kv in (st.k, st.v):
-            c = kv[a, :, :, :T].float().cpu().numpy()
-            err, floor = rel_stored(c[0], c[1]), rel_stored(c[2], c[1])
-            assert err <= max(HID_TOL, 2.0 * floor), (a, err, floor)
-    print("prefill vs frame-by-frame, worst SSM (err, floor):", max(worst.values()))
-    # the next frame from all three slots: the prefilled one against the frame-by-frame one, with
-    # the perturbed one as the floor
-    x1 = torch.from_numpy(synth.frame_inputs(cfg, 0, T, 1)).cuda().view(torch.bfloat16)
-    V = max(cfg.vocab_text, cfg.vocab_func)
-    lg = torch.zeros((2, 3, V), dtype=torch.float32, device="cuda")
-    hid = torch.zeros((cfg.n_layers + 1, 3, cfg.d_model), dtype=torch.float32, device="cuda")
-    bb.set_taps(hid, lg)
-    t3 = torch.zeros((3,), dtype=torch.int32, device="cuda")
-    f3 = torch.zeros_like(t3)
-    bb.step(x1.expand(3, -1).contiguous(), st, t3, f3, slots=torch.tensor([0, 1, 2], dtype=torch.int32, device="cuda"))
-    torch.cuda.synchronize()
-    l = lg.cpu().numpy()
-    hv = hid.cpu().numpy()
-    for layer in range(cfg.n_layers + 1):
-        err, floor = rel(hv[layer, 0], hv[layer, 1]), rel(hv[layer, 2], hv[layer, 1])
-        assert err <= max(HID_TOL, 2.0 * floor), (layer, err, floor)
-    for hsel, tok in ((0, t3), (1, f3)):
-        a, b, c = l[hsel, 0], l[hsel, 1], l[hsel, 2]
-        assert rel(a, b) <= max(HID_TOL, 2.0 * rel(c, b))
-        top2 = np.sort(b)[-2:]
-        if top2[1] - top2[0] > max(MARGIN, 2.0 * float(np.max(np.abs(c - b)))):
-            assert int(tok[0]) == int(tok[1])
-    del bb
-    torch.cuda.empty_cache()
+    g = _prefill_with_taps(cfg, T)
+    om = oracle.Model(cfg, 0)
+    ost = om.new_state(1, cfg.kv_capacity)
+    frames = np.unique(np.concatenate([[0, 1, 255, 256, 257, 2047, 4094, 4095],
+                                       synth.uniform_i32(11, 0, (8,), 0, T - 1)]))
+    E, NG = cfg.d_inner, cfg.norm_groups
+    mi = ai = 0
+    for l in range(cfg.n_layers):
+        kind = cfg.pattern[l]
+        rin = g["hid"][l].astype(np.float64)
+        if kind == "M":
+            v, _ = _mixer_check(om, cfg, l, g["zx"][mi], T, g["ssm"][mi], g["conv"][mi])
+            sp = om.small[l]
+            gs = E // NG
+            for t in frames:
+                u = np.empty(E)
+                for q in range(NG):
+                    c = slice(q * gs, (q + 1) * gs)
+                    iq = 1.0 / np.sqrt(np.mean(v[t, c] ** 2) + cfg.eps)
+                    u[c] = ml.bf16(v[t, c] * sp["gnorm"][c].astype(np.float64)) * iq
+                ro = rin[t] + om.mats[(l, synth.K_OUT)].matvec(u)
+                err = rel(g["hid"][l + 1][t], ro)
+                assert err <= HID_TOL and rel(g["hid"][l + 1][t] - rin[t], ro - rin[t]) <= HID_TOL, (l, t, err)
+            mi += 1
+        elif kind == "*":
+            rc, ro = om.prefill_layer(ost, 0, l, rin, oracle.MIRROR)
+            assert rc == 0
+            assert rel(g["hid"][l + 1], ro) <= HID_TOL and rel(g["hid"][l + 1] - rin, ro - rin) <= HID_TOL, l
+            for name in ("k", "v"):
+                assert rel_stored(g[name][ai], getattr(ost, name)[ai, 0, :, :T]) <= HID_TOL, (l, name)
+            ai += 1
+        else:
+            rc, ro = om.layer_step(ost, l, rin[frames], oracle.MIRROR)
+            assert rc == 0
+            assert rel(g["hid"][l + 1][frames], ro) <= HID_TOL, l
+            assert rel(g["hid"][l + 1][frames] - rin[frames], ro - rin[frames]) <= HID_TOL, l

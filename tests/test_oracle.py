@@ -536,3 +536,110 @@ def test_mirror_mode_stores_bf16_values(how):
     dm, de = rm[1] - rm[0], re[1] - re[0]
     err = rel_err(dm, de)
     assert 0.0 < err < 2e-2
+
+
+# ------------------------------------------------------------------------------------------------
+# teacher-forced layers: the per-layer entry used by the GPU's per-layer parity checks
+# ------------------------------------------------------------------------------------------------
+
+def _prefilled(model, B, seed):
+    cfg = model.cfg
+    st = model.new_state(B, cfg.kv_capacity)
+    st.fill_random(seed, np.array([5 + 3 * b for b in range(B)], np.int32))
+    return st
+
+
+@pytest.mark.parametrize("cfg", [
+    small_cfg(),
+    small_cfg(wfmt=oracle.W4, head_fmt=oracle.W4, pattern="*MM-"),
+    synth.tiny_config(),
+])
+@pytest.mark.parametrize("mode", [oracle.MIRROR, oracle.EXACT])
+def test_layer_steps_chain_to_the_step(cfg, mode):
+    """Chaining or_layer_step over every layer and then or_heads reproduces or_step bit for bit
+    (hidden states, logits, tokens and the updated state), with sessions in permuted slots."""
+    model = oracle.Model(cfg, seed=4)
+    B = 3
+    slots = np.array([2, 0, 1], np.int32)
+    sa, sb = _prefilled(model, B, 9), _prefilled(model, B, 9)
+    x = synth.frame_inputs(cfg, 4, 0, B)
+    ro = model.step(sa, x, mode, slots=slots, taps=True)
+    r = synth.bf16_to_f32(x).astype(np.float64)
+    for l in range(cfg.n_layers):
+        rc, r = model.layer_step(sb, l, r, mode, slots=slots)
+        assert rc == 0
+        assert np.array_equal(r, ro["hidden"][l + 1])
+    sb.ctx_len[slots] += 1
+    rh = model.heads(r, mode)
+    assert np.array_equal(rh["logits"], ro["logits"])
+    assert np.array_equal(rh["tok_text"], ro["tok_text"]) and np.array_equal(rh["tok_func"], ro["tok_func"])
+    for name in ("ssm", "conv", "k", "v", "ctx_len"):
+        assert np.array_equal(getattr(sa, name), getattr(sb, name)), name
+
+
+@pytest.mark.parametrize("cfg", [
+    small_cfg(pattern="M*-", norm_groups=2),
+    small_cfg(wfmt=oracle.W8, pattern="-*M", ssm_groups=1, norm_groups=1),
+    small_cfg(wfmt=oracle.W3, head_fmt=oracle.W4, pattern="M-*"),
+])
+def test_mirror_layer_matches_numpy_restatement(cfg):
+    """Each layer kind of the oracle's mirror mode against tests/mirror_layer.py, an independent
+    numpy restatement of the layer with bf16 rounding at the storage points P1, P2, P4, P5, P6,
+    P7 and P8.  The two evaluate the same roundings of the same sums in different orders, so they
+    agree to ~1e-12; a rounding moved (say bf16 after the 1/rms scale instead of before it, or q
+    left unrounded) changes the result by ~1e-3."""
+    from tests import mirror_layer as ml
+    model = oracle.Model(cfg, seed=6)
+    B = 2
+    slots = [1, 0]
+    so, sn = _prefilled(model, B, 3), _prefilled(model, B, 3)
+    r = 2.0 * synth.normal_f32(17, 1, (B, cfg.d_model)).astype(np.float64)
+    for l in range(cfg.n_layers):
+        rc, ro = model.layer_step(so, l, r, oracle.MIRROR, slots=slots)
+        assert rc == 0
+        rn = ml.layer(model, sn, l, r, slots)
+        assert rel_err(ro - r, rn - r) < 1e-9, (l, cfg.pattern[l])
+        for name in ("ssm", "conv", "k", "v"):
+            assert rel_err(getattr(so, name), getattr(sn, name)) < 1e-9, (l, name)
+        r = ro
+    lo = model.heads(r, oracle.MIRROR)["logits"]
+    lt, lf = ml.heads(model, r)
+    assert rel_err(lo[0, :, :cfg.vocab_text], lt) < 1e-9
+    assert rel_err(lo[1, :, :cfg.vocab_func], lf) < 1e-9
+    # the pin is sensitive to where a rounding sits: one layer's update with the pre-norm rounding
+    # taken after the 1/rms scale instead of before it is far outside the bound
+    l0 = 0
+    sp = model.small[l0]
+    inv = 1.0 / np.sqrt(np.mean(r * r, axis=-1, keepdims=True) + cfg.eps)
+    moved = ml.bf16(r * sp["norm"][None, :] * inv)
+    fair = ml.bf16(r * sp["norm"][None, :]) * inv
+    assert rel_err(moved, fair) > 1e-3
+
+
+def test_teacher_forced_attention_layer_reports_a_full_cache():
+    cfg = small_cfg(pattern="*", kv_capacity=4)
+    model = oracle.Model(cfg, seed=1)
+    st = model.new_state(1, cfg.kv_capacity)
+    st.ctx_len[0] = cfg.kv_capacity
+    rc, _ = model.layer_step(st, 0, np.ones((1, cfg.d_model)), oracle.MIRROR)
+    assert rc == 1
+
+
+@pytest.mark.parametrize("chunk", [0, 4])
+def test_prefill_layers_chain_to_the_prefill(chunk):
+    """Chaining or_prefill_layer over every layer reproduces or_prefill bit for bit (hidden states
+    of every frame and the slot's final state), for a slot that already holds frames."""
+    cfg = small_cfg(pattern="M*-M", wfmt=oracle.W4)
+    model = oracle.Model(cfg, seed=8)
+    sa, sb = model.new_state(2, cfg.kv_capacity), model.new_state(2, cfg.kv_capacity)
+    T = 11
+    x = synth.prefill_inputs(cfg, 8, T)
+    ra = model.prefill(sa, 1, x, oracle.MIRROR, ssd_chunk=chunk, taps=True)
+    r = synth.bf16_to_f32(x).astype(np.float64)
+    for l in range(cfg.n_layers):
+        rc, r = model.prefill_layer(sb, 1, l, r, oracle.MIRROR, ssd_chunk=chunk)
+        assert rc == 0
+        assert np.array_equal(r, ra["hidden"][l + 1])
+    sb.ctx_len[1] += T
+    for name in ("ssm", "conv", "k", "v", "ctx_len"):
+        assert np.array_equal(getattr(sa, name), getattr(sb, name)), name
