@@ -203,30 +203,35 @@ __global__ void __launch_bounds__(256) pf_ssd_state_kernel(const float* __restri
     const int g = (int)((long long)h * G / H);
     __shared__ float w[kChunk];
     __shared__ float lam_s[kChunk];
+    __shared__ double lamd[kChunk];   // the same sums, unrounded
     extern __shared__ float stage[];   // xw [kStJ][P], bs [kStJ][N]
     float* xw = stage;
     float* bs = stage + kStJ * P;
     const float A = -expf(A_log[h]);
-    // inclusive scan of A*dt over the chunk (one warp)
+    // inclusive scan of A*dt over the chunk (one warp), summed in double (see the tensor-core
+    // state kernel): each Lam is rounded to fp32 once
     if (threadIdx.x < 32) {
-        float run = 0.0f;
+        double run = 0.0;
         for (int base = 0; base < len; base += 32) {
             const int i = base + threadIdx.x;
-            float v = i < len ? A * dt[(size_t)(t0 + i) * H + h] : 0.0f;
+            double v = i < len ? (double)(A * dt[(size_t)(t0 + i) * H + h]) : 0.0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, v, o);
+                const double u = __shfl_up_sync(0xffffffffu, v, o);
                 if ((int)threadIdx.x >= o) v += u;
             }
             v += run;
-            if (i < len) lam_s[i] = v;
+            if (i < len) {
+                lam_s[i] = (float)v;
+                lamd[i] = v;
+            }
             run = __shfl_sync(0xffffffffu, v, 31);
         }
     }
     __syncthreads();
-    const float lend = lam_s[len - 1];
+    const double lend = lamd[len - 1];   // weights from differences of the unrounded sums
     for (int i = threadIdx.x; i < len; i += blockDim.x) {
-        w[i] = expf(lend - lam_s[i]) * dt[(size_t)(t0 + i) * H + h];
+        w[i] = expf((float)(lend - lamd[i])) * dt[(size_t)(t0 + i) * H + h];
         lam[(size_t)(t0 + i) * H + h] = lam_s[i];
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -259,7 +259,7 @@ static constexpr int kStTile = 64;
 
 struct StateLayout {
     int sx, sb;
-    size_t off_xh, off_xl, off_bh, off_bl, off_w, total;
+    size_t off_xh, off_xl, off_bh, off_bl, off_w, off_ld, total;
 };
 
 __host__ __device__ inline StateLayout state_layout(int N, int P) {
@@ -273,7 +273,8 @@ __host__ __device__ inline StateLayout state_layout(int N, int P) {
     L.off_bh = 2 * rx;
     L.off_bl = 2 * rx + rb;
     L.off_w = 2 * rx + 2 * rb;
-    L.total = L.off_w + 2 * kSsdChunk * 4;
+    L.off_ld = a16(L.off_w + 2 * kSsdChunk * 4);
+    L.total = L.off_ld + kSsdChunk * 8;
     return L;
 }
 
@@ -299,28 +300,36 @@ __global__ void __launch_bounds__(256) pf_ssd_state_mma_kernel(const float* __re
     uint16_t* Bl = reinterpret_cast<uint16_t*>(smraw + L.off_bl);
     float* lam_s = reinterpret_cast<float*>(smraw + L.off_w);
     float* w = lam_s + kSsdChunk;
+    double* lamd = reinterpret_cast<double*>(smraw + L.off_ld);   // the same sums, unrounded
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
     const float A = -expf(A_log[h]);
-    // inclusive scan of A*dt over the chunk (one warp)
+    // inclusive scan of A*dt over the chunk (one warp), summed in double: over 256 frames the
+    // cumulative log decay of a fast head reaches ~100, where fp32 partial sums would carry ~1e-4
+    // of absolute error into every decay factor exp(Lam_i - Lam_j); each Lam is rounded once
     if (warp == 0) {
-        float run = 0.0f;
+        double run = 0.0;
         for (int base = 0; base < len; base += 32) {
             const int i = base + lane;
-            float v = i < len ? A * dt[(size_t)(t0 + i) * H + h] : 0.0f;
+            double v = i < len ? (double)(A * dt[(size_t)(t0 + i) * H + h]) : 0.0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, v, o);
+                const double u = __shfl_up_sync(0xffffffffu, v, o);
                 if (lane >= o) v += u;
             }
             v += run;
-            if (i < len) lam_s[i] = v;
+            if (i < len) {
+                lam_s[i] = (float)v;
+                lamd[i] = v;
+            }
             run = __shfl_sync(0xffffffffu, v, 31);
         }
     }
     __syncthreads();
-    const float lend = lam_s[len - 1];
+    // the state weights from differences of the unrounded sums: in fp32, two sums of magnitude
+    // ~200 would leave ~1e-5 of absolute error in the small differences that matter most
+    const double lend = lamd[len - 1];
     for (int i = tid; i < len; i += blockDim.x) {
-        w[i] = expf(lend - lam_s[i]) * dt[(size_t)(t0 + i) * H + h];
+        w[i] = expf((float)(lend - lamd[i])) * dt[(size_t)(t0 + i) * H + h];
         lam[(size_t)(t0 + i) * H + h] = lam_s[i];
     }
     const int npairs = N / 16;   // pairs of n8 tiles
