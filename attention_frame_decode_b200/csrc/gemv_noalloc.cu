@@ -8,17 +8,18 @@
 // kStaticSms SMs' worth of CTAs, with its scratch in g_gemv_scratch below, a fixed-size array in
 // the module's device image.  Nothing here calls cudaMalloc, cudaFree or an allocating routine.
 //
-// What must start at zero: the counters (the last kCounterInts ints of the array).  Static device
-// memory is zero when the module loads, and every launch returns each counter it uses to zero
-// (the last contributor to a unit resets it), so they stay zero between calls.  The partial sums
-// are written before they are read and need no initial value.  A launch that ended with
-// VC_DEV_TIMEOUT in the status word may leave counters non-zero; later calls are then not valid.
+// What must start at zero: the counters and the status word (the ints after the partial sums).
+// Static device memory is zero when the module loads, and every launch returns each counter it
+// uses to zero (the last contributor to a unit resets it), so they stay zero between calls.  The
+// partial sums are written before they are read and need no initial value.  The status word
+// collects the launches' device-side conditions (VC_DEV_TIMEOUT when a bounded wait for a weight
+// copy gave up); vc_gemv_noalloc_status reads it.  A launch that timed out leaves counters
+// non-zero, so results of later calls are not valid until vc_gemv_noalloc_reset clears the
+// counters and the status word (a device memset; nothing is allocated).
 //
 // One array serves every call in the process on a device: calls whose executions overlap (on
 // different streams, or from different host threads without ordering) race on it and give wrong
 // results.  Callers order them.
-#include <mutex>
-
 #include "../../include/vc.h"
 #include "gemv.cuh"
 #include "layout.cuh"
@@ -34,30 +35,21 @@ namespace {
 constexpr int kStaticSms = 32;                             // grid cap of the no-alloc launches
 constexpr size_t kPartialBytes = (size_t)4 << 20;          // 4 MiB of stream-K partial sums
 constexpr int kCounterInts = 65536;                        // arrival counters: units of 16*R rows
-constexpr size_t kScratchBytes = kPartialBytes + (size_t)kCounterInts * sizeof(int);   // 4.25 MiB
-constexpr int kMaxDevices = 64;
+constexpr size_t kStatusOffset = kPartialBytes + (size_t)kCounterInts * sizeof(int);
+// partial sums, counters, the status word (padded to 256 bytes): 4.25 MiB + 256 B
+constexpr size_t kScratchBytes = kStatusOffset + 256;
 
 static __device__ __align__(256) unsigned char g_gemv_scratch[kScratchBytes];
 
-std::mutex g_setup_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Set-up, once per device, with that device current: the device address of g_gemv_scratch,
-// looked up by the first vc_debug_gemv_noalloc call on that device and kept.
+// The device address of g_gemv_scratch on the current device.  It is looked up on every call
+// (a cheap runtime query that allocates nothing), so a device reset that reloads the module
+// does not leave a stale address behind.
 vc_status scratch_for_current_device(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return record_cuda_failure(e, "cudaGetDevice");
-    if (dev < 0 || dev >= kMaxDevices) return VC_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress((void**)&p, g_gemv_scratch);
-        if (e != cudaSuccess || !p) return record_cuda_failure(e != cudaSuccess ? e : cudaErrorUnknown,
-                                                               "cudaGetSymbolAddress(g_gemv_scratch)");
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress((void**)&p, g_gemv_scratch);
+    if (e != cudaSuccess || !p)
+        return record_cuda_failure(e != cudaSuccess ? e : cudaErrorUnknown, "cudaGetSymbolAddress(g_gemv_scratch)");
+    *out = p;
     return VC_OK;
 }
 
@@ -94,6 +86,7 @@ extern "C" vc_status vc_debug_gemv_noalloc(const vc_qmat* w, const void* act, in
     a.tap_ld = w->N;
     a.partials = (float*)scratch;
     a.counters = (int*)((unsigned char*)scratch + kPartialBytes);
+    a.status = (int*)((unsigned char*)scratch + kStatusOffset);
     GemvLaunch L{};
     L.fmt = w->fmt;
     L.group = group;
@@ -102,5 +95,27 @@ extern "C" vc_status vc_debug_gemv_noalloc(const vc_qmat* w, const void* act, in
     L.pdl = 0;
     e = launch_gemv(L, a, (cudaStream_t)stream);
     if (e != cudaSuccess) return record_cuda_failure(e, "vc_debug_gemv_noalloc launch");
+    return VC_OK;
+}
+
+extern "C" vc_status vc_gemv_noalloc_status(int32_t* status, vc_stream_t stream) {
+    if (!status) return VC_ERR_INVALID_ARG;
+    void* scratch = nullptr;
+    vc_status st = scratch_for_current_device(&scratch);
+    if (st != VC_OK) return st;
+    cudaError_t e = cudaMemcpyAsync(status, (unsigned char*)scratch + kStatusOffset, sizeof(int32_t),
+                                    cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return record_cuda_failure(e, "vc_gemv_noalloc_status");
+    return VC_OK;
+}
+
+extern "C" vc_status vc_gemv_noalloc_reset(vc_stream_t stream) {
+    void* scratch = nullptr;
+    vc_status st = scratch_for_current_device(&scratch);
+    if (st != VC_OK) return st;
+    const cudaError_t e = cudaMemsetAsync((unsigned char*)scratch + kPartialBytes, 0, kScratchBytes - kPartialBytes,
+                                          (cudaStream_t)stream);
+    if (e != cudaSuccess) return record_cuda_failure(e, "vc_gemv_noalloc_reset");
     return VC_OK;
 }
