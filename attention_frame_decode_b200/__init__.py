@@ -20,7 +20,7 @@ _lib = C.CDLL(LIB_PATH)
 VC_OK, VC_ERR_INVALID_ARG, VC_ERR_UNSUPPORTED, VC_ERR_CUDA, VC_ERR_CAPACITY, VC_ERR_STATE = range(6)
 VC_DEV_CAPACITY, VC_DEV_NONFINITE, VC_DEV_TIMEOUT = 1, 2, 4
 W_BF16, W_INT8_SYM, W_INT4_ASYM, W_INT3_ASYM = 0, 1, 2, 3
-OPT_GRAPH, OPT_PDL = 1, 2
+OPT_GRAPH, OPT_PDL, OPT_FRAME = 1, 2, 3
 
 
 class VcConfig(C.Structure):
@@ -68,6 +68,8 @@ _lib.vc_workspace_bytes.argtypes = [C.POINTER(VcConfig)]
 _lib.vc_workspace_bytes.restype = C.c_size_t
 _lib.vc_backbone_create.argtypes = [C.POINTER(VcConfig), C.POINTER(VcWeights), _p, C.c_size_t, _p, C.POINTER(_p)]
 _lib.vc_set_option.argtypes = [_p, _i, _i]
+_lib.vc_uses_frame_kernel.argtypes = [_p, _i]
+_lib.vc_uses_frame_kernel.restype = _i
 _lib.vc_step.argtypes = [_p, _p, _i, _p, C.POINTER(VcState), _p, _p, _p]
 _lib.vc_step_fused.argtypes = [_p, _p, C.POINTER(VcTokenEmbeddings), _i, _p, C.POINTER(VcState), _p, _p, _p]
 _lib.vc_step_host.argtypes = [_p, _p, _i, _p, C.POINTER(VcState), _p, _p, _p]
@@ -83,6 +85,8 @@ _lib.vc_debug_gemv.argtypes = [C.POINTER(VcQmat), _p, _i, _i, _p, _p, _p]
 _lib.vc_gemv_noalloc_scratch_bytes.argtypes = []
 _lib.vc_gemv_noalloc_scratch_bytes.restype = C.c_size_t
 _lib.vc_debug_gemv_noalloc.argtypes = [C.POINTER(VcQmat), _p, _i, _i, _p, _p]
+_lib.vc_gemv_noalloc_status.argtypes = [C.POINTER(C.c_int32), _p]
+_lib.vc_gemv_noalloc_reset.argtypes = [_p]
 _lib.vc_debug_gemm.argtypes = [_p, _i, _i, _p, _i, _i, _i, _i, _p, _i, _p, _p]
 _lib.vc_debug_mamba_prefill_scratch_bytes.argtypes = [C.POINTER(VcConfig), _i]
 _lib.vc_debug_mamba_prefill_scratch_bytes.restype = C.c_size_t
@@ -97,15 +101,17 @@ _lib.vc_last_cuda_error.restype = C.c_char_p
 for _f in ("vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant", "vc_backbone_create",
            "vc_set_option", "vc_step", "vc_step_fused", "vc_step_host", "vc_prefill", "vc_debug_set_taps",
            "vc_debug_set_prefill_taps", "vc_debug_set_zx_taps", "vc_debug_mamba_step",
-           "vc_debug_gemv", "vc_debug_gemm", "vc_debug_mamba_prefill", "vc_debug_gemv_noalloc"):
+           "vc_debug_gemv", "vc_debug_gemm", "vc_debug_mamba_prefill", "vc_debug_gemv_noalloc",
+           "vc_gemv_noalloc_status", "vc_gemv_noalloc_reset"):
     getattr(_lib, _f).restype = _i
 
 EXPORTS = ("vc_weight_bytes", "vc_quantize_weight", "vc_pack_bf16_weight", "vc_pack_weight", "vc_debug_dequant",
-           "vc_workspace_bytes", "vc_backbone_create", "vc_set_option", "vc_step", "vc_step_fused", "vc_step_host",
+           "vc_workspace_bytes", "vc_backbone_create", "vc_set_option", "vc_uses_frame_kernel", "vc_step", "vc_step_fused", "vc_step_host",
            "vc_prefill",
            "vc_debug_set_taps", "vc_debug_set_prefill_taps", "vc_debug_set_zx_taps", "vc_debug_mamba_step",
            "vc_gemv_scratch_bytes",
            "vc_debug_gemv", "vc_debug_gemm", "vc_gemv_noalloc_scratch_bytes", "vc_debug_gemv_noalloc",
+           "vc_gemv_noalloc_status", "vc_gemv_noalloc_reset",
            "vc_debug_mamba_prefill_scratch_bytes", "vc_debug_mamba_prefill", "vc_destroy",
            "vc_status_string", "vc_last_cuda_error")
 
@@ -229,6 +235,18 @@ def debug_gemv(wbuf, fmt, group, N, K, act, scratch, out=None, stream=None):
     return out
 
 
+def gemv_noalloc_status(stream=None) -> int:
+    """VC_DEV_* bits the no-allocation GEMV's launches left in its static status word"""
+    v = C.c_int32(0)
+    _check(_lib.vc_gemv_noalloc_status(C.byref(v), _stream(stream)), "vc_gemv_noalloc_status")
+    return int(v.value)
+
+
+def gemv_noalloc_reset(stream=None):
+    """zero the no-allocation GEMV's static counters and status word"""
+    _check(_lib.vc_gemv_noalloc_reset(_stream(stream)), "vc_gemv_noalloc_reset")
+
+
 def debug_gemv_noalloc(wbuf, fmt, group, N, K, act, out=None, stream=None):
     """as debug_gemv, with the library's static scratch (no scratch argument, nothing allocated
     by the library)"""
@@ -317,6 +335,10 @@ class Backbone:
 
     def set_option(self, option: int, value: int):
         _check(_lib.vc_set_option(self.h, option, value), "vc_set_option")
+
+    def uses_frame_kernel(self, B: int) -> bool:
+        """whether a step of B rows runs as one launch of the frame kernel"""
+        return bool(_lib.vc_uses_frame_kernel(self.h, B))
 
     def set_taps(self, hidden=None, logits=None):
         self._taps = (hidden, logits)

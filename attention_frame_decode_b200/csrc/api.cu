@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <map>
+#include <memory>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -13,6 +14,7 @@
 #include "../../include/vc.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "frame.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "layout.cuh"
@@ -109,6 +111,8 @@ struct Workspace {
     int32_t* tok_stage;
     uint8_t* prefill;   // prefill scratch (see prefill.cuh)
     size_t prefill_bytes;
+    FrameProgram* prog;  // the frame kernel's program (device copy)
+    int* fk_sync;        // [0] barrier arrivals, [1] abort flag of the frame kernel
 };
 
 struct GraphKey {
@@ -135,7 +139,11 @@ struct vc_backbone {
     vc_weights w;
     Workspace ws;
     int num_sms = 148;
-    int use_graph = 1, use_pdl = 1;
+    int use_graph = 1, use_pdl = 1, use_frame = 0;
+    // the frame kernel's program as last uploaded, and the call signature it was built for
+    std::unique_ptr<FrameProgram> host_prog;
+    GraphKey prog_key;
+    bool prog_valid = false;
     float* tap_hidden = nullptr;
     float* tap_logits = nullptr;
     float* tap_prefill = nullptr;
@@ -173,7 +181,8 @@ static bool dims_from_cfg(const vc_config* c, Dims& D) {
     D.B = c->max_batch; D.cap = c->kv_capacity; D.slots = c->n_slots;
     D.zx_rows = D.E + D.Cx + D.H;
     D.qkv_rows = (D.Hq + 2 * D.Hk) * D.Dh;
-    D.attn_splits = (D.cap + kAttnSplit - 1) / kAttnSplit;
+    // attention split scratch, sized for the smaller splits of the two decode paths
+    D.attn_splits = (D.cap + kFkAttnSplit - 1) / kFkAttnSplit;
     if (D.L < 1 || D.d <= 0 || D.d % 64 || D.B < 1 || D.B > 16 || D.slots < D.B || D.cap < 1) return false;
     if (D.nm) {
         if (D.H <= 0 || D.P <= 0 || D.P % 2 || D.N <= 0 || D.N % 4 || D.G <= 0 || D.H % D.G || D.W < 2 || D.W > 8)
@@ -231,6 +240,8 @@ extern "C" size_t vc_workspace_bytes(const vc_config* cfg) {
     add(2 * 16 * 4);                          // token staging
     add(prefill_workspace_bytes(D.d, D.L, D.E, D.Cx, D.H, D.P, D.N, D.G, D.Hq, D.Hk, D.Dh, D.F, D.cap));
     add(accum_floats(cfg, D) * 4);            // split-unit accumulators
+    add(sizeof(FrameProgram));                // the frame kernel's program
+    add(256);                                 // its barrier and abort words
     return align_up(total, 256);
 }
 
@@ -270,6 +281,8 @@ static void carve(vc_backbone* h, uint8_t* base) {
     W.prefill_bytes = prefill_workspace_bytes(D.d, D.L, D.E, D.Cx, D.H, D.P, D.N, D.G, D.Hq, D.Hk, D.Dh, D.F, D.cap);
     W.prefill = take(W.prefill_bytes);
     W.accum = (float*)take(accum_floats(&h->cfg, D) * 4);
+    W.prog = (FrameProgram*)take(sizeof(FrameProgram));
+    W.fk_sync = (int*)take(256);
 }
 
 static bool qmat_ok(const vc_qmat& m, int fmt, int group, int N, int K) {
@@ -348,8 +361,10 @@ extern "C" vc_status vc_set_option(vc_backbone* h, int option, int value) {
     if (!h) return VC_ERR_INVALID_ARG;
     if (option == VC_OPT_GRAPH) h->use_graph = value != 0;
     else if (option == VC_OPT_PDL) h->use_pdl = value != 0;
+    else if (option == VC_OPT_FRAME) h->use_frame = value != 0;
     else return VC_ERR_INVALID_ARG;
     clear_graphs(h);
+    h->prog_valid = false;
     return VC_OK;
 }
 
@@ -364,6 +379,7 @@ extern "C" vc_status vc_debug_set_zx_taps(vc_backbone* h, float* zx) {
     if (!h) return VC_ERR_INVALID_ARG;
     h->tap_zx = zx;
     clear_graphs(h);
+    h->prog_valid = false;
     return VC_OK;
 }
 
@@ -372,6 +388,7 @@ extern "C" vc_status vc_debug_set_taps(vc_backbone* h, float* hidden, float* log
     h->tap_hidden = hidden;
     h->tap_logits = logits;
     clear_graphs(h);
+    h->prog_valid = false;
     return VC_OK;
 }
 
@@ -380,9 +397,72 @@ static GemvMat gm(const vc_qmat& q) {
     return GemvMat{(const uint8_t*)q.data, q.N, q.K, G.NU, G.KT};
 }
 
-// the step's launch sequence (recorded into a graph, or launched directly)
+// Receives the step's sequence of operations: launched as kernels one by one (recorded into a
+// graph, or launched directly), or collected into the frame kernel's program.
+struct StepSink {
+    virtual cudaError_t input(const InputArgs& a) = 0;
+    virtual cudaError_t gemv(const GemvLaunch& l, const GemvArgs& a) = 0;
+    virtual cudaError_t mamba(const MambaStepArgs& a) = 0;
+    virtual cudaError_t attn(const AttnArgs& a) = 0;
+    virtual ~StepSink() = default;
+};
+
+struct LaunchSink : StepSink {
+    cudaStream_t s;
+    int pdl;
+    LaunchSink(cudaStream_t s_, int pdl_) : s(s_), pdl(pdl_) {}
+    cudaError_t input(const InputArgs& a) override { return launch_input(a, s); }
+    cudaError_t gemv(const GemvLaunch& l, const GemvArgs& a) override { return launch_gemv(l, a, s); }
+    cudaError_t mamba(const MambaStepArgs& a) override { return launch_mamba_step(a, pdl, s); }
+    cudaError_t attn(const AttnArgs& a) override { return launch_attn_decode(a, pdl, s); }
+};
+
+struct ProgramSink : StepSink {
+    FrameProgram& P;
+    int cap;
+    explicit ProgramSink(FrameProgram& p, int cap_) : P(p), cap(cap_) { P.n_ops = P.n_gemv = P.n_mamba = P.n_attn = 0; }
+    cudaError_t op(int kind, int idx) {
+        if (P.n_ops >= kFkMaxOps) return cudaErrorInvalidValue;
+        P.ops[P.n_ops++] = FkOp{kind, idx};
+        return cudaSuccess;
+    }
+    cudaError_t input(const InputArgs& a) override {
+        P.input = a;
+        return op(FK_INPUT, 0);
+    }
+    cudaError_t gemv(const GemvLaunch& l, const GemvArgs& a) override {
+        if (P.n_gemv >= kFkMaxGemv) return cudaErrorInvalidValue;
+        FkGemv& G = P.gemv[P.n_gemv];
+        memset(&G, 0, sizeof(G));
+        G.a = a;
+        G.epi = l.epi;
+        G.head = l.epi == EPI_ARGMAX;
+        return op(FK_GEMV, P.n_gemv++);
+    }
+    cudaError_t mamba(const MambaStepArgs& a) override {
+        if (P.n_mamba >= kFkMaxMix || P.n_gemv < 1) return cudaErrorInvalidValue;
+        // the frame kernel accumulates the gated norm's sums; the in_proj op before clears them
+        FkGemv& prev = P.gemv[P.n_gemv - 1];
+        prev.zero_buf = a.parts;
+        prev.zero_n = a.B * 2 * a.H;
+        P.mamba[P.n_mamba] = a;
+        return op(FK_MAMBA, P.n_mamba++);
+    }
+    cudaError_t attn(const AttnArgs& a) override {
+        if (P.n_attn >= kFkMaxMix) return cudaErrorInvalidValue;
+        AttnArgs f = a;
+        f.max_splits = (cap + kFkAttnSplit - 1) / kFkAttnSplit;
+        P.attn[P.n_attn] = f;
+        cudaError_t e = op(FK_ATTN, P.n_attn);
+        if (e == cudaSuccess) e = op(FK_ATTN_MERGE, P.n_attn);
+        P.n_attn++;
+        return e;
+    }
+};
+
+// the step's sequence of operations
 static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32_t* slots, const vc_state* st,
-                               int32_t* tt, int32_t* tf, const vc_token_embeddings* emb, cudaStream_t s) {
+                               int32_t* tt, int32_t* tf, const vc_token_embeddings* emb, StepSink& sink) {
     const Dims& D = h->D;
     const Workspace& W = h->ws;
     const int fmt = h->cfg.wfmt, grp = h->cfg.group_size;
@@ -390,7 +470,6 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
     const LayoutInfo LI = layout_info(fmt, fmt == VC_W_BF16 ? 64 : grp);
     const int unit_rows = 16 * LI.R;
     const int n_units_d = (D.d + unit_rows - 1) / unit_rows;
-    const int pdl = h->use_pdl;
     cudaError_t e;
 
     InputArgs ia{};
@@ -402,7 +481,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
         ia.emb_t = (const uint16_t*)emb->emb_text; ia.emb_f = (const uint16_t*)emb->emb_func;
         ia.tok_t = tt; ia.tok_f = tf; ia.Vt = D.Vt; ia.Vf = D.Vf;
     }
-    if ((e = launch_input(ia, s)) != cudaSuccess) return e;
+    if ((e = sink.input(ia)) != cudaSuccess) return e;
 
     InScale pre{};
     pre.parts = W.parts_r; pre.n_groups = 1; pre.per_group = n_units_d; pre.group_cols = W.lda;
@@ -413,7 +492,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
     base.status = st->status;
     base.slots = slots; base.ok = W.ok; base.ctx_len = st->ctx_len;
     GemvLaunch gl{};
-    gl.fmt = fmt; gl.group = grp; gl.num_sms = h->num_sms; gl.pdl = pdl;
+    gl.fmt = fmt; gl.group = grp; gl.num_sms = h->num_sms; gl.pdl = h->use_pdl;
 
     auto resid_epi = [&](GemvArgs& a, int l) {
         a.resid = W.r; a.resid_ld = D.d;
@@ -436,7 +515,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
             a.out = W.zx; a.out_ld = D.zx_rows; a.out_f16 = 0;
             if (h->tap_zx) { a.tap = h->tap_zx + (size_t)mi * B * D.zx_rows; a.tap_ld = D.zx_rows; }
             gl.epi = EPI_STORE;
-            if ((e = launch_gemv(gl, a, s)) != cudaSuccess) return e;
+            if ((e = sink.gemv(gl, a)) != cudaSuccess) return e;
 
             MambaStepArgs ma{};
             ma.zx = W.zx; ma.zx_ld = D.zx_rows;
@@ -446,7 +525,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
             ma.gnorm = Lw.gnorm; ma.act = W.act_m; ma.act_ld = W.ldm; ma.act_f16 = act_f16; ma.parts = W.parts_g;
             ma.ctx_len = st->ctx_len; ma.slots = slots; ma.ok = W.ok; ma.B = B; ma.H = D.H; ma.P = D.P; ma.N = D.N;
             ma.G = D.G; ma.W = D.W; ma.E = D.E; ma.Cx = D.Cx; ma.status = st->status;
-            if ((e = launch_mamba_step(ma, pdl, s)) != cudaSuccess) return e;
+            if ((e = sink.mamba(ma)) != cudaSuccess) return e;
 
             a = base;
             a.mat[0] = gm(Lw.out_proj); a.act = W.act_m; a.act_ld = W.ldm;
@@ -454,7 +533,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
             a.insc.group_cols = D.E / D.NG; a.insc.inv_width = (float)D.NG / D.E; a.insc.eps = h->cfg.eps;
             resid_epi(a, l);
             gl.epi = EPI_RESID;
-            if ((e = launch_gemv(gl, a, s)) != cudaSuccess) return e;
+            if ((e = sink.gemv(gl, a)) != cudaSuccess) return e;
             mi++;
         } else if (kind == '*') {
             GemvArgs a = base;
@@ -464,33 +543,33 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
             a.kcache = (uint16_t*)st->k + kvl; a.vcache = (uint16_t*)st->v + kvl;
             a.Hq = D.Hq; a.Hk = D.Hk; a.Dh = D.Dh; a.cap = D.cap;
             gl.epi = EPI_QKV;
-            if ((e = launch_gemv(gl, a, s)) != cudaSuccess) return e;
+            if ((e = sink.gemv(gl, a)) != cudaSuccess) return e;
 
             AttnArgs aa{};
             aa.q = W.q; aa.q_ld = D.Hq * D.Dh; aa.kcache = a.kcache; aa.vcache = a.vcache;
-            aa.Hq = D.Hq; aa.Hk = D.Hk; aa.Dh = D.Dh; aa.cap = D.cap; aa.max_splits = D.attn_splits;
+            aa.Hq = D.Hq; aa.Hk = D.Hk; aa.Dh = D.Dh; aa.cap = D.cap; aa.max_splits = (D.cap + kAttnSplit - 1) / kAttnSplit;
             aa.ctx_len = st->ctx_len; aa.slots = slots; aa.ok = W.ok; aa.scratch = W.attn_scratch;
             aa.counters = W.attn_counters; aa.act = W.act_o; aa.act_ld = W.ldo; aa.act_f16 = act_f16; aa.B = B;
             aa.status = st->status;
-            if ((e = launch_attn_decode(aa, pdl, s)) != cudaSuccess) return e;
+            if ((e = sink.attn(aa)) != cudaSuccess) return e;
 
             a = base;
             a.mat[0] = gm(Lw.o); a.act = W.act_o; a.act_ld = W.ldo;
             resid_epi(a, l);
             gl.epi = EPI_RESID;
-            if ((e = launch_gemv(gl, a, s)) != cudaSuccess) return e;
+            if ((e = sink.gemv(gl, a)) != cudaSuccess) return e;
             ai++;
         } else {
             GemvArgs a = base;
             a.mat[0] = gm(Lw.up); a.act = W.act_a; a.act_ld = W.lda; a.insc = pre;
             a.out = W.act_h; a.out_ld = W.ldh; a.out_f16 = act_f16;
             gl.epi = EPI_RELU2;
-            if ((e = launch_gemv(gl, a, s)) != cudaSuccess) return e;
+            if ((e = sink.gemv(gl, a)) != cudaSuccess) return e;
             a = base;
             a.mat[0] = gm(Lw.down); a.act = W.act_h; a.act_ld = W.ldh;
             resid_epi(a, l);
             gl.epi = EPI_RESID;
-            if ((e = launch_gemv(gl, a, s)) != cudaSuccess) return e;
+            if ((e = sink.gemv(gl, a)) != cudaSuccess) return e;
         }
     }
     // final norm is folded into the last residual epilogue (gamma_final) + the input scale here
@@ -504,7 +583,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
     GemvLaunch hl = gl;
     hl.fmt = h->cfg.head_fmt;
     hl.epi = EPI_ARGMAX;
-    return launch_gemv(hl, a, s);
+    return sink.gemv(hl, a);
 }
 
 static vc_status check_step_args(vc_backbone* h, const void* x, int B, const vc_state* st, const void* tt,
@@ -517,10 +596,65 @@ static vc_status check_step_args(vc_backbone* h, const void* x, int B, const vc_
     return VC_OK;
 }
 
+static FrameGeom frame_geom(const vc_backbone* h, int B) {
+    FrameGeom g{};
+    g.lfmt = h->cfg.wfmt;
+    g.lgrp = g.lfmt == VC_W_BF16 ? 64 : h->cfg.group_size;
+    g.hfmt = h->cfg.head_fmt;
+    g.hgrp = g.hfmt == VC_W_BF16 ? 64 : h->cfg.group_size;
+    g.nt = B > 8 ? 2 : 1;
+    return g;
+}
+
+// the whole frame as one launch of the frame kernel; cudaErrorNotSupported where it has no
+// instantiation for the backbone's formats and shapes (the caller then launches per kernel)
+static cudaError_t run_frame(vc_backbone* h, const void* x, int B, const int32_t* slots, const vc_state* st,
+                             int32_t* tt, int32_t* tf, cudaStream_t s, const vc_token_embeddings* emb) {
+    const FrameGeom g = frame_geom(h, B);
+    if (!frame_supported(g, h->D.na ? h->D.Hq / h->D.Hk : 1, h->D.na ? h->D.Dh : 64, h->D.nm ? h->D.N : 4))
+        return cudaErrorNotSupported;
+    int slots_per_warp = 0, slot_bytes = 0;
+    size_t smem = 0;
+    frame_ring(g, &slots_per_warp, &slot_bytes, &smem);
+    GraphKey key;
+    memset(&key, 0, sizeof(key));
+    key.B = B; key.slots = slots; key.st = *st;
+    key.th = h->tap_hidden; key.tl = h->tap_logits; key.tz = h->tap_zx;
+    if (emb) { key.et = emb->emb_text; key.ef = emb->emb_func; }
+    cudaError_t e;
+    if (!h->prog_valid || memcmp(&key, &h->prog_key, sizeof(key)) != 0) {
+        if (!h->host_prog) h->host_prog.reset(new FrameProgram());
+        ProgramSink ps(*h->host_prog, h->D.cap);
+        // the frame input and the token buffers are the launch's (FrameParams), not the program's
+        if ((e = record_step(h, x, B, slots, st, tt, tf, emb, ps)) != cudaSuccess) return e;
+        if ((e = cudaMemcpyAsync(h->ws.prog, h->host_prog.get(), sizeof(FrameProgram), cudaMemcpyHostToDevice, s)))
+            return e;
+        h->prog_key = key;
+        h->prog_valid = true;
+    }
+    FrameParams fp{};
+    fp.prog = h->ws.prog;
+    fp.x = (const uint16_t*)x;
+    fp.tok_t = tt;
+    fp.tok_f = tf;
+    fp.barrier = (unsigned*)h->ws.fk_sync;   // words 0 and 2; zero since create (workspace clear)
+    fp.abort = h->ws.fk_sync + 1;
+    fp.status = st->status;
+    fp.slots = slots_per_warp;
+    fp.slot_bytes = slot_bytes;
+    return launch_frame(g, fp, h->num_sms, s);
+}
+
 static vc_status run_step(vc_backbone* h, const void* x, int B, const int32_t* slots, const vc_state* st, int32_t* tt,
                           int32_t* tf, cudaStream_t s, const vc_token_embeddings* emb = nullptr) {
+    if (h->use_frame) {
+        const cudaError_t e = run_frame(h, x, B, slots, st, tt, tf, s, emb);
+        if (e == cudaSuccess) return VC_OK;
+        if (e != cudaErrorNotSupported) return cuda_fail(e, "vc_step frame kernel");
+    }
     if (!h->use_graph) {
-        cudaError_t e = record_step(h, x, B, slots, st, tt, tf, emb, s);
+        LaunchSink ls(s, h->use_pdl);
+        cudaError_t e = record_step(h, x, B, slots, st, tt, tf, emb, ls);
         return e == cudaSuccess ? VC_OK : cuda_fail(e, "vc_step launch");
     }
     GraphKey key;
@@ -533,7 +667,8 @@ static vc_status run_step(vc_backbone* h, const void* x, int B, const int32_t* s
         if (h->graphs.size() > 64) clear_graphs(h);
         cudaStream_t cs = h->capture_stream;
         CK(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
-        cudaError_t e = record_step(h, x, B, slots, st, tt, tf, emb, cs);
+        LaunchSink ls(cs, h->use_pdl);
+        cudaError_t e = record_step(h, x, B, slots, st, tt, tf, emb, ls);
         cudaGraph_t g = nullptr;
         cudaError_t e2 = cudaStreamEndCapture(cs, &g);
         if (e != cudaSuccess) {
@@ -572,6 +707,12 @@ static vc_status run_step(vc_backbone* h, const void* x, int B, const int32_t* s
     }
     CK(cudaGraphLaunch(G.exec, s));
     return VC_OK;
+}
+
+extern "C" int vc_uses_frame_kernel(const vc_backbone* h, int B) {
+    if (!h || B < 1 || B > h->D.B || !h->use_frame) return 0;
+    return frame_supported(frame_geom(h, B), h->D.na ? h->D.Hq / h->D.Hk : 1, h->D.na ? h->D.Dh : 64,
+                           h->D.nm ? h->D.N : 4) ? 1 : 0;
 }
 
 extern "C" vc_status vc_step(vc_backbone* h, const void* x, int B, const int32_t* slots, const vc_state* state,

@@ -86,6 +86,11 @@ TRAFFIC = {
 }
 
 
+# DRAM bytes (read + write) per frame-kernel launch, from one ncu capture of the same workload;
+# None where no capture of the current kernel exists
+FRAME_TRAFFIC = {}
+
+
 def max_over_ranks(value: float, world: int) -> float:
     """the largest of every rank's value (device timings are taken as the max over ranks);
     the tensor lives where the process group's backend wants it (CUDA for NCCL, CPU for gloo)"""
@@ -408,8 +413,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-graph", action="store_true",
-                    help="launch each step's kernels directly instead of replaying a CUDA graph (for profilers "
-                         "that cannot replay graph kernel nodes with programmatic dependencies)")
+                    help="per-kernel path: launch each step's kernels directly instead of replaying a CUDA graph "
+                         "(for profilers that cannot replay graph kernel nodes with programmatic dependencies)")
+    ap.add_argument("--per-kernel", action="store_true",
+                    help="run each frame as one kernel per operation instead of one launch of the frame kernel")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     cfg = synth.CONFIGS[args.config]
@@ -446,6 +453,9 @@ def main():
     bb = dm.backbone(B, cap, B)
     if args.no_graph:
         bb.set_option(vc.OPT_GRAPH, 0)
+    if args.per_kernel:
+        bb.set_option(vc.OPT_FRAME, 0)
+    frame = bb.uses_frame_kernel(B)
     st = dm.new_state(B, cap)
     if cfg.random_state:
         fill_state(st, cfg, seed + rank, ctx0, cap)
@@ -539,6 +549,21 @@ def main():
                "sample": f"{n_or} frame-step(s) of the same workload (batch {B}) from the same pre-filled state, "
                          f"{dt:.1f} s"}
 
+    gemv_line = {"kernel": "gemv (mlp up projection, streaming weights)", "achieved": gemv_gbs, "peak": peak,
+                 "peak_kind": peak_kind, "unit": "GB/s", "frac": gemv_gbs / peak, "launch_ms": gemv_ms,
+                 "bytes_per_launch": gemv_bytes}
+    if frame:
+        # the frame kernel is the whole step: one launch per frame, timed above on its stream
+        roofline = {"bound": "hbm", "kernel": "frame kernel (one launch per frame: all layers and both heads)",
+                    "achieved": step_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                    "frac": step_gbs / peak, "traffic": FRAME_TRAFFIC.get(cfg.name), "launch_ms": ms_step,
+                    "bytes_per_launch": rbytes}
+        launch = "frame kernel"
+        n_launches = args.steps
+    else:
+        roofline = dict(gemv_line, bound="hbm", traffic=TRAFFIC.get(cfg.name))
+        launch = "direct" if args.no_graph else "cuda graph"
+        n_launches = launches_per_step(cfg) * args.steps
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "frame-steps/s", "n_gpus": world, "steps": args.steps,
@@ -551,17 +576,14 @@ def main():
                        [int(ctx0.min()), int(ctx0.max())], "layers": cfg.n_layers, "weights": synth.FMT_NAMES[cfg.wfmt],
                        "group": cfg.group_size, "heads": synth.FMT_NAMES[cfg.head_fmt],
                        "l2": f"no flush: {weight_total / 1e9:.2f} GB of weights per step >> 126 MB L2",
-                       "parallelism": f"replicas x{world}", "launch": "direct" if args.no_graph else "cuda graph"},
+                       "parallelism": f"replicas x{world}", "launch": launch},
             "achieved_step_gbs": step_gbs, "step_bytes_read": rbytes, "step_bytes_written": wbytes,
             "step_frac_of_peak": step_gbs / peak,
-            "roofline": {"bound": "hbm", "kernel": "gemv (mlp up projection, streaming weights)",
-                         "achieved": gemv_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": gemv_gbs / peak, "traffic": TRAFFIC.get(cfg.name), "launch_ms": gemv_ms,
-                         "bytes_per_launch": gemv_bytes},
+            "roofline": roofline, "gemv_kernel_alone": gemv_line,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "frame-steps/s", "h2d_bytes_per_step": B * cfg.d_model * 2,
                     "d2h_bytes_per_step": 2 * B * 4, "steps": ne - 1},
-            "gpu_launches": launches_per_step(cfg) * args.steps,
+            "gpu_launches": n_launches,
             "clocks": clk, "device_status": status,
         }
         print(json.dumps(line), flush=True)

@@ -152,25 +152,46 @@ vc_status vc_debug_dequant(const vc_qmat* w, float* out, vc_stream_t stream);
 /* bytes of device workspace a backbone with this config needs (caller allocates) */
 size_t vc_workspace_bytes(const vc_config* cfg);
 
-/* Validates cfg and weights, carves the workspace (device, vc_workspace_bytes, zeroed here on
+/* Creates the backbone of the frame step: the 56-layer hybrid of Mamba-2 and attention layers
+ * (in the order of cfg->pattern) with its two vocabulary heads ("NemotronLabs VoiceChat 11B: GPTQ
+ * 3-bit LLM, MLX", introduction: Nemotron-Nano-9B-v2, 56 layers; "NVIDIA NemotronLabs VoiceChat
+ * 11B" blog, "Key design decisions" 2: Mamba layers interleaved with attention layers;
+ * "NemotronLabs VoiceChat" (SGLang-Omni cookbook), overview: a text head and a function head).
+ * Validates cfg and weights, carves the workspace (device, vc_workspace_bytes, zeroed here on
  * `stream`) and returns a handle.  Weight and workspace memory must stay valid until
  * vc_destroy.  Nothing is launched except the workspace clear.  VC_ERR_UNSUPPORTED (before any
  * CUDA call) for shapes the decode kernels do not cover: an attention head dim that does not
- * divide 256, or a Mamba-2 head with P/2 + 2N > 512. */
+ * divide 256, or a Mamba-2 head with P/2 + 2N > 512.  VC_ERR_INVALID_ARG for a bad config,
+ * missing or misaligned pointers or a workspace that is too small; *out is NULL then. */
 vc_status vc_backbone_create(const vc_config* cfg, const vc_weights* weights, void* workspace,
                              size_t workspace_bytes, vc_stream_t stream, vc_backbone** out);
 
-/* options: VC_OPT_GRAPH (1 = capture and replay one CUDA graph per call signature, default;
- * 0 = launch the kernels directly), VC_OPT_PDL (1 = programmatic dependent launch, default) */
+/* options: VC_OPT_FRAME (1 = run each decode frame as one launch of the persistent frame kernel
+ * where it covers the backbone's formats and shapes; 0 = one kernel per operation, default),
+ * VC_OPT_GRAPH (per-kernel path: 1 = capture and replay one CUDA graph per call signature,
+ * default; 0 = launch the kernels directly), VC_OPT_PDL (per-kernel path: 1 = programmatic
+ * dependent launch, default) */
 #define VC_OPT_GRAPH 1
 #define VC_OPT_PDL 2
+#define VC_OPT_FRAME 3
 vc_status vc_set_option(vc_backbone* h, int option, int value);
 
-/* One decode frame for B sessions (1 <= B <= max_batch).
+/* 1 if a vc_step of B rows on this backbone runs as one launch of the frame kernel (the option is
+ * on and the kernel covers the backbone's weight formats and shapes at this B), else 0 */
+int vc_uses_frame_kernel(const vc_backbone* h, int B);
+
+/* One decode frame for B sessions (1 <= B <= max_batch): each session's fused frame input
+ * goes through every layer and both heads and yields one greedy text token and one greedy
+ * function token ("NemotronLabs VoiceChat" (SGLang-Omni cookbook), overview: the thinker advances
+ * once per 80 ms frame and emits a text and a function token, decoded greedily; "NemotronLabs
+ * VoiceChat 11B: GPTQ 3-bit LLM, MLX", measurement bullets: this per-frame LLM step).
  * x: bf16 [B][d_model] (device) fused frame inputs.  slots: int32 [B] (device) session slot of
  * each row, or NULL for 0..B-1 (slots must be distinct).  tok_text, tok_func: int32 [B]
  * (device) greedy tokens (lowest index on ties).  Advances ctx_len[slot] by 1 for every
- * session whose cache had room. */
+ * session whose cache had room.  Runs as one launch of the frame kernel where it covers the
+ * backbone (vc_uses_frame_kernel), else one kernel per operation; a device-side VC_DEV_TIMEOUT
+ * (a bounded wait gave up) leaves the workspace's internal counters undefined, and the backbone
+ * must then be destroyed and created again. */
 vc_status vc_step(vc_backbone* h, const void* x, int B, const int32_t* slots, const vc_state* state,
                   int32_t* tok_text, int32_t* tok_func, vc_stream_t stream);
 
@@ -204,7 +225,8 @@ vc_status vc_step_host(vc_backbone* h, const void* x_host, int B, const int32_t*
 /* Prefill of T frames x bf16 [T][d_model] (device) into session `slot` -- the opening context a
  * streaming session consumes before its frames ("NemotronLabs VoiceChat 11B: GPTQ 3-bit LLM,
  * MLX", Recipe: the prompt is taken in as one block before the caller's speech).  The slot
- * starts empty: whatever it held is overwritten.  Mamba-2 layers run the chunked SSD (Dao & Gu, "Transformers are SSMs",
+ * starts empty: whatever it held is overwritten -- a used slot is not refused with VC_ERR_STATE,
+ * since telling a used slot from an empty one would need a read of the device's ctx_len.  Mamba-2 layers run the chunked SSD (Dao & Gu, "Transformers are SSMs",
  * chunk 256) over the frames, attention layers causal GQA; the call writes the final SSM state,
  * the conv ring (the last W-1 frames' rows, frame t in slot t mod W, the other slot zero) and
  * KV rows 0..T-1 of the slot and sets ctx_len[slot] = T.  No tokens are produced.
@@ -273,18 +295,31 @@ vc_status vc_debug_gemm(const void* A, int lda, int M, const void* W, int ldw, i
  * real-time loop, where cudaMalloc/cudaFree can synchronize the device and stall the frame; a
  * host whose device memory belongs to another allocator).  No counterpart in the method's
  * sources: an operational variant of the decode GEMV, nothing the model computes differs.
- * Same arguments, results and validation as vc_debug_gemv, without the scratch argument: the
- * scratch is a static device array of vc_gemv_noalloc_scratch_bytes() = 4.25 MiB in the
- * library (4 MiB of partial sums, 65536 arrival counters that are zero at load and that every
- * call leaves zero), and the launch uses at most 32 SMs' worth of CTAs.  A weight with more than
- * 65536 row units (16*R rows each) returns VC_ERR_CAPACITY.  The first call on a device looks
- * up the array's device address for that device and keeps it.
- * All calls on a device share the array: calls that overlap in time race and give wrong
- * results, so callers order them.  Allocates nothing. */
+ * Same arguments and argument checks as vc_debug_gemv, without the scratch argument: the scratch
+ * is a static device array of vc_gemv_noalloc_scratch_bytes() = 4.25 MiB + 256 B in the library
+ * (4 MiB of partial sums, 65536 arrival counters and a status word, the counters and status zero
+ * at load), and the launch uses at most 32 SMs' worth of CTAs.  Results equal vc_debug_gemv's
+ * up to the order of the fp32 sums (a different grid splits the rows differently), not bit for
+ * bit.  A weight with more than 65536 row units (16*R rows each) returns VC_ERR_CAPACITY.  Every
+ * call looks up the array's device address on the current device (a runtime query; nothing is
+ * allocated).  All calls on a device share the array: calls that overlap in time race and give
+ * wrong results, so callers order them.  A completed call leaves the counters zero; a call whose
+ * bounded wait for a weight copy gave up ORs VC_DEV_TIMEOUT into the status word and may leave
+ * counters non-zero, after which results are not valid until vc_gemv_noalloc_reset. */
 size_t vc_gemv_noalloc_scratch_bytes(void);
 vc_status vc_debug_gemv_noalloc(const vc_qmat* w, const void* act, int act_ld, int B, float* out,
                                 vc_stream_t stream);
+/* the status word of the no-allocation GEMV (VC_DEV_* bits of every call since load or the last
+ * reset) into *status (host); synchronizes `stream` */
+vc_status vc_gemv_noalloc_status(int32_t* status, vc_stream_t stream);
+/* zeroes the no-allocation GEMV's counters and status word on `stream` (a device memset) */
+vc_status vc_gemv_noalloc_reset(vc_stream_t stream);
 
+/* Releases the handle and what the library owns for it (host objects, CUDA graphs, its streams
+ * and events); the caller's device memory (weights, state, workspace) is left to the caller.
+ * Work the handle queued must be complete (or its stream synchronized) before the call.  The
+ * handle's lifetime spans the sessions of one served model ("NemotronLabs VoiceChat"
+ * (SGLang-Omni cookbook), overview: one thinker serves the frames of its sessions). */
 void vc_destroy(vc_backbone* h);
 
 const char* vc_status_string(vc_status s);

@@ -81,13 +81,19 @@ def teacher_forced_check(run, x, ctx, hid, lg, zx):
     return worst, ost_pre
 
 
-@pytest.mark.parametrize("name", ["nano_bf16", "nano_w4", "nano_w3", "nano_w8_b16", "nano_w4_qheads"])
-def test_full_size_decode(cuda, name):
+@pytest.mark.parametrize("name,frame", [("nano_bf16", 0), ("nano_w4", 0), ("nano_w3", 0), ("nano_w8_b16", 0),
+                                        ("nano_w4_qheads", 0), ("nano_w4", 1), ("nano_w8_b16", 1)])
+def test_full_size_decode(cuda, name, frame):
+    """frame: 1 = the frame kernel (one launch per frame), 0 = one kernel per operation"""
     import torch
+    import attention_frame_decode_b200 as vc
     cfg = synth.CONFIGS[name]
     B = cfg.batch
     ctx = synth.context_lengths(cfg, 0, B)
     run = Run(cfg, 0, B, cfg.kv_capacity, ctx_lens=ctx)
+    run.bb.set_option(vc.OPT_FRAME, frame)
+    assert run.bb.uses_frame_kernel(B) == bool(frame)
+    run.bb.set_taps(run.hid, run.lg)
     zx_t = torch.zeros((cfg.n_mamba, B, cfg.in_proj_rows), dtype=torch.float32, device="cuda")
     run.bb.set_zx_taps(zx_t)
     x = synth.frame_inputs(cfg, 0, 0, B)
