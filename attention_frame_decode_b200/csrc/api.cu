@@ -17,6 +17,7 @@
 #include "frame.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_core.cuh"
 #include "layout.cuh"
 #include "prefill.cuh"
 
@@ -466,7 +467,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
     const Dims& D = h->D;
     const Workspace& W = h->ws;
     const int fmt = h->cfg.wfmt, grp = h->cfg.group_size;
-    const int act_f16 = fmt != VC_W_BF16;
+    const int act_f16 = act_f16_for(fmt);
     const LayoutInfo LI = layout_info(fmt, fmt == VC_W_BF16 ? 64 : grp);
     const int unit_rows = 16 * LI.R;
     const int n_units_d = (D.d + unit_rows - 1) / unit_rows;
@@ -499,7 +500,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
         const bool last = l == D.L - 1;
         a.gamma_next = last ? h->w.final_norm : h->layers[l + 1].norm;
         a.act_next = W.act_a; a.act_next_ld = W.lda;
-        a.act_next_f16 = last ? (h->cfg.head_fmt != VC_W_BF16) : act_f16;
+        a.act_next_f16 = last ? act_f16_for(h->cfg.head_fmt) : act_f16;
         a.parts_next = W.parts_r; a.parts_ld = n_units_d;
         a.tap = h->tap_hidden ? h->tap_hidden + (size_t)(l + 1) * B * D.d : nullptr;
         a.tap_ld = D.d;

@@ -6,7 +6,8 @@
 
 namespace vc {
 
-static constexpr int kFrameSmemBudget = 220 * 1024;   // dynamic shared memory of one CTA
+// dynamic shared memory of one CTA for the rings (the activation area comes on top)
+static constexpr int kFrameSmemBudget = 224 * 1024 - kFkActBytes;
 
 // the instantiated (layer format, group, head format, group, column tiles) tuples
 #define VC_FRAME_FORMATS(X) \
@@ -44,7 +45,7 @@ void frame_ring(const FrameGeom& g, int* slots, int* slot_bytes, size_t* smem) {
     }
     *slots = best_ns;
     *slot_bytes = best_slot;
-    *smem = (size_t)warps * best_ns * best_slot;
+    *smem = (size_t)warps * best_ns * best_slot + kFkActBytes;
 }
 
 bool frame_supported(const FrameGeom& g, int GQ, int Dh, int N) {

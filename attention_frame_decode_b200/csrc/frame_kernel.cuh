@@ -25,7 +25,9 @@
 
 namespace vc {
 
-__host__ __device__ constexpr int fk_warps(int NT) { return NT == 1 ? 16 : 8; }
+__host__ __device__ constexpr int fk_warps(int NT) { return NT == 1 ? 12 : 8; }
+// the CTA's activation area (after the rings): one batch row of up to 16256 columns
+static constexpr int kFkActBytes = 32 * 1024 + 256;
 
 static constexpr long long kBarrierPolls = 1ll << 24;
 
@@ -174,13 +176,27 @@ VC_DEV void fk_input(const InputArgs& a, const FrameParams& fp, long long gw, lo
 // ------------------------------------------------------------------------------------------
 static constexpr int kFkRows = 4;
 
+// causal conv + SiLU of channel c for frame t: the W-1 ring rows before t and this frame's row,
+// every load issued at once (W <= 8, checked at create)
 VC_DEV float fk_conv(const MambaStepArgs& a, const uint16_t* ring, int t, int c, const uint16_t* xBC) {
-    float acc = a.conv_b[c];
-    for (int k = 0; k < a.W - 1; ++k) {
-        const int rs = ((t - (a.W - 1) + k) % a.W + a.W) % a.W;
-        acc = fmaf(a.conv_w[c * a.W + k], bf16_bits_to_f(ring[(size_t)rs * a.Cx + c]), acc);
+    float wv[8], rv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        wv[k] = 0.0f;
+        rv[k] = 0.0f;
+        if (k < a.W) {
+            wv[k] = __ldg(a.conv_w + (size_t)c * a.W + k);
+            if (k < a.W - 1) {
+                const int rs = ((t - (a.W - 1) + k) % a.W + a.W) % a.W;
+                rv[k] = bf16_bits_to_f(ring[(size_t)rs * a.Cx + c]);
+            } else {
+                rv[k] = bf16_bits_to_f(xBC[c]);
+            }
+        }
     }
-    acc = fmaf(a.conv_w[c * a.W + a.W - 1], bf16_bits_to_f(xBC[c]), acc);
+    float acc = __ldg(a.conv_b + c);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc = fmaf(wv[k], rv[k], acc);
     return silu_f(acc);
 }
 
@@ -317,6 +333,7 @@ VC_DEV void fk_mamba(const MambaStepArgs& a, long long gw, long long Wall, int l
 template <int GQ, int DPL>
 __device__ void fk_attn_t(const AttnArgs& a, long long gw, long long Wall, int lane) {
     constexpr int Dh = 32 * DPL, KB = 4, DW = DPL / 2;   // keys per load batch, 32-bit words per key
+    static_assert(kFkAttnSplit == 32, "one key per lane");
     const int MS = a.max_splits;
     const long long items = (long long)a.B * a.Hk * MS;
     const float scale = rsqrtf((float)Dh);
@@ -332,43 +349,35 @@ __device__ void fk_attn_t(const AttnArgs& a, long long gw, long long Wall, int l
         const size_t head_off = ((size_t)slot * a.Hk + j) * a.cap;
         const uint32_t* Kg = reinterpret_cast<const uint32_t*>(a.kcache + (head_off + k0) * Dh + lane * DPL);
         const uint32_t* Vg = reinterpret_cast<const uint32_t*>(a.vcache + (head_off + k0) * Dh + lane * DPL);
-        // keys of a batch (and the next batch while this one is used) are loaded together
-        uint32_t kw[KB][DW], vw[KB][DW], kn[KB][DW], vn[KB][DW];
-        auto load = [&](int k, uint32_t (&K)[KB][DW], uint32_t (&V)[KB][DW]) {
+        float q[GQ][DPL];
+#pragma unroll
+        for (int i = 0; i < GQ; ++i)
+#pragma unroll
+            for (int d = 0; d < DPL; ++d)
+                q[i][d] = bf16_bits_to_f(__ldcg(a.q + (size_t)b * a.q_ld + (size_t)(j * GQ + i) * Dh + lane * DPL + d)) *
+                          scale;
+        // 1. scores: lane l owns the dims l*DPL.., every key's dot product is a warp sum, and lane
+        //    e keeps key e's scores
+        float sm[GQ];
+#pragma unroll
+        for (int i = 0; i < GQ; ++i) sm[i] = -INFINITY;
+        uint32_t kw[KB][DW], kn[KB][DW];
+        auto loadk = [&](int k, uint32_t (&K)[KB][DW]) {
 #pragma unroll
             for (int e = 0; e < KB; ++e)
 #pragma unroll
-                for (int w = 0; w < DW; ++w) {
-                    const bool in = k + e < nk;
-                    K[e][w] = in ? __ldcg(Kg + (size_t)(k + e) * (Dh / 2) + w) : 0u;
-                    V[e][w] = in ? __ldcg(Vg + (size_t)(k + e) * (Dh / 2) + w) : 0u;
-                }
+                for (int w = 0; w < DW; ++w) K[e][w] = k + e < nk ? __ldcg(Kg + (size_t)(k + e) * (Dh / 2) + w) : 0u;
         };
-        load(0, kw, vw);
-        float q[GQ][DPL], o[GQ][DPL], m[GQ], l[GQ];
-#pragma unroll
-        for (int i = 0; i < GQ; ++i) {
-            m[i] = -INFINITY;
-            l[i] = 0.0f;
-#pragma unroll
-            for (int d = 0; d < DPL; ++d) {
-                o[i][d] = 0.0f;
-                q[i][d] = bf16_bits_to_f(__ldcg(a.q + (size_t)b * a.q_ld + (size_t)(j * GQ + i) * Dh + lane * DPL + d)) *
-                          scale;
-            }
-        }
+        loadk(0, kw);
         for (int kb = 0; kb < nk; kb += KB) {
-            if (kb + KB < nk) load(kb + KB, kn, vn);
+            if (kb + KB < nk) loadk(kb + KB, kn);
 #pragma unroll
             for (int e = 0; e < KB; ++e) {
-                if (kb + e >= nk) break;
-                float kf[DPL], vf[DPL];
+                float kf[DPL];
 #pragma unroll
                 for (int w = 0; w < DW; ++w) {
                     kf[2 * w] = __uint_as_float(kw[e][w] << 16);
                     kf[2 * w + 1] = __uint_as_float(kw[e][w] & 0xFFFF0000u);
-                    vf[2 * w] = __uint_as_float(vw[e][w] << 16);
-                    vf[2 * w + 1] = __uint_as_float(vw[e][w] & 0xFFFF0000u);
                 }
 #pragma unroll
                 for (int i = 0; i < GQ; ++i) {
@@ -376,18 +385,57 @@ __device__ void fk_attn_t(const AttnArgs& a, long long gw, long long Wall, int l
 #pragma unroll
                     for (int d = 0; d < DPL; ++d) s = fmaf(q[i][d], kf[d], s);
                     s = warp_sum(s);
-                    const float mn = fmaxf(m[i], s);
-                    const float corr = expf(m[i] - mn), ex = expf(s - mn);
-                    l[i] = fmaf(l[i], corr, ex);
-#pragma unroll
-                    for (int d = 0; d < DPL; ++d) o[i][d] = fmaf(o[i][d], corr, ex * vf[d]);
-                    m[i] = mn;
+                    if (lane == kb + e && kb + e < nk) sm[i] = s;
                 }
             }
 #pragma unroll
             for (int e = 0; e < KB; ++e)
 #pragma unroll
-                for (int w = 0; w < DW; ++w) { kw[e][w] = kn[e][w]; vw[e][w] = vn[e][w]; }
+                for (int w = 0; w < DW; ++w) kw[e][w] = kn[e][w];
+        }
+        // 2. softmax of the split: max and sum over the lanes' keys
+        float mx[GQ], pe[GQ], ls[GQ];
+#pragma unroll
+        for (int i = 0; i < GQ; ++i) {
+            mx[i] = warp_max(sm[i]);
+            pe[i] = lane < nk ? __expf(sm[i] - mx[i]) : 0.0f;
+            ls[i] = warp_sum(pe[i]);
+        }
+        // 3. unnormalised p . V: lane l owns the dims l*DPL.., key e's weights come from lane e
+        float o[GQ][DPL];
+#pragma unroll
+        for (int i = 0; i < GQ; ++i)
+#pragma unroll
+            for (int d = 0; d < DPL; ++d) o[i][d] = 0.0f;
+        uint32_t vw[KB][DW], vn[KB][DW];
+        auto loadv = [&](int k, uint32_t (&V)[KB][DW]) {
+#pragma unroll
+            for (int e = 0; e < KB; ++e)
+#pragma unroll
+                for (int w = 0; w < DW; ++w) V[e][w] = k + e < nk ? __ldcg(Vg + (size_t)(k + e) * (Dh / 2) + w) : 0u;
+        };
+        loadv(0, vw);
+        for (int kb = 0; kb < nk; kb += KB) {
+            if (kb + KB < nk) loadv(kb + KB, vn);
+#pragma unroll
+            for (int e = 0; e < KB; ++e) {
+                float vf[DPL];
+#pragma unroll
+                for (int w = 0; w < DW; ++w) {
+                    vf[2 * w] = __uint_as_float(vw[e][w] << 16);
+                    vf[2 * w + 1] = __uint_as_float(vw[e][w] & 0xFFFF0000u);
+                }
+#pragma unroll
+                for (int i = 0; i < GQ; ++i) {
+                    const float p = __shfl_sync(0xffffffffu, pe[i], (kb + e) & 31);
+#pragma unroll
+                    for (int d = 0; d < DPL; ++d) o[i][d] = fmaf(p, vf[d], o[i][d]);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < KB; ++e)
+#pragma unroll
+                for (int w = 0; w < DW; ++w) vw[e][w] = vn[e][w];
         }
         float* part = a.scratch + ((((size_t)b * a.Hk + j) * MS + sp) * GQ) * (Dh + 2);
 #pragma unroll
@@ -395,8 +443,8 @@ __device__ void fk_attn_t(const AttnArgs& a, long long gw, long long Wall, int l
 #pragma unroll
             for (int d = 0; d < DPL; ++d) part[i * (Dh + 2) + lane * DPL + d] = o[i][d];
             if (lane == 0) {
-                part[i * (Dh + 2) + Dh] = m[i];
-                part[i * (Dh + 2) + Dh + 1] = l[i];
+                part[i * (Dh + 2) + Dh] = mx[i];
+                part[i * (Dh + 2) + Dh + 1] = ls[i];
             }
         }
     }
@@ -429,10 +477,10 @@ VC_DEV void fk_attn_merge(const AttnArgs& a, long long gw, long long Wall, int l
         const int j = i / GQ, ii = i % GQ;
         const float* base = a.scratch + (((size_t)b * a.Hk + j) * MS * GQ + ii) * (Dh + 2);
         float M = -INFINITY, L = 0.0f, O = 0.0f;
-        for (int s0 = 0; s0 < nsplit; s0 += 8) {   // eight splits' loads in flight together
-            float ms[8], ls[8], os[8];
+        for (int s0 = 0; s0 < nsplit; s0 += 16) {   // sixteen splits' loads in flight together
+            float ms[16], ls[16], os[16];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < 16; ++e) {
                 const float* p = base + (size_t)(s0 + e) * GQ * (Dh + 2);
                 const bool in = s0 + e < nsplit;
                 ms[e] = in ? __ldcg(p + Dh) : -INFINITY;
@@ -440,10 +488,10 @@ VC_DEV void fk_attn_merge(const AttnArgs& a, long long gw, long long Wall, int l
                 os[e] = in ? __ldcg(p + d) : 0.0f;
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < 16; ++e) {
                 if (s0 + e >= nsplit) break;
                 const float mn = fmaxf(M, ms[e]);
-                const float c0 = expf(M - mn), c1 = expf(ms[e] - mn);
+                const float c0 = __expf(M - mn), c1 = __expf(ms[e] - mn);
                 L = L * c0 + ls[e] * c1;
                 O = O * c0 + os[e] * c1;
                 M = mn;
@@ -478,103 +526,171 @@ __device__ __forceinline__ void fk_flush_any(int epi, const GemvArgs& a, const W
     }
 }
 
-template <int FMT, int GRP, int NT>
-__device__ __forceinline__ void fk_load_bv(const GemvArgs& a, int kt, int lane, uint4 (&bv)[layout_info(FMT, GRP).SUB][NT][2]) {
-    constexpr LayoutInfo L = layout_info(FMT, GRP);
-    const int g = lane >> 2, t = lane & 3;
+// The activation of a projection: staged whole in shared memory when it fits the CTA's
+// activation area (every block's fragments are then a shared-memory load), else read from L2
+// one block ahead of its use.
+template <int FMT, int GRP, int NT, bool ACT_SMEM>
+struct FkAct {
+    static constexpr LayoutInfo L = layout_info(FMT, GRP);
+    const uint4* row[NT];   // the lane's row 8j + g (rows past the batch read its last row: their
+                            // sums are computed and never stored), at column 16t, in uint4
+    __device__ __forceinline__ void load(int kt, uint4 (&bv)[L.SUB][NT][2]) const {
 #pragma unroll
-    for (int st = 0; st < L.SUB; ++st)
+        for (int st = 0; st < L.SUB; ++st)
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            const int b = 8 * j + g;
-            bv[st][j][0] = bv[st][j][1] = make_uint4(0, 0, 0, 0);
-            if (b < a.B) {
-                const uint4* p = reinterpret_cast<const uint4*>(a.act + (size_t)b * a.act_ld + (size_t)kt * L.KS +
-                                                                64 * st + 16 * t);
-                bv[st][j][0] = __ldcg(p);
-                bv[st][j][1] = __ldcg(p + 1);
+            for (int j = 0; j < NT; ++j) {
+                const uint4* p = row[j] + kt * (L.KS / 8) + 8 * st;
+                if constexpr (ACT_SMEM) {
+                    bv[st][j][0] = p[0];
+                    bv[st][j][1] = p[1];
+                } else {
+                    bv[st][j][0] = __ldcg(p);
+                    bv[st][j][1] = __ldcg(p + 1);
+                }
             }
-        }
-}
+    }
+};
 
-// returns false when the launch must wind down (a copy never arrived)
-template <int LF, int LG, int HF, int HG, int FMT, int GRP, int NT>
-__device__ bool fk_gemv(const FkGemv& G, const float* insc_tab, const FrameParams& fp, long long gw, long long Wall,
-                        int lane, uint8_t* ring, uint64_t* bar, int n_ops, FkStream& ps, int& ccount) {
+// the warp's share of one projection; false when the launch must wind down (a copy never arrived)
+template <int LF, int LG, int HF, int HG, int FMT, int GRP, int NT, bool ACT_SMEM>
+__device__ __forceinline__ bool fk_gemv_run(const FkGemv& G, const float* insc_tab, const FkAct<FMT, GRP, NT, ACT_SMEM>& act,
+                                            const WarpRange& wr, const FrameParams& fp, long long gw, long long Wall,
+                                            int lane, uint8_t* ring, uint64_t* bar, int n_ops, FkStream& ps, int& ccount,
+                                            unsigned long long (&best)[NT][2]) {
     constexpr LayoutInfo L = layout_info(FMT, GRP);
     constexpr int R = L.R, KS = L.KS;
     const GemvArgs& a = G.a;
     const int B = a.B, t = lane & 3;
-    const WarpRange wr = warp_range(a.mat, a.nmat, gw, Wall);
-    unsigned long long best[NT][2];
+    const int KT = wr.M.KT;
+    const int bpc = max(1, fp.slot_bytes / L.block_bytes);
+    const int ng = a.insc.parts ? a.insc.n_groups : 1;
+    float acc[R][NT][4];
+    auto zero_acc = [&]() {
 #pragma unroll
-    for (int j = 0; j < NT; ++j) best[j][0] = best[j][1] = 0ull;
-    bool alive = true;
-    if (!wr.idle && wr.f0 < wr.f1) {
-        const int KT = wr.M.KT;
-        const int bpc = max(1, fp.slot_bytes / L.block_bytes);
-        const int ng = a.insc.parts ? a.insc.n_groups : 1;
-        float acc[R][NT][4];
-        auto zero_acc = [&]() {
+        for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int r = 0; r < R; ++r)
+            for (int j = 0; j < NT; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[r][j][e] = 0.0f;
+    };
+    zero_acc();
+    int cur_u = wr.f0 / KT, kt = wr.f0 % KT;
+    bool pending = false;
+    float sc[NT][2];
+    int sc_next = kt;
+    uint4 bv[L.SUB][NT][2];
+    if constexpr (!ACT_SMEM) act.load(kt, bv);
+    for (int f = wr.f0; f < wr.f1;) {
+        const int nb = min(bpc, wr.f1 - f);
+        const int slot = ccount % fp.slots;
+        const uint32_t phase = (uint32_t)(ccount / fp.slots) & 1u;
+        if (!mbar_wait(&bar[slot], phase, fp.status)) return false;
+        const uint8_t* base = ring + (size_t)slot * fp.slot_bytes;
+        for (int jb = 0; jb < nb; ++jb) {
+            if (kt == sc_next) {
+                const int qg = ng > 1 ? (kt * KS) / a.insc.group_cols : 0;
+                sc_next = ng > 1 ? min(KT, ((qg + 1) * a.insc.group_cols) / KS) : KT;
 #pragma unroll
                 for (int j = 0; j < NT; ++j)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[r][j][e] = 0.0f;
-        };
-        zero_acc();
-        int cur_u = wr.f0 / KT, kt = wr.f0 % KT;
-        bool pending = false;
-        float sc[NT][2];
-        int sc_next = kt;
-        uint4 bv[L.SUB][NT][2];
-        fk_load_bv<FMT, GRP, NT>(a, kt, lane, bv);
-        for (int f = wr.f0; f < wr.f1;) {
-            const int nb = min(bpc, wr.f1 - f);
-            const int slot = ccount % fp.slots;
-            const uint32_t phase = (uint32_t)(ccount / fp.slots) & 1u;
-            if (!mbar_wait(&bar[slot], phase, fp.status)) { alive = false; break; }
-            const uint8_t* base = ring + (size_t)slot * fp.slot_bytes;
-            for (int jb = 0; jb < nb; ++jb) {
-                if (kt == sc_next) {
-                    const int qg = ng > 1 ? (kt * KS) / a.insc.group_cols : 0;
-                    sc_next = ng > 1 ? min(KT, ((qg + 1) * a.insc.group_cols) / KS) : KT;
-#pragma unroll
-                    for (int j = 0; j < NT; ++j)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int b = 8 * j + 2 * t + e;
-                            sc[j][e] = b < B ? insc_tab[b * ng + qg] : 0.0f;
-                        }
-                }
+                    for (int e = 0; e < 2; ++e) {
+                        const int b = 8 * j + 2 * t + e;
+                        sc[j][e] = b < B ? insc_tab[b * ng + qg] : 0.0f;
+                    }
+            }
+            if constexpr (ACT_SMEM) {
+                act.load(kt, bv);
+                consume_block_bv<FMT, GRP, NT>(base + jb * L.block_bytes, bv, lane, sc, acc);
+            } else {
                 uint4 bn[L.SUB][NT][2];
-                const int kn = kt + 1 == KT ? 0 : kt + 1;
-                fk_load_bv<FMT, GRP, NT>(a, kn, lane, bn);   // one block ahead
+                act.load(kt + 1 == KT ? 0 : kt + 1, bn);   // one block ahead
                 consume_block_bv<FMT, GRP, NT>(base + jb * L.block_bytes, bv, lane, sc, acc);
 #pragma unroll
                 for (int st = 0; st < L.SUB; ++st)
 #pragma unroll
                     for (int j = 0; j < NT; ++j) { bv[st][j][0] = bn[st][j][0]; bv[st][j][1] = bn[st][j][1]; }
-                pending = true;
-                if (++kt == KT) {
-                    fk_flush_any<FMT, GRP, NT>(G.epi, a, wr, cur_u, acc, best, lane);
-                    zero_acc();
-                    pending = false;
-                    kt = 0;
-                    ++cur_u;
-                    if (ng > 1) sc_next = 0;
-                }
             }
-            __syncwarp();
-            if (lane == 0) {
-                fence_proxy_async();
-                fk_issue<LF, LG, HF, HG>(fp.prog, n_ops, gw, Wall, fp.slot_bytes, ps, ring, bar, slot);
+            pending = true;
+            if (++kt == KT) {
+                fk_flush_any<FMT, GRP, NT>(G.epi, a, wr, cur_u, acc, best, lane);
+                zero_acc();
+                pending = false;
+                kt = 0;
+                ++cur_u;
+                if (ng > 1) sc_next = 0;
             }
-            ++ccount;
-            f += nb;
         }
-        if (alive && pending) fk_flush_any<FMT, GRP, NT>(G.epi, a, wr, cur_u, acc, best, lane);
+        __syncwarp();
+        if (lane == 0) {
+            fence_proxy_async();
+            fk_issue<LF, LG, HF, HG>(fp.prog, n_ops, gw, Wall, fp.slot_bytes, ps, ring, bar, slot);
+        }
+        ++ccount;
+        f += nb;
+    }
+    if (pending) fk_flush_any<FMT, GRP, NT>(G.epi, a, wr, cur_u, acc, best, lane);
+    return true;
+}
+
+// one projection: the CTA stages the activation (when it fits its activation area) and builds
+// the input-scale table, then every warp runs its share
+template <int LF, int LG, int HF, int HG, int FMT, int GRP, int NT, int WARPS>
+__device__ bool fk_gemv(const FkGemv& G, float* insc_tab, uint4* act_s, int act_s_bytes, const FrameParams& fp,
+                        long long gw, long long Wall, int warp, int lane, uint8_t* ring, uint64_t* bar, int n_ops,
+                        FkStream& ps, int& ccount) {
+    constexpr LayoutInfo L = layout_info(FMT, GRP);
+    const GemvArgs& a = G.a;
+    const int B = a.B, t = lane & 3;
+    const WarpRange wr = warp_range(a.mat, a.nmat, gw, Wall);
+    const bool busy = !wr.idle && wr.f0 < wr.f1;
+    // activation rows of KT * KS columns, padded by 16 bytes against bank conflicts
+    const int rowq = wr.M.KT * (L.KS / 8) + 1;
+    const bool smem_act = B * rowq * 16 <= act_s_bytes;
+    if (smem_act) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.act);
+        const int ldq = a.act_ld / 8;
+        for (int i = threadIdx.x; i < B * (rowq - 1); i += blockDim.x) {
+            const int b = i / (rowq - 1), c = i - b * (rowq - 1);
+            act_s[b * rowq + c] = __ldcg(src + (size_t)b * ldq + c);
+        }
+    }
+    {
+        const InScale& is = a.insc;
+        const int ng = is.parts ? is.n_groups : 1;
+        for (int idx = warp; idx < B * ng; idx += WARPS) {
+            float v = 1.0f;
+            if (is.parts) {
+                const int b = idx / ng, q = idx % ng;
+                const float* p = is.parts + ((size_t)b * ng + q) * is.per_group;
+                float s = 0.0f;
+                for (int i = lane; i < is.per_group; i += 32) s += __ldcg(p + i);
+                s = warp_sum(s);
+                v = rsqrtf(s * is.inv_width + is.eps);
+            }
+            if (lane == 0) insc_tab[idx] = v;
+        }
+        __syncthreads();
+    }
+    unsigned long long best[NT][2];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) best[j][0] = best[j][1] = 0ull;
+    bool alive = true;
+    if (busy) {
+        if (smem_act) {
+            FkAct<FMT, GRP, NT, true> act;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) act.row[j] = act_s + min(8 * j + (lane >> 2), B - 1) * rowq + 2 * t;
+            alive = fk_gemv_run<LF, LG, HF, HG, FMT, GRP, NT, true>(G, insc_tab, act, wr, fp, gw, Wall, lane, ring, bar,
+                                                                   n_ops, ps, ccount, best);
+        } else {
+            FkAct<FMT, GRP, NT, false> act;
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+                act.row[j] = reinterpret_cast<const uint4*>(a.act + (size_t)min(8 * j + (lane >> 2), B - 1) * a.act_ld) +
+                             2 * t;
+            alive = fk_gemv_run<LF, LG, HF, HG, FMT, GRP, NT, false>(G, insc_tab, act, wr, fp, gw, Wall, lane, ring, bar,
+                                                                    n_ops, ps, ccount, best);
+        }
     }
     if (G.epi == EPI_ARGMAX && alive) argmax_publish<NT>(a, wr.m, best, Wall, lane);
     return alive;
@@ -589,7 +705,7 @@ __global__ void __launch_bounds__(fk_warps(NT) * 32, 1) frame_kernel(const Frame
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t bars[WARPS][kMaxSlots];
     __shared__ float insc_tab[kMaxB * 16];
-    __shared__ __align__(16) FkGemv cur;
+    __shared__ __align__(16) FkGemv cur[2];   // this GEMV op's and the next one's arguments
     __shared__ int s_ok;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -599,6 +715,7 @@ __global__ void __launch_bounds__(fk_warps(NT) * 32, 1) frame_kernel(const Frame
     const int n_ops = P->n_ops;
     uint8_t* ring = smem + (size_t)warp * fp.slots * fp.slot_bytes;
     uint64_t* bar = bars[warp];
+    uint4* act_s = reinterpret_cast<uint4*>(smem + (size_t)WARPS * fp.slots * fp.slot_bytes);
 
     // the weight stream starts at once: the first slots fill while the input op runs
     FkStream ps{};
@@ -612,45 +729,37 @@ __global__ void __launch_bounds__(fk_warps(NT) * 32, 1) frame_kernel(const Frame
     __syncwarp();
     int ccount = 0;   // chunks consumed by this warp
     unsigned nbar = 0;
+    int gsel = 0;     // the buffer of cur holding the next GEMV op's arguments
+    // a GEMV op's arguments are copied to shared memory before the barrier that precedes it
+    auto stage_args = [&](int oi) {
+        if (oi < n_ops && P->ops[oi].kind == FK_GEMV) {
+            const int n4 = (int)(sizeof(FkGemv) / 16);
+            const uint4* src = reinterpret_cast<const uint4*>(&P->gemv[P->ops[oi].idx]);
+            uint4* dst = reinterpret_cast<uint4*>(&cur[gsel]);
+            for (int i = threadIdx.x; i < n4; i += blockDim.x) dst[i] = src[i];
+        }
+    };
+    stage_args(0);
+    __syncthreads();
     bool ok = true;
     for (int oi = 0; oi < n_ops && ok; ++oi) {
         const FkOp op = P->ops[oi];
         if (op.kind == FK_GEMV) {
-            // the op's arguments in shared memory, the heads' token outputs from the launch
-            {
-                const int n4 = (int)(sizeof(FkGemv) / 16);
-                const uint4* src = reinterpret_cast<const uint4*>(&P->gemv[op.idx]);
-                uint4* dst = reinterpret_cast<uint4*>(&cur);
-                for (int i = threadIdx.x; i < n4; i += blockDim.x) dst[i] = src[i];
+            FkGemv& G = cur[gsel];
+            gsel ^= 1;
+            if (threadIdx.x == 0 && G.epi == EPI_ARGMAX) {   // the heads' token outputs are the launch's
+                G.a.tok[0] = fp.tok_t;
+                G.a.tok[1] = fp.tok_f;
             }
-            __syncthreads();
-            if (threadIdx.x == 0 && cur.epi == EPI_ARGMAX) {
-                cur.a.tok[0] = fp.tok_t;
-                cur.a.tok[1] = fp.tok_f;
-            }
-            if (blockIdx.x == 0 && cur.zero_buf)
-                for (int i = threadIdx.x; i < cur.zero_n; i += blockDim.x) cur.zero_buf[i] = 0.0f;
-            // input scales (per CTA): one warp per (row b, norm group q)
-            const InScale& is = cur.a.insc;
-            const int ng = is.parts ? is.n_groups : 1;
-            for (int idx = warp; idx < cur.a.B * ng; idx += WARPS) {
-                float v = 1.0f;
-                if (is.parts) {
-                    const int b = idx / ng, q = idx % ng;
-                    const float* p = is.parts + ((size_t)b * ng + q) * is.per_group;
-                    float s = 0.0f;
-                    for (int i = lane; i < is.per_group; i += 32) s += __ldcg(p + i);
-                    s = warp_sum(s);
-                    v = rsqrtf(s * is.inv_width + is.eps);
-                }
-                if (lane == 0) insc_tab[idx] = v;
-            }
-            __syncthreads();
+            if (blockIdx.x == 0 && G.zero_buf)
+                for (int i = threadIdx.x; i < G.zero_n; i += blockDim.x) G.zero_buf[i] = 0.0f;
             bool alive;
-            if (cur.head)
-                alive = fk_gemv<LF, LG, HF, HG, HF, HG, NT>(cur, insc_tab, fp, gw, Wall, lane, ring, bar, n_ops, ps, ccount);
+            if (G.head)
+                alive = fk_gemv<LF, LG, HF, HG, HF, HG, NT, WARPS>(G, insc_tab, act_s, kFkActBytes, fp, gw, Wall, warp,
+                                                                  lane, ring, bar, n_ops, ps, ccount);
             else
-                alive = fk_gemv<LF, LG, HF, HG, LF, LG, NT>(cur, insc_tab, fp, gw, Wall, lane, ring, bar, n_ops, ps, ccount);
+                alive = fk_gemv<LF, LG, HF, HG, LF, LG, NT, WARPS>(G, insc_tab, act_s, kFkActBytes, fp, gw, Wall, warp,
+                                                                  lane, ring, bar, n_ops, ps, ccount);
             if (!alive && lane == 0) atomicExch(fp.abort, 1);
         } else if (op.kind == FK_MAMBA) {
             fk_mamba(P->mamba[op.idx], gw, Wall, lane);
@@ -661,7 +770,10 @@ __global__ void __launch_bounds__(fk_warps(NT) * 32, 1) frame_kernel(const Frame
         } else {
             fk_input(P->input, fp, gw, Wall, lane);
         }
-        if (oi + 1 < n_ops) ok = fk_barrier(fp, ++nbar, &s_ok);
+        if (oi + 1 < n_ops) {
+            stage_args(oi + 1);
+            ok = fk_barrier(fp, ++nbar, &s_ok);
+        }
     }
     // after an abort, chunks issued but not consumed may still be in flight: wait for them
     // (bounded) before the CTA's shared memory is released.  In a completed frame none are.

@@ -5,10 +5,10 @@
 // A matrix in the device layout (layout.cuh) is a sequence of T = NU * KT blocks (unit u of 16R
 // rows, k-step kt); the warps of a launch split that sequence into equal contiguous ranges
 // (worker w of W owns blocks [w T / W, (w+1) T / W)).  A warp walks its range block by block:
-//   * the A fragments of a 16x64 tile are dequantized in registers (bf16 as stored; W8/W4/W3 by
-//     the fp16 exponent-field trick: OR a code into the mantissa of 1024.0 and subtract 1024 + z,
-//     exact) and multiplied on mma.sync m16n8k16 with fp32 accumulation; the fp32 group sums are
-//     scaled by the group's fp16 scale and by the input scale of the activation row;
+//   * the A fragments of a 16x64 tile are formed in registers (bf16 as stored; W8/W4/W3 the exact
+//     fp16 values q - z by the exponent-field trick: OR a code into the mantissa of 1024.0 and
+//     subtract 1024 + z) and multiplied on mma.sync m16n8k16 with fp32 accumulation; the fp32
+//     group sums are scaled by the group's fp16 scale and by the input scale of the activation row;
 //   * a unit whose k-steps all belong to this warp is finished here (fused epilogue); a unit cut
 //     between warps is finished by its last contributor (atomic counter), which adds the others'
 //     contributions: with an accumulator area through fp32 vector reductions (summation order
@@ -21,6 +21,11 @@
 namespace vc {
 
 static constexpr int kWarps = 16;   // upper bound of warps per CTA (sizes the partial-sum scratch)
+
+// the 16-bit type of the activations a weight format multiplies: bf16 (the values the step stores)
+// for bf16 weights, fp16 (the same values widened, exact in fp16's normal range) for the quantized
+// formats, whose dequantized codes are fp16
+__host__ __device__ constexpr bool act_f16_for(int fmt) { return fmt != 0; }
 static constexpr int kMaxB = 16;
 static constexpr int kMaxSlots = 8;  // ring slots per warp (upper bound)
 
@@ -72,13 +77,13 @@ __device__ __forceinline__ WarpRange warp_range(const GemvMat (&mat)[2], int nma
 }
 
 // ------------------------------------------------------------------------------------------
-// A-fragment extraction, one 16x64 tile per call: a[step][reg]
+// A fragments of the weight tiles
 // ------------------------------------------------------------------------------------------
-struct QConst {
+struct QConst {            // W4 / W3 dequantization constants of a slab (fp16 pairs)
     uint32_t zg, zh;       // (1024 + z) pairs, rows g and g+8
-    uint32_t f16g, f16h;   // -(64 + z)          (W4 high nibble)
-    uint32_t f8g, f8h;     // -(128 + z)         (W3 field 1, 4)
-    uint32_t f64g, f64h;   // -(16 + z)          (W3 field 2)
+    uint32_t f16h;         // -(64 + z), row g+8  (W4 high nibble)
+    uint32_t f8g, f8h;     // -(128 + z)          (W3 fields 1, 4)
+    uint32_t f64g, f64h;   // -(16 + z)           (W3 field 2)
 };
 
 __device__ __forceinline__ uint32_t h2bits(float v) {
@@ -88,74 +93,9 @@ __device__ __forceinline__ uint32_t h2bits(float v) {
 }
 
 template <int FMT>
-__device__ __forceinline__ void load_tile_frags(const uint8_t* tile, int lane, const QConst& qc, uint32_t (&a)[4][4]) {
-    const uint32_t M = 0x64006400u;
-    if constexpr (FMT == FMT_BF16) {
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            uint4 v = *reinterpret_cast<const uint4*>(tile + (s * 32 + lane) * 16);
-            a[s][0] = v.x; a[s][1] = v.y; a[s][2] = v.z; a[s][3] = v.w;
-        }
-    } else if constexpr (FMT == FMT_W8) {
-        const uint32_t K1152 = 0x64806480u;   // 1024 + 128 as an fp16 pair
-        const uint32_t M8 = 0x64646464u;      // prmt source of the 0x64 exponent byte
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            uint4 v = *reinterpret_cast<const uint4*>(tile + (c * 32 + lane) * 16);
-            uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                int s = 2 * c + h;
-                uint32_t A = w[2 * h], B = w[2 * h + 1];
-                a[s][0] = hsub2_u32(prmt(A, M8, 0x4240), K1152);
-                a[s][1] = hsub2_u32(prmt(B, M8, 0x4240), K1152);
-                a[s][2] = hsub2_u32(prmt(A, M8, 0x4341), K1152);
-                a[s][3] = hsub2_u32(prmt(B, M8, 0x4341), K1152);
-            }
-        }
-    } else if constexpr (FMT == FMT_W4) {
-        const uint32_t R16 = h2bits(1.0f / 16.0f);
-        uint4 v = *reinterpret_cast<const uint4*>(tile + lane * 16);
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            uint32_t x = w[s], y = w[s] >> 8;
-            a[s][0] = hsub2_u32(and_or(x, 0x000F000Fu, M), qc.zg);
-            a[s][1] = hfma2_u32(and_or(x, 0x00F000F0u, M), R16, qc.f16h);
-            a[s][2] = hsub2_u32(and_or(y, 0x000F000Fu, M), qc.zg);
-            a[s][3] = hfma2_u32(and_or(y, 0x00F000F0u, M), R16, qc.f16h);
-        }
-    } else {  // W3
-        const uint32_t R8 = h2bits(1.0f / 8.0f), R64 = h2bits(1.0f / 64.0f);
-        uint2 v01 = *reinterpret_cast<const uint2*>(tile + lane * 8);
-        uint32_t w[3] = {v01.x, v01.y, *reinterpret_cast<const uint32_t*>(tile + 256 + lane * 4)};
-#pragma unroll
-        for (int p = 0; p < 16; ++p) {
-            const int s = p / 4, reg = p % 4;
-            const bool hi = reg & 1;
-            const uint32_t z = hi ? qc.zh : qc.zg, f8 = hi ? qc.f8h : qc.f8g, f64 = hi ? qc.f64h : qc.f64g;
-            uint32_t r;
-            if (p < 15) {
-                const uint32_t x = w[p / 5];
-                const int i = p % 5;
-                if (i == 0) r = hsub2_u32(and_or(x, 0x00070007u, M), z);
-                else if (i == 1) r = hfma2_u32(and_or(x, 0x00380038u, M), R8, f8);
-                else if (i == 2) r = hfma2_u32(and_or(x, 0x01C001C0u, M), R64, f64);
-                else if (i == 3) r = hsub2_u32(and_or(x >> 9, 0x00070007u, M), z);
-                else r = hfma2_u32(and_or(x >> 9, 0x00380038u, M), R8, f8);
-            } else {
-                uint32_t c = ((w[0] >> 15) & 0x00010001u) | ((w[1] >> 14) & 0x00020002u) | ((w[2] >> 13) & 0x00040004u);
-                r = hsub2_u32(c | M, z);
-            }
-            a[s][reg] = r;
-        }
-    }
-}
-
-template <int FMT>
 __device__ __forceinline__ void mma_step(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    if constexpr (FMT == FMT_BF16) mma_bf16(d, a, b0, b1, d);
-    else mma_f16(d, a, b0, b1, d);
+    if constexpr (!act_f16_for(FMT)) mma_bf16(d, a, b0, b1);
+    else mma_f16(d, a, b0, b1);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -164,8 +104,9 @@ __device__ __forceinline__ void mma_step(float (&d)[4], const uint32_t (&a)[4], 
 //              64 st + 16 t + 15 of the k-step; zero for rows >= B)
 //   sc[j][e]:  input scale of batch column 8j + 2t + e for this k-step
 // ------------------------------------------------------------------------------------------
-// the raw 32-bit words of one lane's share of a 16x64 tile, and the A fragments of k16 step s
-// computed from them (the same values load_tile_frags gives)
+// The raw 32-bit words of one lane's share of a 16x64 tile, and the A fragments of k16 step s
+// computed from them: bf16 as stored; W8, W4 and W3 the exact fp16 values q - z by the
+// exponent-field trick (OR a code into the mantissa of 1024.0, subtract 1024 + z).
 template <int FMT>
 struct TileWords {
     static constexpr int n = FMT == FMT_BF16 ? 16 : FMT == FMT_W8 ? 8 : FMT == FMT_W4 ? 4 : 3;
@@ -211,6 +152,8 @@ __device__ __forceinline__ void step_frags(const TileWords<FMT>& tw, int s, cons
         a[2] = hsub2_u32(prmt(A, M8, 0x4341), K1152);
         a[3] = hsub2_u32(prmt(B, M8, 0x4341), K1152);
     } else if constexpr (FMT == FMT_W4) {
+        // row g: the low nibble, 1024 + q - (1024 + z); row g+8: the nibble above it, read as
+        // 1024 + 16 q, times 1/16 minus (64 + z).  Both exact in fp16.
         const uint32_t R16 = h2bits(1.0f / 16.0f);
         const uint32_t x = tw.w[s], y = tw.w[s] >> 8;
         a[0] = hsub2_u32(and_or(x, 0x000F000Fu, M), qc.zg);
@@ -278,7 +221,6 @@ __device__ __forceinline__ void consume_block_bv(const uint8_t* blk, const uint4
                 const uint32_t zl = (zb & 15u) | 0x6400u, zh = (zb >> 4) | 0x6400u;
                 qc[r].zg = zl | (zl << 16);
                 qc[r].zh = zh | (zh << 16);
-                qc[r].f16g = hsub2_u32(h2bits(960.0f), qc[r].zg);
                 qc[r].f16h = hsub2_u32(h2bits(960.0f), qc[r].zh);
                 qc[r].f8g = hsub2_u32(h2bits(896.0f), qc[r].zg);
                 qc[r].f8h = hsub2_u32(h2bits(896.0f), qc[r].zh);
@@ -318,6 +260,8 @@ __device__ __forceinline__ void consume_block_bv(const uint8_t* blk, const uint4
 }
 
 //   arow(b): byte address of activation row b's 64-column slice st = 0 of this k-step
+// Columns b >= B read row B-1 instead of zeros: their sums are computed and never stored (every
+// epilogue checks b < B), and the loads need no branch.
 template <int FMT, int GRP, int NT, typename ActRow>
 __device__ __forceinline__ void consume_block(const uint8_t* blk, ActRow arow, int B, int lane, const float (&sc)[NT][2],
                                               float (&acc)[layout_info(FMT, GRP).R][NT][4]) {
@@ -328,13 +272,10 @@ __device__ __forceinline__ void consume_block(const uint8_t* blk, ActRow arow, i
     for (int st = 0; st < SUB; ++st)
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-            const int b = 8 * j + g;
-            bv[st][j][0] = bv[st][j][1] = make_uint4(0, 0, 0, 0);
-            if (b < B) {
-                const uint8_t* p = arow(b) + (64 * st + 16 * t) * 2;
-                bv[st][j][0] = *reinterpret_cast<const uint4*>(p);
-                bv[st][j][1] = *reinterpret_cast<const uint4*>(p + 16);
-            }
+            const int b = min(8 * j + g, B - 1);
+            const uint8_t* p = arow(b) + (64 * st + 16 * t) * 2;
+            bv[st][j][0] = *reinterpret_cast<const uint4*>(p);
+            bv[st][j][1] = *reinterpret_cast<const uint4*>(p + 16);
         }
     consume_block_bv<FMT, GRP, NT>(blk, bv, lane, sc, acc);
 }

@@ -50,6 +50,9 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = lane & 3;
     const int B = args.B;
+    // the ring geometry in registers (read once from the parameter space)
+    const int rg_slots = rg.slots, rg_slot_bytes = rg.slot_bytes, rg_act_row = rg.act_row, rg_act_stride = rg.act_stride;
+    const bool rg_act_smem = rg.act_smem != 0;
 
     // ---- worker range -------------------------------------------------------------------
     const long long Wall = (long long)gridDim.x * WARPS;
@@ -60,7 +63,7 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
     const int nstages = (f1 - f0 + bps - 1) / bps;
     const int KT = M.KT;
 
-    uint8_t* ring = smem + (size_t)warp * rg.slots * rg.slot_bytes;
+    uint8_t* ring = smem + (size_t)warp * rg_slots * rg_slot_bytes;
     uint64_t* bar = bars[warp];
     const int act_rows = B;
 
@@ -69,26 +72,26 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
         const int fb = f0 + i * bps;
         const int nb = min(bps, f1 - fb);
         const uint32_t wbytes = nb * L.block_bytes;
-        const uint32_t abytes = rg.act_smem ? 0u : (uint32_t)(nb * act_rows * KS * 2);
+        const uint32_t abytes = rg_act_smem ? 0u : (uint32_t)(nb * act_rows * KS * 2);
         mbar_arrive_expect_tx(&bar[slot], wbytes + abytes);
-        bulk_g2s(ring + (size_t)slot * rg.slot_bytes, M.w + (size_t)fb * L.block_bytes, wbytes, &bar[slot]);
+        bulk_g2s(ring + (size_t)slot * rg_slot_bytes, M.w + (size_t)fb * L.block_bytes, wbytes, &bar[slot]);
     };
     int act_kt = f0 % KT;   // k-step of the next block whose activation slice is issued
     auto issue_act = [&](int i, int slot) {
         const int nb = min(bps, f1 - (f0 + i * bps));
-        uint8_t* abase = ring + (size_t)slot * rg.slot_bytes + bps * L.block_bytes;
+        uint8_t* abase = ring + (size_t)slot * rg_slot_bytes + bps * L.block_bytes;
         for (int j = 0; j < nb; ++j) {
             for (int b = 0; b < act_rows; ++b)
-                bulk_g2s(abase + (j * act_rows + b) * rg.act_row,
+                bulk_g2s(abase + (j * act_rows + b) * rg_act_row,
                          args.act + (size_t)b * args.act_ld + (size_t)act_kt * KS, KS * 2, &bar[slot]);
             if (++act_kt == KT) act_kt = 0;
         }
     };
 
     if (lane == 0) {
-        for (int s = 0; s < rg.slots; ++s) mbar_init(&bar[s], 1);
+        for (int s = 0; s < rg_slots; ++s) mbar_init(&bar[s], 1);
         fence_mbar_init();
-        for (int i = 0; i < nstages && i < rg.slots; ++i) issue_weights(i, i);
+        for (int i = 0; i < nstages && i < rg_slots; ++i) issue_weights(i, i);
     }
     __syncwarp();
 
@@ -108,19 +111,19 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
         }
         if (lane == 0) insc_tab[idx] = v;
     }
-    uint8_t* act_s = smem + (size_t)WARPS * rg.slots * rg.slot_bytes;
-    if (rg.act_smem) {
+    uint8_t* act_s = smem + (size_t)WARPS * rg_slots * rg_slot_bytes;
+    if (rg_act_smem) {
         const int row16 = args.act_ld / 8;   // 16-byte chunks per row
         for (int idx = threadIdx.x; idx < B * row16; idx += WARPS * 32) {
             const int b = idx / row16, c = idx % row16;
-            *reinterpret_cast<uint4*>(act_s + (size_t)b * rg.act_stride + c * 16) =
+            *reinterpret_cast<uint4*>(act_s + (size_t)b * rg_act_stride + c * 16) =
                 *reinterpret_cast<const uint4*>(args.act + (size_t)b * args.act_ld + (size_t)c * 8);
         }
     }
     __syncthreads();
 
-    if (lane == 0 && !rg.act_smem)
-        for (int i = 0; i < nstages && i < rg.slots; ++i) issue_act(i, i);
+    if (lane == 0 && !rg_act_smem)
+        for (int i = 0; i < nstages && i < rg_slots; ++i) issue_act(i, i);
 
     // ---- accumulation state ---------------------------------------------------------------
     float acc[R][NT][4];
@@ -146,11 +149,11 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
     int sc_next = kt;   // first k-step at which sc must be (re)loaded
     for (int i = 0; i < nstages; ++i) {
         if (!mbar_wait(&bar[slot], phase, args.status)) { alive = false; break; }
-        const uint8_t* base = ring + (size_t)slot * rg.slot_bytes;
+        const uint8_t* base = ring + (size_t)slot * rg_slot_bytes;
         const int nb = min(bps, f1 - (f0 + i * bps));
         for (int jb = 0; jb < nb; ++jb) {
             const uint8_t* blk = base + jb * L.block_bytes;
-            const uint8_t* arow0 = base + bps * L.block_bytes + (size_t)jb * act_rows * rg.act_row;
+            const uint8_t* arow0 = base + bps * L.block_bytes + (size_t)jb * act_rows * rg_act_row;
             // input scales of this k-step (norm group qg) for the lane's batch columns
             if (kt == sc_next) {
                 const int qg = ng > 1 ? (kt * KS) / args.insc.group_cols : 0;
@@ -163,11 +166,11 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
                         sc[j][e] = b < B ? insc_tab[b * ng + qg] : 0.0f;
                     }
             }
-            if (rg.act_smem) {
+            if (rg_act_smem) {
                 const uint8_t* abase = act_s + (size_t)kt * KS * 2;
-                consume_block<FMT, GRP, NT>(blk, [&](int b) { return abase + (size_t)b * rg.act_stride; }, B, lane, sc, acc);
+                consume_block<FMT, GRP, NT>(blk, [&](int b) { return abase + (size_t)b * rg_act_stride; }, B, lane, sc, acc);
             } else {
-                consume_block<FMT, GRP, NT>(blk, [&](int b) { return arow0 + b * rg.act_row; }, B, lane, sc, acc);
+                consume_block<FMT, GRP, NT>(blk, [&](int b) { return arow0 + b * rg_act_row; }, B, lane, sc, acc);
             }
             pending = true;
             if (++kt == KT) {   // the unit's last k-step: finish it (or hand over the partial)
@@ -180,12 +183,12 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
             }
         }
         __syncwarp();
-        if (lane == 0 && i + rg.slots < nstages) {
+        if (lane == 0 && i + rg_slots < nstages) {
             fence_proxy_async();
-            issue_weights(i + rg.slots, slot);
-            if (!rg.act_smem) issue_act(i + rg.slots, slot);
+            issue_weights(i + rg_slots, slot);
+            if (!rg_act_smem) issue_act(i + rg_slots, slot);
         }
-        if (++slot == rg.slots) { slot = 0; phase ^= 1u; }
+        if (++slot == rg_slots) { slot = 0; phase ^= 1u; }
     }
     if (alive && pending) unit_flush<FMT, GRP, NT, EPI>(args, wr, cur_u, acc, best, lane);
 

@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(256, 2) pf_ssd_out_mma_kernel(const float* __r
                 const uint16_t* pbj = B16 + (size_t)j * Cx + k0 + 2 * tq;
                 const uint32_t b0 = j < jn ? ldg32(pbj) : 0u, b1 = j < jn ? ldg32(pbj + 8) : 0u;
 #pragma unroll
-                for (int mt = 0; mt < 4; ++mt) mma_f16(acc[mt][nt], af[mt], b0, b1, acc[mt][nt]);
+                for (int mt = 0; mt < 4; ++mt) mma_f16(acc[mt][nt], af[mt], b0, b1);
             }
         }
 #pragma unroll
@@ -202,8 +202,8 @@ __global__ void __launch_bounds__(256, 2) pf_ssd_out_mma_kernel(const float* __r
                 if (q < qn) {
                     uint32_t xb[4];
                     ldsm_x4_trans(xb, Xs + (k0 + lk) * L.sx + (q0 + q) * 8 + lp);
-                    mma_f16(acc[q], af, xb[0], xb[1], acc[q]);
-                    if (q + 1 < qn) mma_f16(acc[q + 1], af, xb[2], xb[3], acc[q + 1]);
+                    mma_f16(acc[q], af, xb[0], xb[1]);
+                    if (q + 1 < qn) mma_f16(acc[q + 1], af, xb[2], xb[3]);
                 }
         }
         // C . S_in^T: C rows (bf16, staged once), S_in rows p (bf16) from L2
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(256, 2) pf_ssd_out_mma_kernel(const float* __r
             for (int q = 0; q < 8; ++q)
                 if (q < qn) {
                     const uint16_t* br = Sh + (size_t)((q0 + q) * 8 + gq) * N + k0 + 2 * tq;
-                    mma_bf16(acc2[q], af, ldg32(br), ldg32(br + 8), acc2[q]);
+                    mma_bf16(acc2[q], af, ldg32(br), ldg32(br + 8));
                 }
         }
         const float Dh_ = Dv[h];
@@ -395,9 +395,9 @@ __global__ void __launch_bounds__(256) pf_ssd_state_mma_kernel(const float* __re
                     ldsm_x4_trans(al, Xl + (k0 + ar) * L.sx + 16 * mt + ac);
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
-                        mma_f16(acc[mt][q], ah, bh[2 * q], bh[2 * q + 1], acc[mt][q]);
-                        mma_f16(acc[mt][q], ah, bl[2 * q], bl[2 * q + 1], acc[mt][q]);
-                        mma_f16(acc[mt][q], al, bh[2 * q], bh[2 * q + 1], acc[mt][q]);
+                        mma_f16(acc[mt][q], ah, bh[2 * q], bh[2 * q + 1]);
+                        mma_f16(acc[mt][q], ah, bl[2 * q], bl[2 * q + 1]);
+                        mma_f16(acc[mt][q], al, bh[2 * q], bh[2 * q + 1]);
                     }
                 }
             }
@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(128) pf_flash_kernel(const uint16_t* __restric
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 const uint16_t* br = Ks + (nt * 8 + gq) * SK + kk * 16 + 2 * tq;
-                mma_bf16(s[nt], qa[kk], lds32(br), lds32(br + 8), s[nt]);
+                mma_bf16(s[nt], qa[kk], lds32(br), lds32(br + 8));
             }
         // causal mask (keys beyond the row or beyond T) and the running max of each row
         const bool diag = kt == qt;
@@ -550,8 +550,8 @@ __global__ void __launch_bounds__(128) pf_flash_kernel(const uint16_t* __restric
             for (int d = 0; d < DH / 8; d += 2) {
                 uint32_t vb[4];
                 ldsm_x4_trans(vb, Vs + (kb * 16 + lk) * SK + d * 8 + ld8);
-                mma_bf16(o[d], pa[kb], vb[0], vb[1], o[d]);
-                mma_bf16(o[d + 1], pa[kb], vb[2], vb[3], o[d + 1]);
+                mma_bf16(o[d], pa[kb], vb[0], vb[1]);
+                mma_bf16(o[d + 1], pa[kb], vb[2], vb[3]);
             }
     }
 #pragma unroll

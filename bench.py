@@ -416,7 +416,9 @@ def main():
                     help="per-kernel path: launch each step's kernels directly instead of replaying a CUDA graph "
                          "(for profilers that cannot replay graph kernel nodes with programmatic dependencies)")
     ap.add_argument("--per-kernel", action="store_true",
-                    help="run each frame as one kernel per operation instead of one launch of the frame kernel")
+                    help="run each frame as one kernel per operation")
+    ap.add_argument("--frame", action="store_true",
+                    help="run each frame as one launch of the frame kernel")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     cfg = synth.CONFIGS[args.config]
@@ -455,6 +457,8 @@ def main():
         bb.set_option(vc.OPT_GRAPH, 0)
     if args.per_kernel:
         bb.set_option(vc.OPT_FRAME, 0)
+    if args.frame:
+        bb.set_option(vc.OPT_FRAME, 1)
     frame = bb.uses_frame_kernel(B)
     st = dm.new_state(B, cap)
     if cfg.random_state:
