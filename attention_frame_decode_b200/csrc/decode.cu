@@ -10,6 +10,8 @@
 //   applied inside the out_proj GEMV from the per-(head, half) sums of squares written here.
 // The fp32 state slice is prefetched with a bulk copy before griddepcontrol.wait (it was written
 // by the previous frame) and written back once.  (GQA decode attention: attn_decode.cu.)
+#include <algorithm>
+
 #include "common.cuh"
 #include "decode.cuh"
 
@@ -64,133 +66,181 @@ cudaError_t launch_input(const InputArgs& a, cudaStream_t s) {
 }
 
 // ------------------------------------------------------------------------------------------
-// Mamba-2 step
+// Mamba-2 step.  Work item = (session b, head h, half of the head's P channels); a persistent
+// grid walks the items, each CTA its own in order, with the fp32 state slice of the next item
+// bulk-copied into the second of two shared-memory buffers while the current one is updated, so
+// the state stream keeps going across items.  The first item's state copy and conv partial sums
+// (which depend only on the previous frames) are issued before griddepcontrol.wait.
 // ------------------------------------------------------------------------------------------
 static constexpr int kMambaThreads = 256;
+static constexpr int kMambaCtasPerSm = 4;
 
-__global__ void __launch_bounds__(kMambaThreads) mamba_step_kernel(const MambaStepArgs a) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ uint64_t bar;
+struct MambaTile {
+    float *S, *xs, *Bs, *Cs, *zs;   // [Ph][N], [Ph], [N], [N], [Ph]
+};
+
+__device__ __forceinline__ MambaTile mamba_tile(uint8_t* base, int Ph, int N) {
+    MambaTile t;
+    t.S = reinterpret_cast<float*>(base);
+    t.xs = t.S + Ph * N;
+    t.Bs = t.xs + Ph;
+    t.Cs = t.Bs + N;
+    t.zs = t.Cs + N;
+    return t;
+}
+
+__host__ __device__ constexpr size_t mamba_tile_bytes(int Ph, int N) {
+    return ((size_t)(Ph * N + 2 * Ph + 2 * N) * 4 + 127) / 128 * 128;
+}
+
+__global__ void __launch_bounds__(kMambaThreads, kMambaCtasPerSm) mamba_step_kernel(const MambaStepArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t bar[2];
     __shared__ float red[kMambaThreads / 32];
     pdl_trigger();
 
-    const int h2 = blockIdx.x, b = blockIdx.y;
-    const int h = h2 >> 1, half = h2 & 1;
-    const int Ph = a.P / 2, p0 = half * Ph;
-    const int slot = a.slots ? a.slots[b] : b;
+    const int Ph = a.P / 2;
+    const int n_items = a.B * 2 * a.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = (int)((long long)h * a.G / a.H);
-
-    float* S = reinterpret_cast<float*>(smem);                       // [Ph][N]
-    float* xs = S + Ph * a.N;                                         // [Ph]
-    float* Bs = xs + Ph;                                              // [N]
-    float* Cs = Bs + a.N;                                             // [N]
-
-    float* Sg = a.ssm + (((size_t)slot * a.H + h) * a.P + p0) * a.N;
+    const size_t tile_bytes = mamba_tile_bytes(Ph, a.N);
     const uint32_t sbytes = (uint32_t)(Ph * a.N * 4);
-    if (tid == 0) {
-        mbar_init(&bar, 1);
-        fence_mbar_init();
-        mbar_arrive_expect_tx(&bar, sbytes);
-        bulk_g2s(S, Sg, sbytes, &bar);
-    }
+    const int hpg = a.H / a.G;
 
-    // Before griddepcontrol.wait: everything that does not depend on this frame's in_proj output
-    // (the frame counter, the W-1 previous pre-conv rows in the ring, the conv weights): the
-    // partial conv sums of this CTA's x channels and its group's B, C channels.
-    const int t = a.ctx_len[slot];   // advanced only by the last kernel of a step
-    uint16_t* ring = a.conv + (size_t)slot * a.W * a.Cx;
-    const bool writes_bc = (h % (a.H / a.G) == 0) && half == 0;
-    auto channel = [&](int i, float*& dst) -> int {
-        if (i < Ph) { dst = xs + i; return h * a.P + p0 + i; }
-        if (i < Ph + a.N) { dst = Bs + (i - Ph); return a.E + g * a.N + (i - Ph); }
-        dst = Cs + (i - Ph - a.N);
+    // item i: (b, h2) with h2 = (h, half); its state slice and ring
+    auto item_state = [&](int i) {
+        const int b = i / (2 * a.H), h2 = i % (2 * a.H);
+        const int slot = a.slots ? a.slots[b] : b;
+        return a.ssm + (((size_t)slot * a.H + (h2 >> 1)) * a.P + (h2 & 1) * Ph) * a.N;
+    };
+    auto issue_state = [&](int i, int buf) {
+        mbar_arrive_expect_tx(&bar[buf], sbytes);
+        bulk_g2s(smem + (size_t)buf * tile_bytes, item_state(i), sbytes, &bar[buf]);
+    };
+    // the partial conv sums of an item's channels (its x half, its group's B and C) over the
+    // W-1 ring rows before this frame
+    auto channel = [&](const MambaTile& T, int h, int p0, int g, int i, float*& dst) -> int {
+        if (i < Ph) { dst = T.xs + i; return h * a.P + p0 + i; }
+        if (i < Ph + a.N) { dst = T.Bs + (i - Ph); return a.E + g * a.N + (i - Ph); }
+        dst = T.Cs + (i - Ph - a.N);
         return a.E + a.G * a.N + g * a.N + (i - Ph - a.N);
     };
-    for (int i = tid; i < Ph + 2 * a.N; i += kMambaThreads) {
-        float* dst;
-        const int c = channel(i, dst);
-        float acc = a.conv_b[c];
-        for (int k = 0; k < a.W - 1; ++k) {
-            const int rs = ((t - (a.W - 1) + k) % a.W + a.W) % a.W;
-            acc += a.conv_w[c * a.W + k] * bf16_bits_to_f(ring[(size_t)rs * a.Cx + c]);
+    auto conv_partial = [&](const MambaTile& T, int i) {
+        const int b = i / (2 * a.H), h2 = i % (2 * a.H);
+        const int h = h2 >> 1, p0 = (h2 & 1) * Ph, g = h / hpg;
+        const int slot = a.slots ? a.slots[b] : b;
+        const int t = a.ctx_len[slot];   // advanced only by the last kernel of a step
+        const uint16_t* ring = a.conv + (size_t)slot * a.W * a.Cx;
+        for (int k = tid; k < Ph + 2 * a.N; k += kMambaThreads) {
+            float* dst;
+            const int c = channel(T, h, p0, g, k, dst);
+            float acc = a.conv_b[c];
+            for (int q = 0; q < a.W - 1; ++q) {
+                const int rs = ((t - (a.W - 1) + q) % a.W + a.W) % a.W;
+                acc += a.conv_w[c * a.W + q] * bf16_bits_to_f(ring[(size_t)rs * a.Cx + c]);
+            }
+            *dst = acc;
         }
-        *dst = acc;
+    };
+
+    int first = blockIdx.x;
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
+        if (first < n_items) issue_state(first, 0);
+        if (first + (int)gridDim.x < n_items) issue_state(first + gridDim.x, 1);
     }
-    const float dt_bias = a.dt_bias[h], A = -expf(a.A_log[h]), Dh = a.D[h];
+    __syncthreads();
+    if (first < n_items) conv_partial(mamba_tile(smem, Ph, a.N), first);
 
     pdl_wait();
-    // one round trip for this frame's inputs: x/B/C pre-activations (kept raw for the ring),
-    // the gate z and dt_raw; the ring slot t mod W is written at the end
-    const bool okb = a.ok ? a.ok[b] != 0 : true;
-    const uint16_t* zx = a.zx + (size_t)b * a.zx_ld;
-    const uint16_t* xBC = zx + a.E;
-    uint16_t raw[2];
-    int chan[2];
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        const int i = tid + q * kMambaThreads;
-        chan[q] = -1;
-        if (i < Ph + 2 * a.N) {
-            float* dst;
-            chan[q] = channel(i, dst);
-            raw[q] = xBC[chan[q]];
-        }
-    }
-    float* zs = Cs + a.N;   // [Ph] silu(z)
-    for (int i = tid; i < Ph; i += kMambaThreads) zs[i] = silu_f(bf16_bits_to_f(zx[h * a.P + p0 + i]));
-    const float dt_raw = bf16_bits_to_f(zx[a.E + a.Cx + h]);
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        if (chan[q] < 0) continue;
-        float* dst;
-        channel(tid + q * kMambaThreads, dst);
-        *dst = silu_f(*dst + a.conv_w[chan[q] * a.W + a.W - 1] * bf16_bits_to_f(raw[q]));
-    }
-    __syncthreads();
 
-    const float dt = softplus_f(dt_raw + dt_bias);
-    const float decay = expf(A * dt);
-
-    if (!mbar_wait(&bar, 0, a.status)) return;
-
-    float ss = 0.0f;
-    for (int pr = warp; pr < Ph; pr += kMambaThreads / 32) {
-        const float xv = xs[pr];
-        const float dx = dt * xv;
-        float y = 0.0f;
-        float* Srow = S + pr * a.N;
-        float* Sgrow = Sg + (size_t)pr * a.N;
-        for (int n = lane; n < a.N; n += 32) {
-            const float sn = fmaf(decay, Srow[n], dx * Bs[n]);
-            if (okb) Sgrow[n] = sn;
-            y = fmaf(Cs[n], sn, y);
-        }
-        y = warp_sum(y);
-        if (lane == 0) {
-            const int c = h * a.P + p0 + pr;
-            y = fmaf(Dh, xv, y);
-            const float v = y * zs[pr];
-            ss += v * v;
-            const float an = v * a.gnorm[c];
-            a.act[(size_t)b * a.act_ld + c] = a.act_f16 ? act_bits<true>(an) : act_bits<false>(an);
-        }
-    }
-    if (lane == 0) red[warp] = ss;
-    // the ring slot of frame t (disjoint from the W-1 slots any CTA reads this frame)
-    if (okb) {
-        uint16_t* rw = ring + (size_t)(t % a.W) * a.Cx;
+    int k = 0;
+    for (int i = first; i < n_items; i += gridDim.x, ++k) {
+        const int buf = k & 1;
+        const MambaTile T = mamba_tile(smem + (size_t)buf * tile_bytes, Ph, a.N);
+        const int b = i / (2 * a.H), h2 = i % (2 * a.H);
+        const int h = h2 >> 1, half = h2 & 1, p0 = half * Ph, g = h / hpg;
+        const int slot = a.slots ? a.slots[b] : b;
+        const int t = a.ctx_len[slot];
+        uint16_t* ring = a.conv + (size_t)slot * a.W * a.Cx;
+        const bool writes_bc = (h % hpg == 0) && half == 0;
+        const bool okb = a.ok ? a.ok[b] != 0 : true;
+        if (k > 0) conv_partial(T, i);   // the first item's were computed before the wait
+        // this frame's inputs: x/B/C pre-activations (kept raw for the ring), the gate z, dt_raw
+        const uint16_t* zx = a.zx + (size_t)b * a.zx_ld;
+        const uint16_t* xBC = zx + a.E;
+        uint16_t raw[2];
+        int chan[2];
+        __syncthreads();   // this buffer's conv partial sums are written
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-            const int i = tid + q * kMambaThreads;
-            if (chan[q] >= 0 && (i < Ph || writes_bc)) rw[chan[q]] = raw[q];
+            const int ci = tid + q * kMambaThreads;
+            chan[q] = -1;
+            if (ci < Ph + 2 * a.N) {
+                float* dst;
+                chan[q] = channel(T, h, p0, g, ci, dst);
+                raw[q] = xBC[chan[q]];
+                *dst = silu_f(*dst + a.conv_w[chan[q] * a.W + a.W - 1] * bf16_bits_to_f(raw[q]));
+            }
         }
-    }
-    __syncthreads();
-    if (tid == 0) {
-        float tot = 0.0f;
-        for (int w = 0; w < kMambaThreads / 32; ++w) tot += red[w];
-        a.parts[(size_t)b * 2 * a.H + h2] = tot;
+        for (int ci = tid; ci < Ph; ci += kMambaThreads) T.zs[ci] = silu_f(bf16_bits_to_f(zx[h * a.P + p0 + ci]));
+        const float dt = softplus_f(bf16_bits_to_f(zx[a.E + a.Cx + h]) + a.dt_bias[h]);
+        const float decay = expf(-expf(a.A_log[h]) * dt);
+        const float Dh = a.D[h];
+        __syncthreads();
+
+        float* Sg = item_state(i);
+        // every thread waits for the state copy; if it never arrives the CTA leaves together, after
+        // a bounded wait for the other buffer's copy (no copy may land in a CTA that has exited)
+        if (!__syncthreads_and(mbar_wait(&bar[buf], (uint32_t)(k >> 1) & 1u, a.status))) {
+            if (tid == 0 && i + (int)gridDim.x < n_items) mbar_wait(&bar[buf ^ 1], (uint32_t)((k + 1) >> 1) & 1u, nullptr);
+            return;
+        }
+        float ss = 0.0f;
+        for (int pr = warp; pr < Ph; pr += kMambaThreads / 32) {
+            const float xv = T.xs[pr];
+            const float dx = dt * xv;
+            float y = 0.0f;
+            const float* Srow = T.S + pr * a.N;
+            float* Sgrow = Sg + (size_t)pr * a.N;
+            for (int n = lane; n < a.N; n += 32) {
+                const float sn = fmaf(decay, Srow[n], dx * T.Bs[n]);
+                if (okb) Sgrow[n] = sn;
+                y = fmaf(T.Cs[n], sn, y);
+            }
+            y = warp_sum(y);
+            if (lane == 0) {
+                const int c = h * a.P + p0 + pr;
+                y = fmaf(Dh, xv, y);
+                const float v = y * T.zs[pr];
+                ss += v * v;
+                const float an = v * a.gnorm[c];
+                a.act[(size_t)b * a.act_ld + c] = a.act_f16 ? act_bits<true>(an) : act_bits<false>(an);
+            }
+        }
+        if (lane == 0) red[warp] = ss;
+        // the ring slot of frame t (disjoint from the W-1 slots any CTA reads this frame)
+        if (okb) {
+            uint16_t* rw = ring + (size_t)(t % a.W) * a.Cx;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int ci = tid + q * kMambaThreads;
+                if (chan[q] >= 0 && (ci < Ph || writes_bc)) rw[chan[q]] = raw[q];
+            }
+        }
+        __syncthreads();   // the buffer is read; red is complete
+        if (tid == 0) {
+            float tot = 0.0f;
+            for (int w = 0; w < kMambaThreads / 32; ++w) tot += red[w];
+            a.parts[(size_t)b * 2 * a.H + h2] = tot;
+            // the buffer's next item: the one after next of this CTA
+            const int nx = i + 2 * (int)gridDim.x;
+            if (nx < n_items) {
+                fence_proxy_async();
+                issue_state(nx, buf);
+            }
+        }
     }
 }
 
@@ -199,11 +249,16 @@ bool mamba_step_supported(int P, int N) { return P > 0 && N > 0 && P / 2 + 2 * N
 cudaError_t launch_mamba_step(const MambaStepArgs& a, int pdl, cudaStream_t s) {
     const int Ph = a.P / 2;
     if (Ph + 2 * a.N > 2 * kMambaThreads) return cudaErrorInvalidValue;
-    const size_t smem = (size_t)(Ph * a.N + 2 * Ph + 2 * a.N) * sizeof(float);
+    const size_t smem = 2 * mamba_tile_bytes(Ph, a.N);
     cudaError_t e = cudaFuncSetAttribute(mamba_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int n_items = a.B * 2 * a.H;
+    const int grid = std::min(n_items, sms * kMambaCtasPerSm);
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(2 * a.H, a.B);
+    cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kMambaThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
