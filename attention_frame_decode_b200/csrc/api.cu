@@ -852,6 +852,7 @@ extern "C" vc_status vc_debug_mamba_prefill(const vc_config* cfg, const vc_layer
     carve_mixer(m, (uint8_t*)scratch);
     m.ssm = ssm; m.ring = (uint16_t*)conv; m.act = (uint16_t*)act; m.act_ld = D.E;
     cudaStream_t s = (cudaStream_t)stream;
+    CK(cudaMemsetAsync(m.status, 0, 4, s));
     CK(prefill_mixer(m, s));
     CK(cudaMemcpyAsync(y, m.y, (size_t)T * D.E * 4, cudaMemcpyDeviceToDevice, s));
     return VC_OK;

@@ -374,7 +374,7 @@ __global__ void pf_finish_kernel(int32_t* ctx_len, int slot, int T) { ctx_len[sl
 size_t prefill_mixer_scratch_bytes(int T, int E, int Cx, int H, int P, int N) {
     const size_t nch = (size_t)(T + kChunk - 1) / kChunk;
     return al((size_t)T * Cx * 4) + 2 * al((size_t)T * H * 4) + al((size_t)T * E * 4) + al(nch * H * P * N * 4) +
-           al(nch * H * P * N * 2) + al((size_t)T * Cx * 2);
+           al(nch * H * P * N * 2) + al((size_t)T * Cx * 2) + al(4);
 }
 
 void carve_mixer(PfMixer& m, uint8_t* base) {
@@ -392,6 +392,7 @@ void carve_mixer(PfMixer& m, uint8_t* base) {
     m.schunk = take(nch * m.H * m.P * m.N * 4);
     m.sin16 = (uint16_t*)take(nch * m.H * m.P * m.N * 2);
     m.xc16 = (uint16_t*)take((size_t)m.T * m.Cx * 2);
+    m.status = (int*)take(4);
 }
 
 cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
@@ -417,7 +418,11 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
     const dim3 sg(nch, H);
     const bool st_mma = N % 16 == 0 && N <= 128 && (P == 80 || P == 32);
     const StateLayout STL = state_layout(N, P);
-    if (st_mma) {
+    if (m.status && ssd_state_tc_supported(N, P, E, Cx)) {
+        if ((e = launch_ssd_state_tc(m.xc, m.dt, Lw.A_log, T, H, P, N, m.G, E, Cx, m.lam, m.schunk, m.status, s)) !=
+            cudaSuccess)
+            return e;
+    } else if (st_mma) {
         auto kst = P == 80 ? pf_ssd_state_mma_kernel<5> : pf_ssd_state_mma_kernel<2>;
         if ((e = cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STL.total)) != cudaSuccess)
             return e;
@@ -433,8 +438,14 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
                                                               m.schunk);
     const long long n = (long long)H * P * N;
     pf_ssd_scan_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(m.schunk, m.lam, T, H, P, N, m.sin16, m.ssm);
-    pf_ssd_out_mma_kernel<<<dim3(nch, m.G, kChunk / kSsdTi), 256, SL.total, s>>>(m.xc, m.xc16, m.dt, m.lam, m.sin16, Lw.D, T, H,
-                                                                                 P, N, m.G, E, Cx, m.y);
+    if (m.status && ssd_out_tc_supported(N, P, E, Cx)) {
+        if ((e = launch_ssd_out_tc(m.xc16, m.sin16, m.dt, m.lam, Lw.D, m.y, T, H, P, N, m.G, E, Cx, m.status, s)) !=
+            cudaSuccess)
+            return e;
+    } else {
+        pf_ssd_out_mma_kernel<<<dim3(nch, m.G, kChunk / kSsdTi), 256, SL.total, s>>>(m.xc, m.xc16, m.dt, m.lam, m.sin16,
+                                                                                     Lw.D, T, H, P, N, m.G, E, Cx, m.y);
+    }
     pf_gated_norm_kernel<<<T, 32 * m.NG, 0, s>>>(m.y, m.zx, zxw, Lw.gnorm, E, m.NG, m.eps, m.act, m.act_ld,
                                                        m.f16);
     return cudaGetLastError();
@@ -528,6 +539,7 @@ cudaError_t run_prefill(const PrefillCtx& c, const uint16_t* x, int T, int slot,
             m.ssm = c.ssm + ((size_t)mi * c.n_slots + slot) * H * P * N;
             m.ring = c.conv + ((size_t)mi * c.n_slots + slot) * W * Cx;
             m.act = b.act_big; m.act_ld = b.ld_big;
+            m.status = c.status;
             // the GEMM's GE_ROWSCALE outputs are the bf16 in_proj values (the decode path's zx)
             if ((e = gemm(GE_ROWSCALE, b.act_d, b.ld_d, T, Lw.in_proj, b.inv, b.zx, zxw, nullptr, 0))) return e;
             m.zx = b.zx;

@@ -39,10 +39,23 @@ struct PfMixer {
     uint16_t* ring;                                  // [W][Cx]
     uint16_t* act;                                   // [T][act_ld]
     int act_ld;
+    int* status;                                     // device status word (bounded waits of the tcgen05 kernels)
 };
 size_t prefill_mixer_scratch_bytes(int T, int E, int Cx, int H, int P, int N);
 void carve_mixer(PfMixer& m, uint8_t* base);
 cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s);
+
+// chunk outputs of the chunked SSD on tcgen05 (ssd_tc.cu); shapes: N in {64, 128}, P a multiple of
+// 16 up to 128
+bool ssd_out_tc_supported(int N, int P, int E, int Cx);
+// chunk states (and the within-chunk cumulative log decay) on tcgen05; shapes: N = 128, P a
+// multiple of 16
+bool ssd_state_tc_supported(int N, int P, int E, int Cx);
+cudaError_t launch_ssd_state_tc(const float* xc, const float* dt, const float* A_log, int T, int H, int P, int N, int G,
+                                int E, int Cx, float* lam, float* schunk, int* status, cudaStream_t s);
+cudaError_t launch_ssd_out_tc(const uint16_t* xc16, const uint16_t* sin16, const float* dt, const float* lam,
+                              const float* Dv, float* y, int T, int H, int P, int N, int G, int E, int Cx, int* status,
+                              cudaStream_t s);
 
 size_t prefill_workspace_bytes(int d, int L, int E, int Cx, int H, int P, int N, int G, int Hq, int Hk, int Dh, int F,
                                int cap);
