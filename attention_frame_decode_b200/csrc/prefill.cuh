@@ -49,7 +49,7 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s);
 // 16 up to 128
 bool ssd_out_tc_supported(int N, int P, int E, int Cx);
 // chunk states (and the within-chunk cumulative log decay) on tcgen05; shapes: N = 128, P a
-// multiple of 16
+// multiple of 16 up to 128
 bool ssd_state_tc_supported(int N, int P, int E, int Cx);
 cudaError_t launch_ssd_state_tc(const float* xc, const float* dt, const float* A_log, int T, int H, int P, int N, int G,
                                 int E, int Cx, float* lam, float* schunk, int* status, cudaStream_t s);

@@ -20,7 +20,7 @@
 //     element, and write M_h as fp16 into shared memory in the K-major swizzled layout; one
 //     thread then issues M_h X_h (fp16) into columns [256, 256 + P) and C S_in^T (bf16) into
 //     [384, 384 + P); the threads read both back, add exp(Lam_i) x the second and D x_i, store y;
-//     the next head's x and S_in are copied while its M_h is formed.
+//     x and S_in are double-buffered: the next head's copies run under this head's work.
 // The C rows are converted to bf16 in place once G is done (the entering-state product keeps
 // bf16 operands: the state's range).  Every wait is bounded; a timeout sets the status word,
 // the CTA waits (bounded) for its copies in flight and frees its TMEM.
@@ -35,11 +35,12 @@ static constexpr int kRows = 128;       // frames of one CTA's output tile (TMEM
 static constexpr int kOutThreads = 256;
 static constexpr uint32_t kTmemCols = 512;
 static constexpr uint32_t kColY1 = 256, kColY2 = 384;
+static_assert(kQ == kOutThreads, "one thread per frame of the chunk stages the decay of a head");
 
 // shared-memory plan of the output kernel (byte offsets from a 1024-aligned base)
 struct SsdOutPlan {
     int NA, PA;                                 // 64-wide atoms of N, 16-wide blocks of P
-    uint32_t off_c, off_bm, off_x, off_s, total;
+    uint32_t off_c, off_bm, off_x0, off_s0, off_x1, off_s1, total;
 };
 
 __host__ __device__ inline SsdOutPlan ssd_out_plan(int N, int P) {
@@ -48,10 +49,16 @@ __host__ __device__ inline SsdOutPlan ssd_out_plan(int N, int P) {
     L.PA = P / 16;
     L.off_c = 0;                                               // C rows: NA atoms x 128 rows x 128 B
     const uint32_t bm = (uint32_t)L.NA * 32768u > 65536u ? (uint32_t)L.NA * 32768u : 65536u;
-    L.off_bm = L.off_c + (uint32_t)L.NA * 16384u;              // B rows (NA x 256 x 128 B), later M_h (4 x 128 x 128 B)
-    L.off_x = L.off_bm + bm;                                   // x_h: PA blocks x 256 rows x 32 B
-    L.off_s = L.off_x + (uint32_t)L.PA * 8192u;                // S_in,h: NA atoms x P rows x 128 B
-    L.total = L.off_s + (uint32_t)L.NA * (uint32_t)P * 128u;
+    L.off_bm = L.off_c + (uint32_t)L.NA * 16384u;              // B rows (NA x 256 x 128 B), then M_h (4 x 128 x 128 B)
+                                                               // and the y staging tile (PA x 128 rows x 64 B)
+    // two buffers (heads alternate) of x_h (PA blocks x 256 rows x 32 B) and S_in,h (NA atoms x P
+    // rows x 128 B)
+    const uint32_t xb = (uint32_t)L.PA * 8192u, sb = (uint32_t)L.NA * (uint32_t)P * 128u;
+    L.off_x0 = L.off_bm + bm;
+    L.off_s0 = L.off_x0 + xb;
+    L.off_x1 = L.off_s0 + sb;
+    L.off_s1 = L.off_x1 + xb;
+    L.total = L.off_s1 + sb;
     return L;
 }
 
@@ -61,10 +68,17 @@ VC_DEV float ex2_approx(float x) {
     return y;
 }
 
+VC_DEV float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// fp16 pair (lo in the low half), saturated to the finite range
 VC_DEV uint32_t pack_f16x2_sat(float lo, float hi) {
-    lo = fminf(fmaxf(lo, -65504.0f), 65504.0f);
-    hi = fminf(fmaxf(hi, -65504.0f), 65504.0f);
-    return h2_as_u32(__floats2half2_rn(lo, hi));
+    uint32_t d;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
 }
 
 VC_DEV uint32_t f16x2_to_bf16x2(uint32_t v) {
@@ -73,24 +87,37 @@ VC_DEV uint32_t f16x2_to_bf16x2(uint32_t v) {
     return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+VC_DEV void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x),
+                 "r"(y), "r"(smem_u32(src))
+                 : "memory");
+}
+VC_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+VC_DEV void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+VC_DEV void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 struct SsdOutArgs {
     const float* dt;    // [T][H]
     const float* lam;   // [T][H] within-chunk cumulative A dt
     const float* Dv;    // [H]
-    float* y;           // [T][E]
     int T, H, P, N, G, E;
     int* status;
 };
 
+// warp 4 (whose rows see the fewest unmasked columns) issues the copies, one per lane (the TMA
+// engine works on several boxes at once), and its lane 0 the MMAs
+static constexpr int kIssuerWarp = 4;
+
 __global__ void __launch_bounds__(kOutThreads, 1)
-    pf_ssd_out_tc_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
-                         const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mS,
+    pf_ssd_out_tc_kernel(const __grid_constant__ CUtensorMap mBC, const __grid_constant__ CUtensorMap mX,
+                         const __grid_constant__ CUtensorMap mS, const __grid_constant__ CUtensorMap mY,
                          const SsdOutArgs a) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_cb, bar_g, bar_x, bar_y;
+    __shared__ uint64_t bar_cb, bar_g, bar_x[2], bar_y;
     __shared__ uint32_t tmem_base;
-    __shared__ float lam2[kQ], dts[kQ];
+    __shared__ __align__(16) float lam2[kQ];   // log2 of the cumulative decay, per frame
+    __shared__ __align__(16) float qv[kQ];     // lam2_j - log2(dt_j): 2^(lam2_i - qv_j) = decay x dt_j
 
     const int H = a.H, P = a.P, N = a.N, G = a.G;
     const int nch = (a.T + kQ - 1) / kQ;
@@ -105,15 +132,15 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     const SsdOutPlan L = ssd_out_plan(N, P);
     uint8_t* sC = sm + L.off_c;
     uint8_t* sBM = sm + L.off_bm;
-    uint8_t* sX = sm + L.off_x;
-    uint8_t* sS = sm + L.off_s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int hpg = H / G, nkN = N / 16;
+    const bool iwarp = warp == kIssuerWarp, issuer = iwarp && lane == 0;
 
     if (tid == 0) {
         mbar_init(&bar_cb, 1);
         mbar_init(&bar_g, 1);
-        mbar_init(&bar_x, 1);
+        mbar_init(&bar_x[0], 1);
+        mbar_init(&bar_x[1], 1);
         mbar_init(&bar_y, 1);
         fence_mbar_init();
     }
@@ -123,23 +150,44 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     tc_fence_after();
     const uint32_t tmem = tmem_base;
 
-    bool cb_pending = false, x_pending = false;   // copies in flight (thread 0)
-    uint32_t x_phase = 0;
-    auto issue_xs = [&](int h, uint32_t phase) {
-        mbar_arrive_expect_tx(&bar_x, (uint32_t)L.PA * 8192u + (uint32_t)L.NA * (uint32_t)P * 128u);
-        for (int q = 0; q < L.PA; ++q) tma_load_2d(sX + q * 8192, &mX, h * P + 16 * q, t0, &bar_x);
-        for (int q = 0; q < L.NA; ++q) tma_load_2d(sS + q * P * 128, &mS, 64 * q, (c * H + h) * P, &bar_x);
-        x_pending = true;
-        x_phase = phase;
+    // copies of head hh's x and S_in go to buffer hh & 1 (completion phase (hh >> 1) & 1); the
+    // issuer warp calls this together: lane 0 registers the bytes, then each lane issues one box
+    const int nrh = jn / kRows;   // 128-row halves of the frames j < jn
+    bool cb_pending = false;
+    uint32_t x_pend = 0u, x_ph = 0u;   // copies in flight per buffer (bit b) and their phases
+    auto issue_xs = [&](int hh) {
+        const int b = hh & 1, h = g * hpg + hh;
+        uint64_t* bar = &bar_x[b];
+        uint8_t* sX = sm + (b ? L.off_x1 : L.off_x0);
+        uint8_t* sS = sm + (b ? L.off_s1 : L.off_s0);
+        if (lane == 0)
+            mbar_arrive_expect_tx(bar, (uint32_t)L.PA * (uint32_t)jn * 32u + (uint32_t)L.NA * (uint32_t)P * 128u);
+        __syncwarp();
+        const int nx = L.PA * nrh;
+        if (lane < nx) {
+            const int q = lane / nrh, r0 = (lane - q * nrh) * kRows;
+            tma_load_2d(sX + q * 8192 + r0 * 32, &mX, h * P + 16 * q, t0 + r0, bar);
+        } else if (lane < nx + L.NA) {
+            const int q = lane - nx;
+            tma_load_2d(sS + q * P * 128, &mS, 64 * q, (c * H + h) * P, bar);
+        }
+        x_pend |= 1u << b;
+        x_ph = (x_ph & ~(1u << b)) | ((uint32_t)((hh >> 1) & 1) << b);
     };
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bar_cb, (uint32_t)L.NA * (16384u + 32768u));
-        for (int q = 0; q < L.NA; ++q) {
-            tma_load_2d(sC + q * 16384, &mC, a.E + (G + g) * N + 64 * q, t0 + i0, &bar_cb);
-            tma_load_2d(sBM + q * 32768, &mB, a.E + g * N + 64 * q, t0, &bar_cb);
+    if (iwarp) {
+        // C rows of the tile; B rows of the frames j < jn (128-row boxes)
+        if (lane == 0) mbar_arrive_expect_tx(&bar_cb, (uint32_t)L.NA * (16384u + (uint32_t)jn * 128u));
+        __syncwarp();
+        if (lane < L.NA) {
+            tma_load_2d(sC + lane * 16384, &mBC, a.E + (G + g) * N + 64 * lane, t0 + i0, &bar_cb);
+        } else if (lane < L.NA + L.NA * nrh) {
+            const int q = (lane - L.NA) / nrh, r0 = (lane - L.NA - q * nrh) * kRows;
+            tma_load_2d(sBM + q * 32768 + r0 * 128, &mBC, a.E + g * N + 64 * q, t0 + r0, &bar_cb);
         }
         cb_pending = true;
-        issue_xs(g * hpg, 0);
+        issue_xs(0);
+    }
+    if (issuer) {
         if (mbar_wait(&bar_cb, 0, a.status)) {
             cb_pending = false;
             tc_fence_after();
@@ -171,52 +219,82 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     const int i = i0 + r;                // frame within the chunk
     const int ilim = i < len ? i : -1;   // columns j <= ilim are unmasked
     const int jh = jn / 2, jbeg = warp < 4 ? 0 : jh;
-    const int wmax = i0 + lb + 31;       // the warp's last row
+    const int wmin = i0 + lb, wmax = wmin + 31;   // the warp's rows
+    const bool wfull = wmax < len;                 // every row of the warp is a frame of the chunk
     const int qh = (L.PA + 1) / 2;
     const int qa = warp < 4 ? 0 : qh, qb = warp < 4 ? qh : L.PA;
     const uint32_t trow = tmem + ((uint32_t)lb << 16);
     constexpr float kLog2e = 1.4426950408889634f;
+    // Lam and dt of frame tid for the next head, loaded one head ahead (kQ == kOutThreads)
+    const bool fr = tid < len;
+    float nl = fr ? a.lam[(size_t)(t0 + tid) * H + g * hpg] : 0.0f;
+    float nd = fr ? a.dt[(size_t)(t0 + tid) * H + g * hpg] : 0.0f;
 
     for (int hh = 0; hh < hpg && ok; ++hh) {
-        const int h = g * hpg + hh;
-        for (int j = tid; j < kQ; j += kOutThreads) {
-            lam2[j] = j < len ? a.lam[(size_t)(t0 + j) * H + h] * kLog2e : 0.0f;
-            dts[j] = j < len ? a.dt[(size_t)(t0 + j) * H + h] : 0.0f;
+        const int h = g * hpg + hh, b = hh & 1;
+        uint8_t* sX = sm + (b ? L.off_x1 : L.off_x0);
+        uint8_t* sS = sm + (b ? L.off_s1 : L.off_s0);
+        {
+            const float l2 = nl * kLog2e;
+            lam2[tid] = l2;
+            qv[tid] = nd > 0.0f ? l2 - lg2_approx(nd) : INFINITY;
+            if (hh + 1 < hpg && fr) {
+                nl = a.lam[(size_t)(t0 + tid) * H + h + 1];
+                nd = a.dt[(size_t)(t0 + tid) * H + h + 1];
+            }
         }
+        const float Dh = a.Dv[h];
+        // the previous head's y store has read the staging tile (the M_h buffer)
+        if (iwarp && hh > 0 && lane < L.PA) bulk_wait_read0();
         __syncthreads();
-        // M_h[i][j] = G[i][j] 2^(lam2_i - lam2_j) dt_j for j <= i, fp16, K-major 128-byte swizzle
+        // the next head's copies into the other buffer (its last reader, head hh - 1, is done)
+        if (iwarp && hh + 1 < hpg) issue_xs(hh + 1);
+        // M_h[i][j] = G[i][j] 2^(lam2_i - qv_j) for j <= i, fp16, K-major 128-byte swizzle
         {
             const float li = lam2[min(i, kQ - 1)];
-            for (int j0 = jbeg; j0 < jbeg + jh; j0 += 32) {
-                uint32_t pk[16];
+            for (int j0 = jbeg; j0 < jbeg + jh; j0 += 64) {
+                uint32_t pk[32];
                 if (j0 > wmax) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    for (int e = 0; e < 32; ++e) pk[e] = 0u;
                 } else {
-                    float gv[32];
-                    tc_ld32(trow + (uint32_t)j0, gv);
+                    float gv[64];
+                    tc_ld64(trow + (uint32_t)j0, gv);
+                    if (wfull && j0 + 63 <= wmin) {   // below the diagonal for every row of the warp
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int j = j0 + e;
-                        const float v0 = j <= ilim ? gv[e] * ex2_approx(li - lam2[j]) * dts[j] : 0.0f;
-                        const float v1 = j + 1 <= ilim ? gv[e + 1] * ex2_approx(li - lam2[j + 1]) * dts[j + 1] : 0.0f;
-                        pk[e >> 1] = pack_f16x2_sat(v0, v1);
+                        for (int e = 0; e < 64; e += 4) {
+                            const float4 q4 = *reinterpret_cast<const float4*>(qv + j0 + e);
+                            pk[e >> 1] = pack_f16x2_sat(gv[e] * ex2_approx(li - q4.x), gv[e + 1] * ex2_approx(li - q4.y));
+                            pk[(e >> 1) + 1] =
+                                pack_f16x2_sat(gv[e + 2] * ex2_approx(li - q4.z), gv[e + 3] * ex2_approx(li - q4.w));
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 64; e += 4) {
+                            const int j = j0 + e;
+                            const float4 q4 = *reinterpret_cast<const float4*>(qv + j);
+                            const float v0 = j <= ilim ? gv[e] * ex2_approx(li - q4.x) : 0.0f;
+                            const float v1 = j + 1 <= ilim ? gv[e + 1] * ex2_approx(li - q4.y) : 0.0f;
+                            const float v2 = j + 2 <= ilim ? gv[e + 2] * ex2_approx(li - q4.z) : 0.0f;
+                            const float v3 = j + 3 <= ilim ? gv[e + 3] * ex2_approx(li - q4.w) : 0.0f;
+                            pk[e >> 1] = pack_f16x2_sat(v0, v1);
+                            pk[(e >> 1) + 1] = pack_f16x2_sat(v2, v3);
+                        }
                     }
                 }
                 uint8_t* rowp = sBM + (j0 >> 6) * 16384 + r * 128;
-                const int c0 = (j0 & 63) >> 3;
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4*>(rowp + (((c0 + q) ^ (r & 7)) << 4)) =
+                for (int q = 0; q < 8; ++q)
+                    *reinterpret_cast<uint4*>(rowp + ((q ^ (r & 7)) << 4)) =
                         make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
             }
         }
         fence_proxy_async();   // the generic-proxy writes of M_h (and C) -> the tensor core's reads
         tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
-            if (mbar_wait(&bar_x, x_phase, a.status)) {
-                x_pending = false;
+        if (issuer) {
+            if (mbar_wait(&bar_x[b], (uint32_t)((hh >> 1) & 1), a.status)) {
+                x_pend &= ~(1u << b);
                 tc_fence_after();
                 // Y1 = M_h X_h: fp16, x MN-major (16-wide blocks 8 KB apart, 8-frame groups 256 B apart)
                 for (int k = 0; k < jn / 16; ++k)
@@ -234,46 +312,47 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         ok = __syncthreads_and(mbar_wait(&bar_y, (uint32_t)(hh & 1), a.status));
         tc_fence_after();
         if (!ok) break;
-        // y_i = Y1 + exp(Lam_i) Y2 + D x_i; x_i from the staged fp16 tile (32-byte swizzle: the two
-        // 16-byte halves of row j swap when bit 2 of j is set)
+        // y_i = Y1 + exp(Lam_i) Y2 + D x_i into the staging tile (the M_h buffer is free): block q of
+        // 16 columns is 128 rows x 64 B with the 64-byte swizzle (16-byte chunk c of row r at
+        // c ^ ((r >> 1) & 3)).  x_i comes from the staged fp16 tile (32-byte swizzle: the two
+        // 16-byte halves of row j swap when bit 2 of j is set).
         {
             const float el = ex2_approx(lam2[min(i, kQ - 1)]);
-            const float Dh = a.Dv[h];
-            float* yrow = a.y + (size_t)(t0 + min(i, len - 1)) * a.E + (size_t)h * P;
             const uint32_t sw = ((uint32_t)i >> 2) & 1u;
             for (int q = qa; q < qb; ++q) {
                 float y1[16], y2[16];
-                tc_ld16(trow + kColY1 + 16 * q, y1);
-                tc_ld16(trow + kColY2 + 16 * q, y2);
+                tc_ld16x2(trow + kColY1 + 16 * q, trow + kColY2 + 16 * q, y1, y2);
                 const uint8_t* xr = sX + q * 8192 + i * 32;
                 const uint4 xa = *reinterpret_cast<const uint4*>(xr + (sw << 4));
                 const uint4 xb = *reinterpret_cast<const uint4*>(xr + ((sw ^ 1u) << 4));
                 const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-                if (i < len) {
+                uint8_t* yr = sBM + q * 8192 + r * 64;
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const __half2 p0 = u32_as_h2(xw[2 * e4]), p1 = u32_as_h2(xw[2 * e4 + 1]);
-                        const float xv[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
-                        float4 o;
-                        o.x = fmaf(Dh, xv[0], fmaf(el, y2[4 * e4], y1[4 * e4]));
-                        o.y = fmaf(Dh, xv[1], fmaf(el, y2[4 * e4 + 1], y1[4 * e4 + 1]));
-                        o.z = fmaf(Dh, xv[2], fmaf(el, y2[4 * e4 + 2], y1[4 * e4 + 2]));
-                        o.w = fmaf(Dh, xv[3], fmaf(el, y2[4 * e4 + 3], y1[4 * e4 + 3]));
-                        reinterpret_cast<float4*>(yrow + 16 * q)[e4] = o;
-                    }
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const __half2 p0 = u32_as_h2(xw[2 * e4]), p1 = u32_as_h2(xw[2 * e4 + 1]);
+                    float4 o;
+                    o.x = fmaf(Dh, __low2float(p0), fmaf(el, y2[4 * e4], y1[4 * e4]));
+                    o.y = fmaf(Dh, __high2float(p0), fmaf(el, y2[4 * e4 + 1], y1[4 * e4 + 1]));
+                    o.z = fmaf(Dh, __low2float(p1), fmaf(el, y2[4 * e4 + 2], y1[4 * e4 + 2]));
+                    o.w = fmaf(Dh, __high2float(p1), fmaf(el, y2[4 * e4 + 3], y1[4 * e4 + 3]));
+                    *reinterpret_cast<float4*>(yr + ((e4 ^ ((r >> 1) & 3)) << 4)) = o;
                 }
             }
         }
+        fence_proxy_async();   // the staging tile -> the TMA store's reads
         tc_fence_before();
-        __syncthreads();   // TMEM, x and lam2 reads done before the next head's copies and writes
-        // the next head's x and S_in: the buffers are free (MMAs complete, epilogue read x); the
-        // copies overlap the next head's M_h
-        if (tid == 0 && hh + 1 < hpg) issue_xs(h + 1, (uint32_t)((hh + 1) & 1));
+        __syncthreads();       // TMEM, x, lam2 and staging done before the store and the next head
+        if (iwarp && lane < L.PA) {   // rows beyond T are clipped by the store
+            tma_store_2d(&mY, sBM + lane * 8192, h * P + 16 * lane, t0 + i0);
+            bulk_commit();
+        }
     }
     // a failed wait may leave copies in flight: give them a bounded chance to land
-    if (tid == 0) {
+    if (iwarp && lane < L.PA) bulk_wait0();
+    if (issuer) {
         if (cb_pending) mbar_wait(&bar_cb, 0, nullptr);
-        if (x_pending) mbar_wait(&bar_x, x_phase, nullptr);
+        for (int b = 0; b < 2; ++b)
+            if (x_pend & (1u << b)) mbar_wait(&bar_x[b], (x_ph >> b) & 1u, nullptr);
     }
     tc_fence_before();
     __syncthreads();
@@ -281,6 +360,33 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+bool ssd_out_tc_supported(int N, int P, int E, int Cx) {
+    return N % 64 == 0 && N >= 64 && N <= 128 && P % 16 == 0 && P >= 16 && P <= 128 && E % 8 == 0 && Cx % 8 == 0;
+}
+
+cudaError_t launch_ssd_out_tc(const uint16_t* xc16, const uint16_t* sin16, const float* dt, const float* lam,
+                              const float* Dv, float* y, int T, int H, int P, int N, int G, int E, int Cx, int* status,
+                              cudaStream_t s) {
+    if (!ssd_out_tc_supported(N, P, E, Cx) || H % G || T < 1 || !status) return cudaErrorInvalidValue;
+    if ((((uintptr_t)xc16) & 15) || (((uintptr_t)sin16) & 15) || (((uintptr_t)y) & 15)) return cudaErrorInvalidValue;
+    const int nch = (T + kQ - 1) / kQ;
+    CUtensorMap mBC, mX, mS, mY;
+    if (!tma_map_2d(&mBC, xc16, T, Cx, Cx, 64, kRows, true, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tma_map_2d(&mX, xc16, T, Cx, Cx, 16, kRows, true, CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !tma_map_2d(&mS, sin16, nch * H * P, N, N, 64, P, false, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tma_map_2d_f32(&mY, y, T, E, E, 16, kRows, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    const size_t smem = (size_t)ssd_out_plan(N, P).total + 1024;
+    cudaError_t e = cudaFuncSetAttribute(pf_ssd_out_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    SsdOutArgs a{};
+    a.dt = dt; a.lam = lam; a.Dv = Dv;
+    a.T = T; a.H = H; a.P = P; a.N = N; a.G = G; a.E = E;
+    a.status = status;
+    pf_ssd_out_tc_kernel<<<2 * nch * G, kOutThreads, smem, s>>>(mBC, mX, mS, mY, a);
+    return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------------------------------
@@ -333,6 +439,8 @@ __global__ void __launch_bounds__(kStThreads) pf_ssd_state_tc_kernel(const float
                                                                      float* __restrict__ lam,
                                                                      float* __restrict__ schunk, int* status) {
     constexpr int N = 128;
+    constexpr int AR = kStSlab * (N / 8) / kStThreads;   // B rows: 8-value items per thread and slab
+    constexpr int XR = kStSlab * (128 / 8) / kStThreads; // x rows: up to P = 128
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     __shared__ double lamd[kQ];
@@ -345,7 +453,63 @@ __global__ void __launch_bounds__(kStThreads) pf_ssd_state_tc_kernel(const float
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const SsdStPlan L = ssd_st_plan(P);
     const float A = -expf(A_log[h]);
+    const float* xh = xc + (size_t)t0 * Cx + (size_t)h * P;
+    const float* bg = xc + (size_t)t0 * Cx + E + (size_t)g * N;
+    const int p8 = P / 8;
 
+    // the next slab's rows, prefetched into registers while the tensor core works on this one
+    float4 ra[AR][2], rx[XR][2];
+    auto load = [&](int f0) {
+#pragma unroll
+        for (int m = 0; m < AR; ++m) {
+            const int idx = tid + m * kStThreads, j = idx >> 4, nc = idx & 15;
+            ra[m][0] = ra[m][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (f0 + j < len) {
+                const float* src = bg + (size_t)(f0 + j) * Cx + 8 * nc;
+                ra[m][0] = *reinterpret_cast<const float4*>(src);
+                ra[m][1] = *reinterpret_cast<const float4*>(src + 4);
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < XR; ++m) {
+            const int idx = tid + m * kStThreads, j = idx / p8, pc = idx - j * p8;
+            rx[m][0] = rx[m][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (j < kStSlab && f0 + j < len) {
+                const float* src = xh + (size_t)(f0 + j) * Cx + 8 * pc;
+                rx[m][0] = *reinterpret_cast<const float4*>(src);
+                rx[m][1] = *reinterpret_cast<const float4*>(src + 4);
+            }
+        }
+    };
+    // split into fp16 halves and write the MN-major swizzled tiles (x scaled by w_j)
+    auto store = [&](int f0) {
+#pragma unroll
+        for (int m = 0; m < AR; ++m) {
+            const int idx = tid + m * kStThreads, j = idx >> 4, nc = idx & 15;
+            const float v[8] = {ra[m][0].x, ra[m][0].y, ra[m][0].z, ra[m][0].w,
+                                ra[m][1].x, ra[m][1].y, ra[m][1].z, ra[m][1].w};
+            uint4 hi, lo;
+            split_f16x8(v, hi, lo);
+            const uint32_t off = (uint32_t)(nc >> 3) * 8192u + (uint32_t)j * 128u + ((uint32_t)((nc & 7) ^ (j & 7)) << 4);
+            *reinterpret_cast<uint4*>(sm + L.off_ah + off) = hi;
+            *reinterpret_cast<uint4*>(sm + L.off_al + off) = lo;
+        }
+#pragma unroll
+        for (int m = 0; m < XR; ++m) {
+            const int idx = tid + m * kStThreads, j = idx / p8, pc = idx - j * p8;
+            if (j >= kStSlab) continue;
+            const float wj = f0 + j < len ? w[f0 + j] : 0.0f;
+            const float v[8] = {rx[m][0].x * wj, rx[m][0].y * wj, rx[m][0].z * wj, rx[m][0].w * wj,
+                                rx[m][1].x * wj, rx[m][1].y * wj, rx[m][1].z * wj, rx[m][1].w * wj};
+            uint4 hi, lo;
+            split_f16x8(v, hi, lo);
+            const uint32_t off = (uint32_t)(pc >> 1) * 2048u + (uint32_t)j * 32u + ((uint32_t)((pc & 1) ^ ((j >> 2) & 1)) << 4);
+            *reinterpret_cast<uint4*>(sm + L.off_xh + off) = hi;
+            *reinterpret_cast<uint4*>(sm + L.off_xl + off) = lo;
+        }
+    };
+
+    load(0);   // in flight during the scan
     if (tid == 0) {
         mbar_init(&bar_mma, 1);
         fence_mbar_init();
@@ -376,13 +540,9 @@ __global__ void __launch_bounds__(kStThreads) pf_ssd_state_tc_kernel(const float
     const uint32_t tmem = tmem_base;
     // decay weights from differences of the unrounded sums
     const double lend = lamd[len - 1];
-    for (int i = tid; i < kQ; i += kStThreads)
-        w[i] = i < len ? expf((float)(lend - lamd[i])) * dt[(size_t)(t0 + i) * H + h] : 0.0f;
+    for (int i = tid; i < len; i += kStThreads) w[i] = expf((float)(lend - lamd[i])) * dt[(size_t)(t0 + i) * H + h];
     __syncthreads();
 
-    const float* xh = xc + (size_t)t0 * Cx + (size_t)h * P;
-    const float* bg = xc + (size_t)t0 * Cx + E + (size_t)g * N;
-    const int p8 = P / 8;
     const uint32_t idesc = umma_idesc(false, true, N, P, true);
     const int nsl = (len + kStSlab - 1) / kStSlab;
     bool ok = true;
@@ -391,43 +551,8 @@ __global__ void __launch_bounds__(kStThreads) pf_ssd_state_tc_kernel(const float
             ok = __syncthreads_and(mbar_wait(&bar_mma, (uint32_t)((sl - 1) & 1), status));
             if (!ok) break;
         }
-        const int f0 = sl * kStSlab;
-        for (int idx = tid; idx < kStSlab * (N / 8); idx += kStThreads) {
-            const int j = idx >> 4, nc = idx & 15;
-            float v[8];
-            if (f0 + j < len) {
-                const float4 a0 = *reinterpret_cast<const float4*>(bg + (size_t)(f0 + j) * Cx + 8 * nc);
-                const float4 a1 = *reinterpret_cast<const float4*>(bg + (size_t)(f0 + j) * Cx + 8 * nc + 4);
-                v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w; v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = 0.0f;
-            }
-            uint4 hi, lo;
-            split_f16x8(v, hi, lo);
-            const uint32_t off = (uint32_t)(nc >> 3) * 8192u + (uint32_t)j * 128u + ((uint32_t)((nc & 7) ^ (j & 7)) << 4);
-            *reinterpret_cast<uint4*>(sm + L.off_ah + off) = hi;
-            *reinterpret_cast<uint4*>(sm + L.off_al + off) = lo;
-        }
-        for (int idx = tid; idx < kStSlab * p8; idx += kStThreads) {
-            const int j = idx / p8, pc = idx - j * p8;
-            float v[8];
-            if (f0 + j < len) {
-                const float wj = w[f0 + j];
-                const float4 a0 = *reinterpret_cast<const float4*>(xh + (size_t)(f0 + j) * Cx + 8 * pc);
-                const float4 a1 = *reinterpret_cast<const float4*>(xh + (size_t)(f0 + j) * Cx + 8 * pc + 4);
-                v[0] = a0.x * wj; v[1] = a0.y * wj; v[2] = a0.z * wj; v[3] = a0.w * wj;
-                v[4] = a1.x * wj; v[5] = a1.y * wj; v[6] = a1.z * wj; v[7] = a1.w * wj;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = 0.0f;
-            }
-            uint4 hi, lo;
-            split_f16x8(v, hi, lo);
-            const uint32_t off = (uint32_t)(pc >> 1) * 2048u + (uint32_t)j * 32u + ((uint32_t)((pc & 1) ^ ((j >> 2) & 1)) << 4);
-            *reinterpret_cast<uint4*>(sm + L.off_xh + off) = hi;
-            *reinterpret_cast<uint4*>(sm + L.off_xl + off) = lo;
-        }
+        store(sl * kStSlab);
+        if (sl + 1 < nsl) load((sl + 1) * kStSlab);
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -472,7 +597,7 @@ __global__ void __launch_bounds__(kStThreads) pf_ssd_state_tc_kernel(const float
 }
 
 bool ssd_state_tc_supported(int N, int P, int E, int Cx) {
-    return N == 128 && P % 16 == 0 && P >= 16 && P <= 256 && E % 4 == 0 && Cx % 4 == 0;
+    return N == 128 && P % 16 == 0 && P >= 16 && P <= 128 && E % 4 == 0 && Cx % 4 == 0;
 }
 
 cudaError_t launch_ssd_state_tc(const float* xc, const float* dt, const float* A_log, int T, int H, int P, int N, int G,
@@ -485,33 +610,6 @@ cudaError_t launch_ssd_state_tc(const float* xc, const float* dt, const float* A
     const int nch = (T + kQ - 1) / kQ;
     pf_ssd_state_tc_kernel<<<dim3(nch, H), kStThreads, smem, s>>>(xc, dt, A_log, T, H, P, G, E, Cx, lam, schunk,
                                                                   status);
-    return cudaGetLastError();
-}
-
-bool ssd_out_tc_supported(int N, int P, int E, int Cx) {
-    return N % 64 == 0 && N >= 64 && N <= 128 && P % 16 == 0 && P >= 16 && P <= 128 && E % 8 == 0 && Cx % 8 == 0;
-}
-
-cudaError_t launch_ssd_out_tc(const uint16_t* xc16, const uint16_t* sin16, const float* dt, const float* lam,
-                              const float* Dv, float* y, int T, int H, int P, int N, int G, int E, int Cx, int* status,
-                              cudaStream_t s) {
-    if (!ssd_out_tc_supported(N, P, E, Cx) || H % G || T < 1 || !status) return cudaErrorInvalidValue;
-    if ((((uintptr_t)xc16) & 15) || (((uintptr_t)sin16) & 15)) return cudaErrorInvalidValue;
-    const int nch = (T + kQ - 1) / kQ;
-    CUtensorMap mC, mB, mX, mS;
-    if (!tma_map_2d(&mC, xc16, T, Cx, Cx, 64, kRows, true, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !tma_map_2d(&mB, xc16, T, Cx, Cx, 64, kQ, true, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !tma_map_2d(&mX, xc16, T, Cx, Cx, 16, kQ, true, CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !tma_map_2d(&mS, sin16, nch * H * P, N, N, 64, P, false, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    const size_t smem = (size_t)ssd_out_plan(N, P).total + 1024;
-    cudaError_t e = cudaFuncSetAttribute(pf_ssd_out_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    SsdOutArgs a{};
-    a.dt = dt; a.lam = lam; a.Dv = Dv; a.y = y;
-    a.T = T; a.H = H; a.P = P; a.N = N; a.G = G; a.E = E;
-    a.status = status;
-    pf_ssd_out_tc_kernel<<<2 * nch * G, kOutThreads, smem, s>>>(mC, mB, mX, mS, a);
     return cudaGetLastError();
 }
 
