@@ -96,17 +96,43 @@ __global__ void pf_rownorm_kernel(const uint16_t* x, float* r, const float* gamm
                                   int d, float eps, int f16) {
     const int t = blockIdx.x;
     float* rr = r + (size_t)t * d;
+    uint16_t* ar = act + (size_t)t * ld;
     float ss = 0.0f;
-    for (int k = threadIdx.x; k < d; k += blockDim.x) {
-        float v;
-        if (x) {
-            v = bf16_bits_to_f(x[(size_t)t * d + k]);
-            rr[k] = v;
-        } else {
-            v = rr[k];
+    if ((d & 3) == 0 && (ld & 3) == 0) {   // 4 columns per step: 16-byte r, 8-byte act accesses
+        for (int k = 4 * threadIdx.x; k < d; k += 4 * blockDim.x) {
+            float4 v;
+            if (x) {
+                const uint2 xb = *reinterpret_cast<const uint2*>(x + (size_t)t * d + k);
+                v = make_float4(bf16_bits_to_f((uint16_t)(xb.x & 0xFFFFu)), bf16_bits_to_f((uint16_t)(xb.x >> 16)),
+                                bf16_bits_to_f((uint16_t)(xb.y & 0xFFFFu)), bf16_bits_to_f((uint16_t)(xb.y >> 16)));
+                *reinterpret_cast<float4*>(rr + k) = v;
+            } else {
+                v = *reinterpret_cast<const float4*>(rr + k);
+            }
+            ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+            const float4 g = *reinterpret_cast<const float4*>(gamma + k);
+            uint2 o;
+            if (f16) {
+                o.x = (uint32_t)act_bits<true>(v.x * g.x) | ((uint32_t)act_bits<true>(v.y * g.y) << 16);
+                o.y = (uint32_t)act_bits<true>(v.z * g.z) | ((uint32_t)act_bits<true>(v.w * g.w) << 16);
+            } else {
+                o.x = (uint32_t)act_bits<false>(v.x * g.x) | ((uint32_t)act_bits<false>(v.y * g.y) << 16);
+                o.y = (uint32_t)act_bits<false>(v.z * g.z) | ((uint32_t)act_bits<false>(v.w * g.w) << 16);
+            }
+            *reinterpret_cast<uint2*>(ar + k) = o;
         }
-        ss += v * v;
-        act[(size_t)t * ld + k] = f16 ? act_bits<true>(v * gamma[k]) : act_bits<false>(v * gamma[k]);
+    } else {
+        for (int k = threadIdx.x; k < d; k += blockDim.x) {
+            float v;
+            if (x) {
+                v = bf16_bits_to_f(x[(size_t)t * d + k]);
+                rr[k] = v;
+            } else {
+                v = rr[k];
+            }
+            ss += v * v;
+            ar[k] = f16 ? act_bits<true>(v * gamma[k]) : act_bits<false>(v * gamma[k]);
+        }
     }
     __shared__ float red[32];
     ss = warp_sum(ss);
@@ -176,6 +202,70 @@ __global__ void __launch_bounds__(256) pf_conv_kernel(const uint16_t* __restrict
 }
 
 // dt = softplus(dt_raw + dt_bias) for every frame and head
+// the same for conv width 4 with 4 adjacent channels per thread (8-byte input loads, 16- and
+// 8-byte output stores); requires E, Cx and the zx row width to be multiples of 4
+__global__ void __launch_bounds__(256) pf_conv4x4_kernel(const uint16_t* __restrict__ zx, int zxw, int T, int E, int Cx,
+                                                         const float* __restrict__ conv_w,
+                                                         const float* __restrict__ conv_b, float* __restrict__ xc,
+                                                         uint16_t* __restrict__ xc16, uint16_t* __restrict__ ring) {
+    constexpr int W = 4;
+    const int c = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (c >= Cx) return;
+    const int t0 = blockIdx.y * kConvTF, t1 = min(T, t0 + kConvTF);
+    const uint16_t* col = zx + E + c;
+    float w[4][W], hist[4][W - 1], bias[4];
+    auto unpack = [](uint2 v, float (&f)[4]) {
+        f[0] = bf16_bits_to_f((uint16_t)(v.x & 0xFFFFu));
+        f[1] = bf16_bits_to_f((uint16_t)(v.x >> 16));
+        f[2] = bf16_bits_to_f((uint16_t)(v.y & 0xFFFFu));
+        f[3] = bf16_bits_to_f((uint16_t)(v.y >> 16));
+    };
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        bias[ch] = conv_b[c + ch];
+#pragma unroll
+        for (int k = 0; k < W; ++k) w[ch][k] = conv_w[(c + ch) * W + k];
+    }
+#pragma unroll
+    for (int k = 0; k < W - 1; ++k) {
+        const int tt = t0 - (W - 1) + k;
+        float f[4] = {0.f, 0.f, 0.f, 0.f};
+        if (tt >= 0) unpack(*reinterpret_cast<const uint2*>(col + (size_t)tt * zxw), f);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) hist[ch][k] = f[ch];
+    }
+    constexpr int U = 8;   // frames whose inputs are loaded together
+    for (int tb = t0; tb < t1; tb += U) {
+        uint2 raws[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            raws[u] = tb + u < t1 ? *reinterpret_cast<const uint2*>(col + (size_t)(tb + u) * zxw) : make_uint2(0u, 0u);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int t = tb + u;
+            if (t >= t1) break;
+            float xv[4], v[4];
+            unpack(raws[u], xv);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                float acc = bias[ch];
+#pragma unroll
+                for (int k = 0; k < W - 1; ++k) acc += w[ch][k] * hist[ch][k];
+                acc += w[ch][W - 1] * xv[ch];
+#pragma unroll
+                for (int k = 0; k < W - 2; ++k) hist[ch][k] = hist[ch][k + 1];
+                hist[ch][W - 2] = xv[ch];
+                v[ch] = silu_f(acc);
+            }
+            *reinterpret_cast<float4*>(xc + (size_t)t * Cx + c) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<uint2*>(xc16 + (size_t)t * Cx + c) =
+                make_uint2((uint32_t)f16_bits(v[0]) | ((uint32_t)f16_bits(v[1]) << 16),
+                           (uint32_t)f16_bits(v[2]) | ((uint32_t)f16_bits(v[3]) << 16));
+            if (t >= T - (W - 1)) *reinterpret_cast<uint2*>(ring + (size_t)(t % W) * Cx + c) = raws[u];
+        }
+    }
+}
+
 __global__ void pf_dt_kernel(const uint16_t* __restrict__ zx, int zxw, int T, int off, int H,
                              const float* __restrict__ dt_bias, float* __restrict__ dt) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -284,7 +374,9 @@ __global__ void __launch_bounds__(256) pf_ssd_state_kernel(const float* __restri
         }
 }
 
-// scan over chunks: S_in(0) = 0, S_in(c+1) = exp(Lam_end(c)) S_in(c) + S_c; final -> ssm state
+// scan over chunks: S_in(0) = 0, S_in(c+1) = exp(Lam_end(c)) S_in(c) + S_c; final -> ssm state.
+// The chunk states and decays of 8 chunks are loaded before their part of the recurrence, so
+// the loads overlap instead of following the chain one by one.
 __global__ void pf_ssd_scan_kernel(const float* schunk, const float* lam, int T, int H, int P, int N,
                                    uint16_t* sin16, float* ssm_out) {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -292,17 +384,35 @@ __global__ void pf_ssd_scan_kernel(const float* schunk, const float* lam, int T,
     if (idx >= (long long)H * per_head) return;
     const int h = (int)(idx / per_head);
     const int nch = (T + kChunk - 1) / kChunk;
+    const size_t cs = (size_t)H * per_head;
     float s = 0.0f;
-    for (int c = 0; c < nch; ++c) {
-        sin16[(size_t)c * H * per_head + idx] = bf16_bits(s);
-        const int tend = min(T, (c + 1) * kChunk) - 1;
-        s = expf(lam[(size_t)tend * H + h]) * s + schunk[(size_t)c * H * per_head + idx];
+    for (int c0 = 0; c0 < nch; c0 += 8) {
+        float sc[8], dec[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int c = c0 + k;
+            sc[k] = dec[k] = 0.0f;
+            if (c < nch) {
+                sc[k] = schunk[(size_t)c * cs + idx];
+                dec[k] = lam[(size_t)(min(T, (c + 1) * kChunk) - 1) * H + h];
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (c0 + k < nch) {
+                sin16[(size_t)(c0 + k) * cs + idx] = bf16_bits(s);
+                s = expf(dec[k]) * s + sc[k];
+            }
     }
     ssm_out[idx] = s;
 }
 
 // v = y * silu(z); per row and norm group: act = bf16(v * rsqrt(mean(v^2) + eps) * gamma).
-// CTA = one frame, one warp per norm group (warp-level reductions only)
+// CTA = one frame, one warp per norm group (warp-level reductions only).  Groups of a multiple
+// of 128 columns: each lane takes 4 consecutive columns per step (16-byte y, 8-byte z loads)
+// and keeps v in registers between the two passes.
+static constexpr int kGnMaxPerLane = 64;   // vector path: group size up to 32 x 64 columns
+
 __global__ void pf_gated_norm_kernel(const float* __restrict__ y, const uint16_t* __restrict__ zx, int zxw,
                                      const float* __restrict__ gnorm, int E, int NG, float eps,
                                      uint16_t* __restrict__ act, int ld, int f16) {
@@ -311,6 +421,46 @@ __global__ void pf_gated_norm_kernel(const float* __restrict__ y, const uint16_t
     const int gs = E / NG, c0 = q * gs;
     const float* yr = y + (size_t)t * E;
     const uint16_t* zr = zx + (size_t)t * zxw;
+    uint16_t* ar = act + (size_t)t * ld;
+    const bool vec = (gs & 127) == 0 && gs / 32 <= kGnMaxPerLane && (zxw & 3) == 0 && (ld & 3) == 0 && (E & 3) == 0;
+    if (vec) {
+        float v[kGnMaxPerLane];
+        const int steps = gs / 128;
+        float ss = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kGnMaxPerLane / 4; ++k) {
+            if (k >= steps) break;
+            const int c = c0 + 128 * k + 4 * lane;
+            const float4 y4 = *reinterpret_cast<const float4*>(yr + c);
+            const uint2 z4 = *reinterpret_cast<const uint2*>(zr + c);
+            v[4 * k] = y4.x * silu_f(bf16_bits_to_f((uint16_t)(z4.x & 0xFFFFu)));
+            v[4 * k + 1] = y4.y * silu_f(bf16_bits_to_f((uint16_t)(z4.x >> 16)));
+            v[4 * k + 2] = y4.z * silu_f(bf16_bits_to_f((uint16_t)(z4.y & 0xFFFFu)));
+            v[4 * k + 3] = y4.w * silu_f(bf16_bits_to_f((uint16_t)(z4.y >> 16)));
+            ss += v[4 * k] * v[4 * k] + v[4 * k + 1] * v[4 * k + 1] + v[4 * k + 2] * v[4 * k + 2] +
+                  v[4 * k + 3] * v[4 * k + 3];
+        }
+        ss = warp_sum(ss);
+        const float ginv = rsqrtf(ss / gs + eps);
+#pragma unroll
+        for (int k = 0; k < kGnMaxPerLane / 4; ++k) {
+            if (k >= steps) break;
+            const int c = c0 + 128 * k + 4 * lane;
+            const float4 g4 = *reinterpret_cast<const float4*>(gnorm + c);
+            const float u0 = v[4 * k] * ginv * g4.x, u1 = v[4 * k + 1] * ginv * g4.y;
+            const float u2 = v[4 * k + 2] * ginv * g4.z, u3 = v[4 * k + 3] * ginv * g4.w;
+            uint2 o;
+            if (f16) {
+                o.x = (uint32_t)act_bits<true>(u0) | ((uint32_t)act_bits<true>(u1) << 16);
+                o.y = (uint32_t)act_bits<true>(u2) | ((uint32_t)act_bits<true>(u3) << 16);
+            } else {
+                o.x = (uint32_t)act_bits<false>(u0) | ((uint32_t)act_bits<false>(u1) << 16);
+                o.y = (uint32_t)act_bits<false>(u2) | ((uint32_t)act_bits<false>(u3) << 16);
+            }
+            *reinterpret_cast<uint2*>(ar + c) = o;
+        }
+        return;
+    }
     float ss = 0.0f;
 #pragma unroll 4
     for (int c = c0 + lane; c < c0 + gs; c += 32) {
@@ -322,7 +472,7 @@ __global__ void pf_gated_norm_kernel(const float* __restrict__ y, const uint16_t
 #pragma unroll 4
     for (int c = c0 + lane; c < c0 + gs; c += 32) {
         const float u = yr[c] * silu_f(bf16_bits_to_f(zr[c])) * ginv * gnorm[c];
-        act[(size_t)t * ld + c] = f16 ? act_bits<true>(u) : act_bits<false>(u);
+        ar[c] = f16 ? act_bits<true>(u) : act_bits<false>(u);
     }
 }
 
@@ -409,7 +559,10 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
     if ((e = cudaMemsetAsync(m.ring, 0, (size_t)W * Cx * 2, s)) != cudaSuccess) return e;
     if (W > 8 || m.NG > 32) return cudaErrorNotSupported;
     const dim3 cg((Cx + 255) / 256, (T + kConvTF - 1) / kConvTF);
-    if (W == 4)
+    if (W == 4 && E % 4 == 0 && Cx % 4 == 0 && zxw % 4 == 0)
+        pf_conv4x4_kernel<<<dim3((Cx / 4 + 255) / 256, (T + kConvTF - 1) / kConvTF), 256, 0, s>>>(
+            m.zx, zxw, T, E, Cx, Lw.conv_w, Lw.conv_b, m.xc, m.xc16, m.ring);
+    else if (W == 4)
         pf_conv_kernel<4><<<cg, 256, 0, s>>>(m.zx, zxw, T, E, Cx, W, Lw.conv_w, Lw.conv_b, m.xc, m.xc16, m.ring);
     else
         pf_conv_kernel<0><<<cg, 256, 0, s>>>(m.zx, zxw, T, E, Cx, W, Lw.conv_w, Lw.conv_b, m.xc, m.xc16, m.ring);
