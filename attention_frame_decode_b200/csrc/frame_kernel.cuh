@@ -600,11 +600,11 @@ __device__ __forceinline__ bool fk_gemv_run(const FkGemv& G, const float* insc_t
             }
             if constexpr (ACT_SMEM) {
                 act.load(kt, bv);
-                consume_block_bv<FMT, GRP, NT>(base + jb * L.block_bytes, bv, lane, sc, acc);
+                consume_block_bv<FMT, GRP, NT>(base + jb * L.block_bytes, bv, lane, sc, acc, B > 1, G.epi == EPI_ARGMAX);
             } else {
                 uint4 bn[L.SUB][NT][2];
                 act.load(kt + 1 == KT ? 0 : kt + 1, bn);   // one block ahead
-                consume_block_bv<FMT, GRP, NT>(base + jb * L.block_bytes, bv, lane, sc, acc);
+                consume_block_bv<FMT, GRP, NT>(base + jb * L.block_bytes, bv, lane, sc, acc, B > 1, G.epi == EPI_ARGMAX);
 #pragma unroll
                 for (int st = 0; st < L.SUB; ++st)
 #pragma unroll

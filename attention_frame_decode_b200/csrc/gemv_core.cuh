@@ -186,17 +186,155 @@ __device__ __forceinline__ void step_frags(const TileWords<FMT>& tw, int s, cons
     }
 }
 
+// W8 and W4 with the zero point deferred: the A fragments hold the codes read as fp16 1024 + code
+// (W8: one prmt per register; W4: one lop3, the nibble of row g+8 read as 1024 + 16 q), so the
+// products are sum (1024 + code) u; the group's activation sum U = sum u, produced by an MMA of
+// the same activation fragments with an all-ones A, removes the offset once per group:
+//   W8 (stored q + 128):  sum q u = c - 1152 U
+//   W4 row g:             sum (q - z) u = c - (1024 + z) U
+//   W4 row g+8:           sum (q - z) u = c / 16 - (64 + z) U
+// Products of fp16 values are exact and summed in fp32; the offset sums are ~10^3 x the result
+// at most, which leaves ~1e-4 relative error per group sum.  SYM (the vocabulary heads, whose
+// greedy argmax must see equal rows as equal): both rows of a slab are read at scale 1 (two more
+// shifts per word), so two rows holding the same codes give the same sums bit for bit.
+template <int FMT>
+__host__ __device__ constexpr bool deferred_zero() { return FMT == FMT_W8 || FMT == FMT_W4; }
+
+template <int FMT, bool SYM>
+__device__ __forceinline__ void step_frags_raw(const TileWords<FMT>& tw, int s, uint32_t (&a)[4]) {
+    if constexpr (FMT == FMT_W8) {
+        const uint32_t M8 = 0x64646464u;      // prmt source of the 0x64 exponent byte
+        const int c = s >> 1, h = s & 1;
+        const uint32_t A = tw.w[4 * c + 2 * h], B = tw.w[4 * c + 2 * h + 1];
+        a[0] = prmt(A, M8, 0x4240);
+        a[1] = prmt(B, M8, 0x4240);
+        a[2] = prmt(A, M8, 0x4341);
+        a[3] = prmt(B, M8, 0x4341);
+    } else if constexpr (SYM) {
+        const uint32_t M = 0x64006400u;
+        const uint32_t x = tw.w[s];
+        a[0] = and_or(x, 0x000F000Fu, M);
+        a[1] = and_or(x >> 4, 0x000F000Fu, M);
+        a[2] = and_or(x >> 8, 0x000F000Fu, M);
+        a[3] = and_or(x >> 12, 0x000F000Fu, M);
+    } else {
+        const uint32_t M = 0x64006400u;
+        const uint32_t x = tw.w[s], y = tw.w[s] >> 8;
+        a[0] = and_or(x, 0x000F000Fu, M);
+        a[1] = and_or(x, 0x00F000F0u, M);
+        a[2] = and_or(y, 0x000F000Fu, M);
+        a[3] = and_or(y, 0x00F000F0u, M);
+    }
+}
+
+// exact float of a small non-negative integer n < 2^23 (bits OR-ed into 2^23, minus 2^23)
+__device__ __forceinline__ float small_int_f(uint32_t n) { return __uint_as_float(0x4B000000u | n) - 8388608.0f; }
+
 // one block: acc[r][j] += scale * (slab r of the block) . (activation k-step, column tile j)
 //   bv[st][j]: the lane's two 16-byte pieces of activation row 8j + g (columns 64 st + 16 t ..
 //              64 st + 16 t + 15 of the k-step; zero for rows >= B)
 //   sc[j][e]:  input scale of batch column 8j + 2t + e for this k-step
+//   col1:      the odd batch columns 2t + 1 are used (B > 1); when false their sums are not formed
 // All tiles' words and slab metadata are loaded first; then each k16 step dequantizes one
 // register quad per slab and issues the slabs' MMAs back to back, so the R accumulation chains
 // interleave instead of running one after another.
+template <int FMT, int GRP, int NT, bool SYM>
+__device__ __forceinline__ void consume_block_dz(const uint8_t* blk, const uint4 (&bv)[layout_info(FMT, GRP).SUB][NT][2],
+                                                 int lane, const float (&sc)[NT][2],
+                                                 float (&acc)[layout_info(FMT, GRP).R][NT][4], bool col1) {
+    constexpr LayoutInfo L = layout_info(FMT, GRP);
+    constexpr int R = L.R, SUB = L.SUB;
+    const int g = lane >> 2;
+    TileWords<FMT> tw[R][SUB];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int st = 0; st < SUB; ++st) load_tile_words<FMT>(blk + (r * SUB + st) * L.tile_bytes, lane, tw[r][st]);
+    float c[R][NT][4], cu[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        cu[j][0] = cu[j][1] = cu[j][2] = cu[j][3] = 0.0f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) c[r][j][0] = c[r][j][1] = c[r][j][2] = c[r][j][3] = 0.0f;
+    }
+    const uint32_t ones[4] = {0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u};   // fp16 1.0 pairs
+#pragma unroll
+    for (int st = 0; st < SUB; ++st)
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const uint4& v = bv[st][j][s >> 1];
+                mma_f16(cu[j], ones, (s & 1) ? v.z : v.x, (s & 1) ? v.w : v.y);
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                uint32_t a[4];
+                step_frags_raw<FMT, SYM>(tw[r][st], s, a);
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    const uint4& v = bv[st][j][s >> 1];
+                    mma_f16(c[r][j], a, (s & 1) ? v.z : v.x, (s & 1) ? v.w : v.y);
+                }
+            }
+        }
+    // slab metadata (scales; W4 zeros) read after the products, so its registers are not live
+    // across them
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const uint8_t* meta = blk + R * SUB * L.tile_bytes + r * L.meta_bytes;
+        const __half2 sp = *reinterpret_cast<const __half2*>(meta + g * 4);
+        const float s_lo = __low2float(sp), s_hi = __high2float(sp);
+        float zl = 1152.0f, zh = 1152.0f;
+        if constexpr (FMT == FMT_W4) {
+            const uint32_t zb = meta[32 + g];
+            zl = small_int_f(1024u + (zb & 15u));
+            zh = small_int_f((SYM ? 1024u : 64u) + (zb >> 4));
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            float v0, v2;
+            if constexpr (FMT == FMT_W4 && SYM) {
+                v0 = fmaf(-zl, cu[j][0], c[r][j][0]);
+                v2 = fmaf(-zh, cu[j][0], c[r][j][2]);
+            } else if constexpr (FMT == FMT_W4) {
+                v0 = fmaf(-zl, cu[j][0], c[r][j][0]);
+                v2 = fmaf(c[r][j][2], 0.0625f, -zh * cu[j][0]);
+            } else {
+                v0 = fmaf(-1152.0f, cu[j][0], c[r][j][0]);
+                v2 = fmaf(-1152.0f, cu[j][0], c[r][j][2]);
+            }
+            acc[r][j][0] = fmaf(s_lo * sc[j][0], v0, acc[r][j][0]);
+            acc[r][j][2] = fmaf(s_hi * sc[j][0], v2, acc[r][j][2]);
+            if (NT > 1 || col1) {
+                float v1, v3;
+                if constexpr (FMT == FMT_W4 && SYM) {
+                    v1 = fmaf(-zl, cu[j][1], c[r][j][1]);
+                    v3 = fmaf(-zh, cu[j][1], c[r][j][3]);
+                } else if constexpr (FMT == FMT_W4) {
+                    v1 = fmaf(-zl, cu[j][1], c[r][j][1]);
+                    v3 = fmaf(c[r][j][3], 0.0625f, -zh * cu[j][1]);
+                } else {
+                    v1 = fmaf(-1152.0f, cu[j][1], c[r][j][1]);
+                    v3 = fmaf(-1152.0f, cu[j][1], c[r][j][3]);
+                }
+                acc[r][j][1] = fmaf(s_lo * sc[j][1], v1, acc[r][j][1]);
+                acc[r][j][3] = fmaf(s_hi * sc[j][1], v3, acc[r][j][3]);
+            }
+        }
+    }
+}
+
 template <int FMT, int GRP, int NT>
 __device__ __forceinline__ void consume_block_bv(const uint8_t* blk, const uint4 (&bv)[layout_info(FMT, GRP).SUB][NT][2],
                                                  int lane, const float (&sc)[NT][2],
-                                                 float (&acc)[layout_info(FMT, GRP).R][NT][4]) {
+                                                 float (&acc)[layout_info(FMT, GRP).R][NT][4], bool col1 = true,
+                                                 bool sym = false) {
+    if constexpr (deferred_zero<FMT>()) {
+        if (FMT == FMT_W4 && sym) consume_block_dz<FMT, GRP, NT, true>(blk, bv, lane, sc, acc, col1);
+        else consume_block_dz<FMT, GRP, NT, false>(blk, bv, lane, sc, acc, col1);
+        return;
+    }
     constexpr LayoutInfo L = layout_info(FMT, GRP);
     constexpr int R = L.R, SUB = L.SUB;
     const int g = lane >> 2;
@@ -262,7 +400,7 @@ __device__ __forceinline__ void consume_block_bv(const uint8_t* blk, const uint4
 //   arow(b): byte address of activation row b's 64-column slice st = 0 of this k-step
 // Columns b >= B read row B-1 instead of zeros: their sums are computed and never stored (every
 // epilogue checks b < B), and the loads need no branch.
-template <int FMT, int GRP, int NT, typename ActRow>
+template <int FMT, int GRP, int NT, bool SYM = false, typename ActRow>
 __device__ __forceinline__ void consume_block(const uint8_t* blk, ActRow arow, int B, int lane, const float (&sc)[NT][2],
                                               float (&acc)[layout_info(FMT, GRP).R][NT][4]) {
     constexpr int SUB = layout_info(FMT, GRP).SUB;
@@ -277,7 +415,7 @@ __device__ __forceinline__ void consume_block(const uint8_t* blk, ActRow arow, i
             bv[st][j][0] = *reinterpret_cast<const uint4*>(p);
             bv[st][j][1] = *reinterpret_cast<const uint4*>(p + 16);
         }
-    consume_block_bv<FMT, GRP, NT>(blk, bv, lane, sc, acc);
+    consume_block_bv<FMT, GRP, NT>(blk, bv, lane, sc, acc, B > 1, SYM);
 }
 
 // ------------------------------------------------------------------------------------------

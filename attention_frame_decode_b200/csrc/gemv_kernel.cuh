@@ -168,9 +168,11 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
             }
             if (rg_act_smem) {
                 const uint8_t* abase = act_s + (size_t)kt * KS * 2;
-                consume_block<FMT, GRP, NT>(blk, [&](int b) { return abase + (size_t)b * rg_act_stride; }, B, lane, sc, acc);
+                consume_block<FMT, GRP, NT, EPI == EPI_ARGMAX>(blk, [&](int b) { return abase + (size_t)b * rg_act_stride; }, B,
+                                                              lane, sc, acc);
             } else {
-                consume_block<FMT, GRP, NT>(blk, [&](int b) { return arow0 + b * rg_act_row; }, B, lane, sc, acc);
+                consume_block<FMT, GRP, NT, EPI == EPI_ARGMAX>(blk, [&](int b) { return arow0 + b * rg_act_row; }, B, lane,
+                                                              sc, acc);
             }
             pending = true;
             if (++kt == KT) {   // the unit's last k-step: finish it (or hand over the partial)

@@ -333,10 +333,11 @@ def test_mamba_step_kernel_state(cuda, T):
 
 def _planted_rows(win, V):
     """destination of a copy of head row `win`: its partner in the same 16-row slab (rows g and
-    g+8, one lane's two accumulator rows).  Both rows then take the same dequantized values through
-    the same products and the same split of the row unit between warps, so their logits are equal
-    bit for bit.  (A copy in another row unit is cut between warps at other k-steps; its fp32 sum
-    may round differently, so it is not an exact tie.)"""
+    g+8, one lane's two accumulator rows, merged between warps by the same vector reductions).
+    The head GEMV reads both rows' codes at the same scale, so they take the same dequantized
+    values through the same products and the same split of the row unit between warps: their
+    logits are equal bit for bit.  (A copy in another slab or row unit is merged by other
+    reductions, whose order between warps may differ, so it is not an exact tie.)"""
     return [win - 8 if win % 16 >= 8 else win + 8]
 
 
