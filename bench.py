@@ -2,12 +2,14 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl vc|reference]
 
-Default workload: the Nemotron-Nano-9B-v2-shaped backbone with bf16 weights, batch 1, steady
-state decode at a context of 2000 frames (KV cache and SSM state pre-filled from N(0,1)),
-synthetic seeded weights N(0, 0.02) and inputs N(0, 1).  One "step" is one frame through all
-56 layers and both vocabulary heads.  Other workloads: --config nano_w4 | nano_w3 |
-nano_w8_b16 | tiny_w8 (see synth.CONFIGS), and nano_prefill: one step is then one prefill of the
-4096-frame opening context (tensor-core GEMMs, chunked SSD, causal attention).
+Default workload: the Nemotron-Nano-9B-v2-shaped backbone with W4 group-64 weights (bf16 heads),
+batch 1, steady state decode at a context of 2000 frames (KV cache and SSM state pre-filled from
+N(0,1)), synthetic seeded weights N(0, 0.02) and inputs N(0, 1).  One "step" is one frame through
+all 56 layers and both vocabulary heads.  The same run then measures the bf16-weight backbone
+(nano_bf16) for up to 300 steps and reports it under "also" (--no-second skips it).  Other
+workloads: --config nano_bf16 | nano_w3 | nano_w4_qheads | nano_w8_b16 | tiny_w8 (see
+synth.CONFIGS), and nano_prefill: one step is then one prefill of the 4096-frame opening context
+(tensor-core GEMMs, chunked SSD, causal attention).
 
 With N > 1 (torchrun) every rank serves its own independent sessions with a full replica of
 the weights (no collective on the data path); the reported value is the sum over ranks of
@@ -31,6 +33,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "backbone frame-steps/s & ms/frame at batch 1 and 16; achieved HBM GB/s vs 8 TB/s"
+DEFAULT_CONFIG = "nano_w4"   # the batch-1 W4 backbone (the configuration the HBM-roofline target names)
 
 
 # ------------------------------------------------------------------------------------------------
@@ -399,6 +402,163 @@ def run_prefill_bench(args, cfg, world, rank, local):
         dist.destroy_process_group()
 
 
+def run_decode(args, cfg, world, rank, local, steps, e2e_steps, cpu_baseline):
+    """one decode measurement of workload cfg: `steps` timed frame-steps after args.warmup, the GEMV
+    roofline launch and the end-to-end host run; returns the JSON line on rank 0 (else None)"""
+    import torch
+    import torch.distributed as dist
+    import attention_frame_decode_b200 as vc
+    from attention_frame_decode_b200.synthetic import build_model, fill_state
+
+    B = cfg.batch
+    seed = 0
+    dm = build_model(cfg, seed)
+    ctx0 = synth.context_lengths(cfg, seed, B)
+    total = args.warmup + steps
+    # the workload's cache capacity, grown when the run itself needs more frames than it holds
+    cap = max(cfg.kv_capacity, int(ctx0.max()) + total + e2e_steps + 8)
+    bb = dm.backbone(B, cap, B)
+    if args.no_graph:
+        bb.set_option(vc.OPT_GRAPH, 0)
+    if args.per_kernel:
+        bb.set_option(vc.OPT_FRAME, 0)
+    if args.frame:
+        bb.set_option(vc.OPT_FRAME, 1)
+    frame = bb.uses_frame_kernel(B)
+    st = dm.new_state(B, cap)
+    if cfg.random_state:
+        fill_state(st, cfg, seed + rank, ctx0, cap)
+    # every frame input of the run, resident in HBM before timing (rank r serves its own sessions)
+    xs = torch.empty((total, B, cfg.d_model), dtype=torch.bfloat16, device="cuda")
+    for s in range(total):
+        xs[s] = torch.from_numpy(synth.frame_inputs(cfg, seed + 1000 * rank, s, B)).view(torch.bfloat16)
+    tt = torch.zeros((B,), dtype=torch.int32, device="cuda")
+    tf = torch.zeros((B,), dtype=torch.int32, device="cuda")
+    if int(cap - ctx0.max()) < total + e2e_steps + 8:
+        raise SystemExit(f"kv capacity {cap} too small for {total + e2e_steps} steps")
+
+    for s in range(args.warmup):
+        bb.step(xs[s], st, tt, tf)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(args.warmup, total):
+        bb.step(xs[s], st, tt, tf)
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms, world)
+    status = int(st.status.cpu()[0])
+    ms_step = ms / steps
+    value = replica_rate(B * steps, world, ms / 1000.0)
+    ctx_mean = float(ctx0.mean()) + args.warmup + steps / 2.0
+    rbytes, wbytes, weight_total = step_bytes(cfg, B, ctx_mean)
+    step_gbs = rbytes / (ms_step / 1000.0) / 1e9
+
+    # ---- roofline of the dominant kernel: the streaming GEMV on the layer MLP up projection ----
+    peak, peak_kind = load_peaks()
+    mlp = cfg.pattern.index("-")
+    up = dm.layers[mlp].up
+    K_up = cfg.d_model
+    act_ld = (K_up + 127) // 128 * 128
+    act = torch.zeros((B, act_ld), dtype=torch.bfloat16 if cfg.wfmt == synth.FMT_BF16 else torch.float16,
+                      device="cuda")
+    act[:, :K_up] = torch.randn((B, K_up), device="cuda").to(act.dtype)
+    scratch = vc.gemv_scratch()
+    ybuf = torch.empty((B, up.N), dtype=torch.float32, device="cuda")
+    wbuf = next(t for t in dm.keep if t.data_ptr() == up.data)
+    for _ in range(5):
+        vc.debug_gemv(wbuf, cfg.wfmt, cfg.group_size, up.N, up.K, act, scratch, out=ybuf)
+    reps = 50
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    g0.record()
+    for _ in range(reps):
+        vc.debug_gemv(wbuf, cfg.wfmt, cfg.group_size, up.N, up.K, act, scratch, out=ybuf)
+    g1.record()
+    torch.cuda.synchronize()
+    gemv_ms = g0.elapsed_time(g1) / reps
+    gemv_bytes = matrix_bytes(cfg.wfmt, cfg.group_size, up.N, up.K) + B * K_up * 2 + B * up.N * 4
+    gemv_gbs = gemv_bytes / (gemv_ms / 1000.0) / 1e9
+
+    # ---- end to end through the C ABI with host buffers (pinned x in, tokens out, every step) ----
+    ne = max(1, e2e_steps)
+    xh = torch.empty((ne, B, cfg.d_model), dtype=torch.bfloat16).pin_memory()
+    for s in range(ne):
+        xh[s] = torch.from_numpy(synth.frame_inputs(cfg, seed + 1000 * rank, total + s, B)).view(torch.bfloat16)
+    th = torch.empty((B,), dtype=torch.int32).pin_memory()
+    fh = torch.empty((B,), dtype=torch.int32).pin_memory()
+    stream = torch.cuda.current_stream()
+    bb.step_host(xh[0], st, th, fh)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for s in range(1, ne):
+        bb.step_host(xh[s], st, th, fh)
+        stream.synchronize()   # the frame's tokens are on the host before the next frame
+    e2e_s = time.perf_counter() - t0
+    e2e_s = max_over_ranks(e2e_s, world)
+    e2e_value = world * B * (ne - 1) / e2e_s
+
+    cpu = None
+    if rank == 0 and world == 1 and cpu_baseline:
+        # a bounded sample: frame-steps from the same pre-filled state until 15 s of work, 64 at most
+        v, dt, n_or = oracle_run(cfg, 64, budget_s=15.0)
+        cpu = {"value": v, "unit": "frame-steps/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{n_or} frame-step(s) of the same workload (batch {B}) from the same pre-filled state, "
+                         f"{dt:.1f} s"}
+
+    gemv_line = {"kernel": "gemv (mlp up projection, streaming weights)", "achieved": gemv_gbs, "peak": peak,
+                 "peak_kind": peak_kind, "unit": "GB/s", "frac": gemv_gbs / peak, "launch_ms": gemv_ms,
+                 "bytes_per_launch": gemv_bytes}
+    if frame:
+        # the frame kernel is the whole step: one launch per frame, timed above on its stream
+        roofline = {"bound": "hbm", "kernel": "frame kernel (one launch per frame: all layers and both heads)",
+                    "achieved": step_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                    "frac": step_gbs / peak, "traffic": FRAME_TRAFFIC.get(cfg.name), "launch_ms": ms_step,
+                    "bytes_per_launch": rbytes}
+        launch = "frame kernel"
+        n_launches = steps
+    else:
+        roofline = dict(gemv_line, bound="hbm", traffic=TRAFFIC.get(cfg.name))
+        launch = "direct" if args.no_graph else "cuda graph"
+        n_launches = launches_per_step(cfg) * steps
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "frame-steps/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": {synth.FMT_BF16: "bf16", synth.FMT_W8: "w8-fp16", synth.FMT_W4: "w4-fp16",
+                      synth.FMT_W3: "w3-fp16"}[cfg.wfmt] + "-weights/fp32-accum",
+            "data": "synthetic (seeded N(0,0.02) weights, N(0,1) inputs and pre-filled state)",
+            "config": {"workload": cfg.name, "batch": B, "ctx_start": int(ctx0.max()) if B == 1 else
+                       [int(ctx0.min()), int(ctx0.max())], "layers": cfg.n_layers, "weights": synth.FMT_NAMES[cfg.wfmt],
+                       "group": cfg.group_size, "heads": synth.FMT_NAMES[cfg.head_fmt],
+                       "l2": f"no flush: {weight_total / 1e9:.2f} GB of weights per step >> 126 MB L2",
+                       "parallelism": f"replicas x{world}", "launch": launch},
+            "achieved_step_gbs": step_gbs, "step_bytes_read": rbytes, "step_bytes_written": wbytes,
+            "step_frac_of_peak": step_gbs / peak,
+            "roofline": roofline, "gemv_kernel_alone": gemv_line,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "frame-steps/s", "h2d_bytes_per_step": B * cfg.d_model * 2,
+                    "d2h_bytes_per_step": 2 * B * 4, "steps": ne - 1},
+            "gpu_launches": n_launches,
+            "clocks": clk, "device_status": status,
+        }
+    bb.close()
+    return line if rank == 0 else None
+
+
 # ------------------------------------------------------------------------------------------------
 # GPU arm
 # ------------------------------------------------------------------------------------------------
@@ -408,9 +568,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="nano_bf16", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="vc", choices=["vc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-second", action="store_true",
+                    help="default workload only: skip the second, bf16-weight measurement")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-graph", action="store_true",
                     help="per-kernel path: launch each step's kernels directly instead of replaying a CUDA graph "
@@ -442,156 +604,21 @@ def main():
         run_prefill_bench(args, cfg, world, rank, local)
         return
 
-    import attention_frame_decode_b200 as vc
-    from attention_frame_decode_b200.synthetic import build_model, fill_state
-
-    B = cfg.batch
-    seed = 0
-    dm = build_model(cfg, seed)
-    ctx0 = synth.context_lengths(cfg, seed, B)
-    total = args.warmup + args.steps
-    # the workload's cache capacity, grown when the run itself needs more frames than it holds
-    cap = max(cfg.kv_capacity, int(ctx0.max()) + total + args.e2e_steps + 8)
-    bb = dm.backbone(B, cap, B)
-    if args.no_graph:
-        bb.set_option(vc.OPT_GRAPH, 0)
-    if args.per_kernel:
-        bb.set_option(vc.OPT_FRAME, 0)
-    if args.frame:
-        bb.set_option(vc.OPT_FRAME, 1)
-    frame = bb.uses_frame_kernel(B)
-    st = dm.new_state(B, cap)
-    if cfg.random_state:
-        fill_state(st, cfg, seed + rank, ctx0, cap)
-    # every frame input of the run, resident in HBM before timing (rank r serves its own sessions)
-    xs = torch.empty((total, B, cfg.d_model), dtype=torch.bfloat16, device="cuda")
-    for s in range(total):
-        xs[s] = torch.from_numpy(synth.frame_inputs(cfg, seed + 1000 * rank, s, B)).view(torch.bfloat16)
-    tt = torch.zeros((B,), dtype=torch.int32, device="cuda")
-    tf = torch.zeros((B,), dtype=torch.int32, device="cuda")
-    if int(cap - ctx0.max()) < total + args.e2e_steps + 8:
-        raise SystemExit(f"kv capacity {cap} too small for {total + args.e2e_steps} steps")
-
-    for s in range(args.warmup):
-        bb.step(xs[s], st, tt, tf)
-    torch.cuda.synchronize()
-
-    clocks = ClockSampler(local)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for s in range(args.warmup, total):
-        bb.step(xs[s], st, tt, tf)
-    e1.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    ms = e0.elapsed_time(e1)
-    ms = max_over_ranks(ms, world)
-    status = int(st.status.cpu()[0])
-    ms_step = ms / args.steps
-    value = replica_rate(B * args.steps, world, ms / 1000.0)
-    ctx_mean = float(ctx0.mean()) + args.warmup + args.steps / 2.0
-    rbytes, wbytes, weight_total = step_bytes(cfg, B, ctx_mean)
-    step_gbs = rbytes / (ms_step / 1000.0) / 1e9
-
-    # ---- roofline of the dominant kernel: the streaming GEMV on the layer MLP up projection ----
-    peak, peak_kind = load_peaks()
-    mlp = cfg.pattern.index("-")
-    up = dm.layers[mlp].up
-    K_up = cfg.d_model
-    act_ld = (K_up + 127) // 128 * 128
-    act = torch.zeros((B, act_ld), dtype=torch.bfloat16 if cfg.wfmt == synth.FMT_BF16 else torch.float16,
-                      device="cuda")
-    act[:, :K_up] = torch.randn((B, K_up), device="cuda").to(act.dtype)
-    scratch = vc.gemv_scratch()
-    ybuf = torch.empty((B, up.N), dtype=torch.float32, device="cuda")
-    wbuf = next(t for t in dm.keep if t.data_ptr() == up.data)
-    for _ in range(5):
-        vc.debug_gemv(wbuf, cfg.wfmt, cfg.group_size, up.N, up.K, act, scratch, out=ybuf)
-    reps = 50
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    g0.record()
-    for _ in range(reps):
-        vc.debug_gemv(wbuf, cfg.wfmt, cfg.group_size, up.N, up.K, act, scratch, out=ybuf)
-    g1.record()
-    torch.cuda.synchronize()
-    gemv_ms = g0.elapsed_time(g1) / reps
-    gemv_bytes = matrix_bytes(cfg.wfmt, cfg.group_size, up.N, up.K) + B * K_up * 2 + B * up.N * 4
-    gemv_gbs = gemv_bytes / (gemv_ms / 1000.0) / 1e9
-
-    # ---- end to end through the C ABI with host buffers (pinned x in, tokens out, every step) ----
-    ne = max(1, args.e2e_steps)
-    xh = torch.empty((ne, B, cfg.d_model), dtype=torch.bfloat16).pin_memory()
-    for s in range(ne):
-        xh[s] = torch.from_numpy(synth.frame_inputs(cfg, seed + 1000 * rank, total + s, B)).view(torch.bfloat16)
-    th = torch.empty((B,), dtype=torch.int32).pin_memory()
-    fh = torch.empty((B,), dtype=torch.int32).pin_memory()
-    stream = torch.cuda.current_stream()
-    bb.step_host(xh[0], st, th, fh)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    t0 = time.perf_counter()
-    for s in range(1, ne):
-        bb.step_host(xh[s], st, th, fh)
-        stream.synchronize()   # the frame's tokens are on the host before the next frame
-    e2e_s = time.perf_counter() - t0
-    e2e_s = max_over_ranks(e2e_s, world)
-    e2e_value = world * B * (ne - 1) / e2e_s
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # a bounded sample: frame-steps from the same pre-filled state until 15 s of work, 64 at most
-        v, dt, n_or = oracle_run(cfg, 64, budget_s=15.0)
-        cpu = {"value": v, "unit": "frame-steps/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"{n_or} frame-step(s) of the same workload (batch {B}) from the same pre-filled state, "
-                         f"{dt:.1f} s"}
-
-    gemv_line = {"kernel": "gemv (mlp up projection, streaming weights)", "achieved": gemv_gbs, "peak": peak,
-                 "peak_kind": peak_kind, "unit": "GB/s", "frac": gemv_gbs / peak, "launch_ms": gemv_ms,
-                 "bytes_per_launch": gemv_bytes}
-    if frame:
-        # the frame kernel is the whole step: one launch per frame, timed above on its stream
-        roofline = {"bound": "hbm", "kernel": "frame kernel (one launch per frame: all layers and both heads)",
-                    "achieved": step_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                    "frac": step_gbs / peak, "traffic": FRAME_TRAFFIC.get(cfg.name), "launch_ms": ms_step,
-                    "bytes_per_launch": rbytes}
-        launch = "frame kernel"
-        n_launches = args.steps
-    else:
-        roofline = dict(gemv_line, bound="hbm", traffic=TRAFFIC.get(cfg.name))
-        launch = "direct" if args.no_graph else "cuda graph"
-        n_launches = launches_per_step(cfg) * args.steps
+    line = run_decode(args, cfg, world, rank, local, steps=args.steps, e2e_steps=args.e2e_steps,
+                      cpu_baseline=not args.no_cpu_baseline)
+    if cfg.name == DEFAULT_CONFIG and not args.no_second:
+        # the bf16-weight backbone (the pages' unquantized model) as a second, shorter measurement
+        torch.cuda.empty_cache()
+        second = run_decode(args, synth.CONFIGS["nano_bf16"], world, rank, local, steps=min(args.steps, 300),
+                            e2e_steps=min(args.e2e_steps, 20), cpu_baseline=False)
+        if rank == 0:
+            line["also"] = {"nano_bf16": {k: second[k] for k in ("value", "unit", "ms_per_step", "steps",
+                                                                  "achieved_step_gbs", "step_frac_of_peak",
+                                                                  "e2e", "clocks")}}
+            line["also"]["nano_bf16"]["roofline_frac"] = second["roofline"]["frac"]
+            line["gpu_launches"] += second["gpu_launches"]
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "frame-steps/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": {synth.FMT_BF16: "bf16", synth.FMT_W8: "w8-fp16", synth.FMT_W4: "w4-fp16",
-                      synth.FMT_W3: "w3-fp16"}[cfg.wfmt] + "-weights/fp32-accum",
-            "data": "synthetic (seeded N(0,0.02) weights, N(0,1) inputs and pre-filled state)",
-            "config": {"workload": cfg.name, "batch": B, "ctx_start": int(ctx0.max()) if B == 1 else
-                       [int(ctx0.min()), int(ctx0.max())], "layers": cfg.n_layers, "weights": synth.FMT_NAMES[cfg.wfmt],
-                       "group": cfg.group_size, "heads": synth.FMT_NAMES[cfg.head_fmt],
-                       "l2": f"no flush: {weight_total / 1e9:.2f} GB of weights per step >> 126 MB L2",
-                       "parallelism": f"replicas x{world}", "launch": launch},
-            "achieved_step_gbs": step_gbs, "step_bytes_read": rbytes, "step_bytes_written": wbytes,
-            "step_frac_of_peak": step_gbs / peak,
-            "roofline": roofline, "gemv_kernel_alone": gemv_line,
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "frame-steps/s", "h2d_bytes_per_step": B * cfg.d_model * 2,
-                    "d2h_bytes_per_step": 2 * B * 4, "steps": ne - 1},
-            "gpu_launches": n_launches,
-            "clocks": clk, "device_status": status,
-        }
         print(json.dumps(line), flush=True)
-    bb.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
