@@ -24,6 +24,7 @@ __host__ __device__ constexpr int warps_for(int) { return 8; }
 // start their weight copies while this kernel drains; one CTA for 9..16 rows
 __host__ __device__ constexpr int ctas_per_sm(int NT) { return NT == 1 ? 2 : 1; }
 static constexpr int kRingBudget = 210 * 1024; // dynamic shared memory for the rings of one CTA
+static constexpr int kMaxDynSmem = 220 * 1024;  // dynamic shared memory of one CTA, at most
 
 // ------------------------------------------------------------------------------------------
 // the kernel
@@ -43,6 +44,7 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
     constexpr int R = L.R, KS = L.KS;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t bars[WARPS][kMaxSlots];
+    __shared__ uint64_t act_bar;   // the staged activation rows (act_smem)
     __shared__ float insc_tab[kMaxB * 16];
 
     pdl_trigger();
@@ -90,6 +92,7 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
 
     if (lane == 0) {
         for (int s = 0; s < rg_slots; ++s) mbar_init(&bar[s], 1);
+        if (warp == 0) mbar_init(&act_bar, 1);
         fence_mbar_init();
         for (int i = 0; i < nstages && i < rg_slots; ++i) issue_weights(i, i);
     }
@@ -111,15 +114,17 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
         }
         if (lane == 0) insc_tab[idx] = v;
     }
+    // the activation rows to shared memory, one bulk copy per row (rows padded by 16 bytes)
     uint8_t* act_s = smem + (size_t)WARPS * rg_slots * rg_slot_bytes;
-    if (rg_act_smem) {
-        const int row16 = args.act_ld / 8;   // 16-byte chunks per row
-        for (int idx = threadIdx.x; idx < B * row16; idx += WARPS * 32) {
-            const int b = idx / row16, c = idx % row16;
-            *reinterpret_cast<uint4*>(act_s + (size_t)b * rg_act_stride + c * 16) =
-                *reinterpret_cast<const uint4*>(args.act + (size_t)b * args.act_ld + (size_t)c * 8);
-        }
+    __syncthreads();   // act_bar initialised
+    if (rg_act_smem && threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&act_bar, (uint32_t)(B * args.act_ld * 2));
+        for (int b = 0; b < B; ++b)
+            bulk_g2s(act_s + (size_t)b * rg_act_stride, args.act + (size_t)b * args.act_ld, (uint32_t)(args.act_ld * 2),
+                     &act_bar);
     }
+    bool act_ok = true;
+    if (rg_act_smem) act_ok = mbar_wait(&act_bar, 0, args.status);
     __syncthreads();
 
     if (lane == 0 && !rg_act_smem)
@@ -140,7 +145,7 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
     };
 
     zero_acc();
-    bool alive = true;
+    bool alive = act_ok;
     int cur_u = f0 / KT, kt = f0 % KT;   // unit and k-step of the next block to consume
     bool pending = false;                 // acc holds contributions of cur_u not yet flushed
     int slot = 0;
@@ -204,18 +209,22 @@ cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
     rg.act_row = L.KS * 2 + 16;
     rg.act_stride = a.act_ld * 2 + 16;
     const int act_total = a.B * rg.act_stride;
-    rg.act_smem = act_total <= 32 * 1024;
     const int wbytes = L.bps * L.block_bytes;
+    constexpr int WARPS = warps_for(NT);
+    // the whole activation goes to shared memory once per CTA when it fits beside rings of two
+    // weight-only slots per warp (one CTA per SM for 9..16 rows leaves room for ~140 KB of
+    // activations: 16 rows of K = 4480); otherwise each block's activation slice rides in the ring
+    const int act_room = NT == 1 ? 32 * 1024 : kMaxDynSmem - WARPS * 2 * round_up(wbytes, 128);
+    rg.act_smem = act_total <= act_room;
     rg.slot_bytes = round_up(wbytes + (rg.act_smem ? 0 : L.bps * a.B * rg.act_row), 128);
     // as many 4 KB-class slots per warp as the budget allows: the bytes in flight per SM
     // (warps x (slots - 1) x slot) must cover HBM latency x per-SM bandwidth (~60-100 KB)
-    constexpr int WARPS = warps_for(NT);
     const int budget = kRingBudget / ctas_per_sm(NT) - 4096;   // two CTAs must fit one SM
     rg.slots = (budget - (rg.act_smem ? act_total : 0)) / (WARPS * rg.slot_bytes);
     if (rg.slots > kMaxSlots) rg.slots = kMaxSlots;
     if (rg.slots < 2) rg.slots = 2;
     const size_t smem = (size_t)WARPS * rg.slots * rg.slot_bytes + (rg.act_smem ? act_total : 0);
-    if (smem > 220 * 1024) return cudaErrorInvalidValue;
+    if (smem > kMaxDynSmem) return cudaErrorInvalidValue;
     auto kern = gemv_kernel<FMT, GRP, NT, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

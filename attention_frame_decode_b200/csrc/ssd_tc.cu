@@ -396,14 +396,16 @@ cudaError_t launch_ssd_out_tc(const uint16_t* xc16, const uint16_t* sin16, const
 //   A = B_g^T: 128-byte swizzle, two 64-wide n blocks;  B = (w x_h): 32-byte swizzle, P/16 blocks.
 // The state that decode continues from must meet the fp32 bound, so each operand is split into
 // two fp16 halves (v = hi + lo, lo = v - hi) and the product is hi.hi + hi.lo + lo.hi (the dropped
-// lo.lo term is ~2^-22 of the product), accumulated in fp32 in TMEM.  CTA = (chunk, head), frames
+// lo.lo term is ~2^-22 of the product), accumulated in fp32 in TMEM: the hi.hi products in one
+// accumulator and the two correction products, ~2^-11 smaller, in a second one, added in fp32 at
+// the end, so that the corrections are not rounded against the much larger main sums.  CTA = (chunk, head), frames
 // in slabs of 64 staged by the threads (the split needs the fp32 values); a few CTAs per SM
 // overlap one CTA's staging with another's MMAs.  The within-chunk cumulative log decay is
 // scanned in double precision (one warp), as the decay weights come from its differences.
 // ------------------------------------------------------------------------------------------
 static constexpr int kStSlab = 64;
 static constexpr int kStThreads = 256;
-static constexpr uint32_t kStTmemCols = 128;
+static constexpr uint32_t kStTmemCols = 256;   // hi.hi sums in [0, P), hi.lo + lo.hi sums in [128, 128 + P)
 
 struct SsdStPlan {
     uint32_t off_ah, off_al, off_xh, off_xl, total;
@@ -567,8 +569,8 @@ __global__ void __launch_bounds__(kStThreads) pf_ssd_state_tc_kernel(const float
                 const uint64_t dbh = umma_desc(bh + k * 512, 2048, 256, UMMA_SW32);
                 const uint64_t dbl = umma_desc(bl + k * 512, 2048, 256, UMMA_SW32);
                 tc_mma(tmem, dah, dbh, idesc, (sl | k) != 0);
-                tc_mma(tmem, dah, dbl, idesc, 1);
-                tc_mma(tmem, dal, dbh, idesc, 1);
+                tc_mma(tmem + 128, dah, dbl, idesc, (sl | k) != 0);
+                tc_mma(tmem + 128, dal, dbh, idesc, 1);
             }
             tc_commit(&bar_mma);
         }
@@ -582,10 +584,10 @@ __global__ void __launch_bounds__(kStThreads) pf_ssd_state_tc_kernel(const float
         const int qa = warp < 4 ? 0 : qh, qb = warp < 4 ? qh : PA;
         float* S = schunk + ((size_t)c * H + h) * P * N;
         for (int q = qa; q < qb; ++q) {
-            float v[16];
-            tc_ld16(tmem + ((uint32_t)lb << 16) + 16 * q, v);
+            float v[16], cr[16];
+            tc_ld16x2(tmem + ((uint32_t)lb << 16) + 16 * q, tmem + ((uint32_t)lb << 16) + 128 + 16 * q, v, cr);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) S[(size_t)(16 * q + e) * N + n] = v[e];
+            for (int e = 0; e < 16; ++e) S[(size_t)(16 * q + e) * N + n] = v[e] + cr[e];
         }
     }
     tc_fence_before();
