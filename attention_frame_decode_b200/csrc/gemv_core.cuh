@@ -418,6 +418,28 @@ __device__ __forceinline__ void consume_block(const uint8_t* blk, ActRow arow, i
     consume_block_bv<FMT, GRP, NT>(blk, bv, lane, sc, acc, B > 1, SYM);
 }
 
+// the same with the k-step's activation staged as SUB boxes (box st at box0 + st * box_bytes) of
+// B rows x 64 columns, 128 B per row with the 128-byte swizzle: 16-byte chunk c of row b sits at
+// chunk c ^ (b & 7)
+template <int FMT, int GRP, int NT, bool SYM = false>
+__device__ __forceinline__ void consume_block_swz(const uint8_t* blk, const uint8_t* box0, int box_bytes, int B, int lane,
+                                                  const float (&sc)[NT][2],
+                                                  float (&acc)[layout_info(FMT, GRP).R][NT][4]) {
+    constexpr int SUB = layout_info(FMT, GRP).SUB;
+    const int g = lane >> 2, t = lane & 3;
+    uint4 bv[SUB][NT][2];
+#pragma unroll
+    for (int st = 0; st < SUB; ++st)
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            const int b = min(8 * j + g, B - 1);
+            const uint8_t* row = box0 + st * box_bytes + b * 128;
+            bv[st][j][0] = *reinterpret_cast<const uint4*>(row + (((2 * t) ^ (b & 7)) << 4));
+            bv[st][j][1] = *reinterpret_cast<const uint4*>(row + (((2 * t + 1) ^ (b & 7)) << 4));
+        }
+    consume_block_bv<FMT, GRP, NT>(blk, bv, lane, sc, acc, B > 1, SYM);
+}
+
 // ------------------------------------------------------------------------------------------
 // epilogue of a finished unit u (values v) of matrix wr.m of the launch
 // ------------------------------------------------------------------------------------------

@@ -14,6 +14,7 @@
 //     building blocks of gemv_core.cuh.
 #pragma once
 #include "gemv_core.cuh"
+#include "tc.cuh"
 
 namespace vc {
 
@@ -31,18 +32,25 @@ static constexpr int kMaxDynSmem = 220 * 1024;  // dynamic shared memory of one 
 // ------------------------------------------------------------------------------------------
 struct RingGeom {
     int slots;        // ring slots per warp
-    int slot_bytes;   // weights (bps blocks) [+ activation rows when act_smem == 0]
-    int act_row;      // bytes per staged activation row (KS*2 + 16)
+    int slot_bytes;   // weights (bps blocks) [+ activation slices when act_smem == 0]
+    int act_row;      // bytes per staged activation row (KS*2 + 16), act_tma == 0
     int act_smem;     // 1: the whole activation [B][act_ld] is copied to shared memory once per CTA
     int act_stride;   // bytes per activation row in shared memory (act_ld*2 + 16)
+    int act_tma;      // 1: each block's activation slice is one tensor copy per 64 columns (B rows x
+                      // 128 B, 128-byte swizzle) into a 1 KB-aligned region of the slot
+    int act_off;      // byte offset of the activation slices in a slot
+    int act_box;      // bytes per 64-column box region (B x 128 rounded up to 1 KB)
 };
 
 template <int FMT, int GRP, int NT, int EPI>
-__global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kernel(const GemvArgs args, const RingGeom rg) {
+__global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT))
+    gemv_kernel(const GemvArgs args, const RingGeom rg, const __grid_constant__ CUtensorMap act_map) {
     constexpr int WARPS = warps_for(NT);
     constexpr LayoutInfo L = layout_info(FMT, GRP);
-    constexpr int R = L.R, KS = L.KS;
-    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int R = L.R, KS = L.KS, SUB = L.SUB;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    // 1 KB alignment: the swizzled activation boxes' pattern repeats every 1 KB
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t bars[WARPS][kMaxSlots];
     __shared__ uint64_t act_bar;   // the staged activation rows (act_smem)
     __shared__ float insc_tab[kMaxB * 16];
@@ -54,7 +62,8 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
     const int B = args.B;
     // the ring geometry in registers (read once from the parameter space)
     const int rg_slots = rg.slots, rg_slot_bytes = rg.slot_bytes, rg_act_row = rg.act_row, rg_act_stride = rg.act_stride;
-    const bool rg_act_smem = rg.act_smem != 0;
+    const bool rg_act_smem = rg.act_smem != 0, rg_act_tma = rg.act_tma != 0;
+    const int rg_act_off = rg.act_off, rg_act_box = rg.act_box;
 
     // ---- worker range -------------------------------------------------------------------
     const long long Wall = (long long)gridDim.x * WARPS;
@@ -74,18 +83,23 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
         const int fb = f0 + i * bps;
         const int nb = min(bps, f1 - fb);
         const uint32_t wbytes = nb * L.block_bytes;
-        const uint32_t abytes = rg_act_smem ? 0u : (uint32_t)(nb * act_rows * KS * 2);
+        const uint32_t abytes = rg_act_smem ? 0u : (uint32_t)(nb * act_rows * KS * 2);   // the same for both forms
         mbar_arrive_expect_tx(&bar[slot], wbytes + abytes);
         bulk_g2s(ring + (size_t)slot * rg_slot_bytes, M.w + (size_t)fb * L.block_bytes, wbytes, &bar[slot]);
     };
     int act_kt = f0 % KT;   // k-step of the next block whose activation slice is issued
     auto issue_act = [&](int i, int slot) {
         const int nb = min(bps, f1 - (f0 + i * bps));
-        uint8_t* abase = ring + (size_t)slot * rg_slot_bytes + bps * L.block_bytes;
+        uint8_t* abase = ring + (size_t)slot * rg_slot_bytes + rg_act_off;
         for (int j = 0; j < nb; ++j) {
-            for (int b = 0; b < act_rows; ++b)
-                bulk_g2s(abase + (j * act_rows + b) * rg_act_row,
-                         args.act + (size_t)b * args.act_ld + (size_t)act_kt * KS, KS * 2, &bar[slot]);
+            if (rg_act_tma) {
+                for (int st = 0; st < SUB; ++st)
+                    tma_load_2d(abase + (j * SUB + st) * rg_act_box, &act_map, act_kt * KS + 64 * st, 0, &bar[slot]);
+            } else {
+                for (int b = 0; b < act_rows; ++b)
+                    bulk_g2s(abase + (j * act_rows + b) * rg_act_row,
+                             args.act + (size_t)b * args.act_ld + (size_t)act_kt * KS, KS * 2, &bar[slot]);
+            }
             if (++act_kt == KT) act_kt = 0;
         }
     };
@@ -114,17 +128,27 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
         }
         if (lane == 0) insc_tab[idx] = v;
     }
-    // the activation rows to shared memory, one bulk copy per row (rows padded by 16 bytes)
+    // the activation rows to shared memory (rows padded by 16 bytes): up to 32 KB by the threads'
+    // own loads (they overlap the weight copies already queued on the copy engine); beyond that
+    // one bulk copy per row
     uint8_t* act_s = smem + (size_t)WARPS * rg_slots * rg_slot_bytes;
+    const bool act_bulk = rg_act_smem && B * args.act_ld * 2 > 32 * 1024;
     __syncthreads();   // act_bar initialised
-    if (rg_act_smem && threadIdx.x == 0) {
+    if (act_bulk && threadIdx.x == 0) {
         mbar_arrive_expect_tx(&act_bar, (uint32_t)(B * args.act_ld * 2));
         for (int b = 0; b < B; ++b)
             bulk_g2s(act_s + (size_t)b * rg_act_stride, args.act + (size_t)b * args.act_ld, (uint32_t)(args.act_ld * 2),
                      &act_bar);
+    } else if (rg_act_smem) {
+        const int row16 = args.act_ld / 8;   // 16-byte chunks per row
+        for (int idx = threadIdx.x; idx < B * row16; idx += WARPS * 32) {
+            const int b = idx / row16, c = idx % row16;
+            *reinterpret_cast<uint4*>(act_s + (size_t)b * rg_act_stride + c * 16) =
+                *reinterpret_cast<const uint4*>(args.act + (size_t)b * args.act_ld + (size_t)c * 8);
+        }
     }
     bool act_ok = true;
-    if (rg_act_smem) act_ok = mbar_wait(&act_bar, 0, args.status);
+    if (act_bulk) act_ok = mbar_wait(&act_bar, 0, args.status);
     __syncthreads();
 
     if (lane == 0 && !rg_act_smem)
@@ -158,7 +182,7 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
         const int nb = min(bps, f1 - (f0 + i * bps));
         for (int jb = 0; jb < nb; ++jb) {
             const uint8_t* blk = base + jb * L.block_bytes;
-            const uint8_t* arow0 = base + bps * L.block_bytes + (size_t)jb * act_rows * rg_act_row;
+            const uint8_t* arow0 = base + rg_act_off + (size_t)jb * (rg_act_tma ? SUB * rg_act_box : act_rows * rg_act_row);
             // input scales of this k-step (norm group qg) for the lane's batch columns
             if (kt == sc_next) {
                 const int qg = ng > 1 ? (kt * KS) / args.insc.group_cols : 0;
@@ -175,6 +199,8 @@ __global__ void __launch_bounds__(warps_for(NT) * 32, ctas_per_sm(NT)) gemv_kern
                 const uint8_t* abase = act_s + (size_t)kt * KS * 2;
                 consume_block<FMT, GRP, NT, EPI == EPI_ARGMAX>(blk, [&](int b) { return abase + (size_t)b * rg_act_stride; }, B,
                                                               lane, sc, acc);
+            } else if (rg_act_tma) {
+                consume_block_swz<FMT, GRP, NT, EPI == EPI_ARGMAX>(blk, arow0, rg_act_box, B, lane, sc, acc);
             } else {
                 consume_block<FMT, GRP, NT, EPI == EPI_ARGMAX>(blk, [&](int b) { return arow0 + b * rg_act_row; }, B, lane,
                                                               sc, acc);
@@ -206,6 +232,8 @@ template <int FMT, int GRP, int NT, int EPI>
 cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
     constexpr LayoutInfo L = layout_info(FMT, GRP);
     RingGeom rg{};
+    CUtensorMap act_map;
+    memset(&act_map, 0, sizeof(act_map));
     rg.act_row = L.KS * 2 + 16;
     rg.act_stride = a.act_ld * 2 + 16;
     const int act_total = a.B * rg.act_stride;
@@ -216,15 +244,27 @@ cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
     // activations: 16 rows of K = 4480); otherwise each block's activation slice rides in the ring
     const int act_room = NT == 1 ? 32 * 1024 : kMaxDynSmem - WARPS * 2 * round_up(wbytes, 128);
     rg.act_smem = act_total <= act_room;
-    rg.slot_bytes = round_up(wbytes + (rg.act_smem ? 0 : L.bps * a.B * rg.act_row), 128);
+    // otherwise, for 9..16 rows (one CTA per SM, room for 1 KB-aligned slices), each block's slice
+    // is one tensor copy per 64 columns instead of a copy per row (rows keep the per-row copies,
+    // as does any shape whose tensor map cannot be made)
+    rg.act_tma = NT == 2 && !rg.act_smem &&
+                 tma_map_2d(&act_map, a.act, a.B, a.act_ld, a.act_ld, 64, a.B, act_f16_for(FMT), CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rg.act_tma) {
+        rg.act_box = round_up(a.B * 128, 1024);
+        rg.act_off = round_up(wbytes, 1024);
+        rg.slot_bytes = round_up(rg.act_off + L.bps * L.SUB * rg.act_box, 1024);
+    } else {
+        rg.act_off = wbytes;
+        rg.slot_bytes = round_up(wbytes + (rg.act_smem ? 0 : L.bps * a.B * rg.act_row), 128);
+    }
     // as many 4 KB-class slots per warp as the budget allows: the bytes in flight per SM
     // (warps x (slots - 1) x slot) must cover HBM latency x per-SM bandwidth (~60-100 KB)
     const int budget = kRingBudget / ctas_per_sm(NT) - 4096;   // two CTAs must fit one SM
     rg.slots = (budget - (rg.act_smem ? act_total : 0)) / (WARPS * rg.slot_bytes);
     if (rg.slots > kMaxSlots) rg.slots = kMaxSlots;
     if (rg.slots < 2) rg.slots = 2;
-    const size_t smem = (size_t)WARPS * rg.slots * rg.slot_bytes + (rg.act_smem ? act_total : 0);
-    if (smem > kMaxDynSmem) return cudaErrorInvalidValue;
+    const size_t smem = (size_t)WARPS * rg.slots * rg.slot_bytes + (rg.act_smem ? act_total : 0) + 1024;   // + alignment
+    if (smem > kMaxDynSmem + 1024) return cudaErrorInvalidValue;
     auto kern = gemv_kernel<FMT, GRP, NT, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -238,7 +278,7 @@ cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = Lh.pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a, rg);
+    return cudaLaunchKernelEx(&cfg, kern, a, rg, act_map);
 }
 
 template <int FMT, int GRP, int NT>
