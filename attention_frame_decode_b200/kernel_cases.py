@@ -90,6 +90,34 @@ def case_ssd(a):
     print(f"prefill mixer (conv + chunked SSD + gated norm), Nano widths, T={T}: {us:.1f} us/call")
 
 
+def case_mamba(a):
+    """decode frames of one Nano Mamba-2 layer (W8 g128 projections) for `batch` sessions with
+    random state, launched kernel by kernel: its Mamba-2 step is the kernel of interest"""
+    import numpy as np
+    import torch
+    import attention_frame_decode_b200 as vc
+    import synth
+    from attention_frame_decode_b200.synthetic import build_model, fill_state
+    B = a.batch
+    cfg = synth.nano_config(name="nano_mamba_layer", pattern="M", wfmt=synth.FMT_W8, group_size=128,
+                            vocab_text=4096, vocab_func=2048)
+    dm = build_model(cfg, 0)
+    cap = 64
+    bb = dm.backbone(B, cap, B)
+    bb.set_option(vc.OPT_GRAPH, 0)
+    st = dm.new_state(B, cap)
+    fill_state(st, cfg, 0, np.full(B, 8), cap)
+    tt = torch.zeros((B,), dtype=torch.int32, device="cuda")
+    tf = torch.zeros_like(tt)
+    x = torch.from_numpy(synth.frame_inputs(cfg, 0, 0, B)).cuda().view(torch.bfloat16)
+    run = lambda: bb.step(x, st, tt, tf)
+    for _ in range(a.warmup):
+        run()
+    us = _time(run, a.reps)
+    print(f"one Nano Mamba-2 layer + heads, {B} sessions: {us:.1f} us/step, status {int(st.status.cpu()[0])}")
+    bb.close()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     sub = ap.add_subparsers(dest="case", required=True)
@@ -105,11 +133,13 @@ def main(argv=None):
     m.add_argument("--k", type=int, default=4480)
     s = sub.add_parser("ssd")
     s.add_argument("--frames", type=int, default=1024)
-    for p in (g, m, s):
+    mb = sub.add_parser("mamba")
+    mb.add_argument("--batch", type=int, default=16)
+    for p in (g, m, s, mb):
         p.add_argument("--warmup", type=int, default=3)
         p.add_argument("--reps", type=int, default=20)
     a = ap.parse_args(argv)
-    {"gemv": case_gemv, "gemm": case_gemm, "ssd": case_ssd}[a.case](a)
+    {"gemv": case_gemv, "gemm": case_gemm, "ssd": case_ssd, "mamba": case_mamba}[a.case](a)
 
 
 if __name__ == "__main__":
