@@ -94,6 +94,7 @@ __device__ __forceinline__ MambaTile mamba_tile(uint8_t* base, int Ph, int N) {
 __host__ __device__ constexpr size_t mamba_tile_bytes(int Ph, int N) {
     return ((size_t)(Ph * N + 2 * Ph + 2 * N) * 4 + 127) / 128 * 128;
 }
+// (with P/2 a multiple of 2, the B and C rows of a tile start on 16-byte boundaries)
 
 // one item's inputs for the thread's channels tid and tid + kMambaThreads (x half, then the
 // group's B, then C): the conv sum over the W-1 ring rows before this frame, the last tap's
@@ -247,14 +248,27 @@ __global__ void __launch_bounds__(kMambaThreads, kMambaCtasPerSm) mamba_step_ker
             float y = 0.0f;
             const float* Srow = T.S + pr * N;
             float* Sgrow = Sg + (size_t)pr * N;
+            if constexpr (N_ == 128) {   // four consecutive states per lane: 16-byte accesses
+                const float4 s4 = *reinterpret_cast<const float4*>(Srow + 4 * lane);
+                const float4 b4 = *reinterpret_cast<const float4*>(T.Bs + 4 * lane);
+                const float4 c4 = *reinterpret_cast<const float4*>(T.Cs + 4 * lane);
+                float4 n4;
+                n4.x = fmaf(decay, s4.x, dx * b4.x);
+                n4.y = fmaf(decay, s4.y, dx * b4.y);
+                n4.z = fmaf(decay, s4.z, dx * b4.z);
+                n4.w = fmaf(decay, s4.w, dx * b4.w);
+                if (okb) *reinterpret_cast<float4*>(Sgrow + 4 * lane) = n4;
+                y = fmaf(c4.x, n4.x, fmaf(c4.y, n4.y, fmaf(c4.z, n4.z, c4.w * n4.w)));
+            } else {
 #pragma unroll
-            for (int n0 = 0; n0 < (N_ ? N_ : 256); n0 += 32) {
-                if (!N_ && n0 >= N) break;
-                const int n = n0 + lane;
-                if (!N_ && n >= N) break;
-                const float sn = fmaf(decay, Srow[n], dx * T.Bs[n]);
-                if (okb) Sgrow[n] = sn;
-                y = fmaf(T.Cs[n], sn, y);
+                for (int n0 = 0; n0 < (N_ ? N_ : 256); n0 += 32) {
+                    if (!N_ && n0 >= N) break;
+                    const int n = n0 + lane;
+                    if (!N_ && n >= N) break;
+                    const float sn = fmaf(decay, Srow[n], dx * T.Bs[n]);
+                    if (okb) Sgrow[n] = sn;
+                    y = fmaf(T.Cs[n], sn, y);
+                }
             }
             y = warp_sum(y);
             if (lane == 0) {

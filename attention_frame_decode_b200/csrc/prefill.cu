@@ -413,6 +413,7 @@ __global__ void pf_ssd_scan_kernel(const float* schunk, const float* lam, int T,
 // and keeps v in registers between the two passes.
 static constexpr int kGnMaxPerLane = 64;   // vector path: group size up to 32 x 64 columns
 
+template <int STEPS>   // 128-column steps per group when fixed at compile time (the backbone's 10), else 0
 __global__ void pf_gated_norm_kernel(const float* __restrict__ y, const uint16_t* __restrict__ zx, int zxw,
                                      const float* __restrict__ gnorm, int E, int NG, float eps,
                                      uint16_t* __restrict__ act, int ld, int f16) {
@@ -422,10 +423,11 @@ __global__ void pf_gated_norm_kernel(const float* __restrict__ y, const uint16_t
     const float* yr = y + (size_t)t * E;
     const uint16_t* zr = zx + (size_t)t * zxw;
     uint16_t* ar = act + (size_t)t * ld;
-    const bool vec = (gs & 127) == 0 && gs / 32 <= kGnMaxPerLane && (zxw & 3) == 0 && (ld & 3) == 0 && (E & 3) == 0;
+    const bool vec = STEPS ? true
+                           : (gs & 127) == 0 && gs / 32 <= kGnMaxPerLane && (zxw & 3) == 0 && (ld & 3) == 0 && (E & 3) == 0;
     if (vec) {
         float v[kGnMaxPerLane];
-        const int steps = gs / 128;
+        const int steps = STEPS ? STEPS : gs / 128;
         float ss = 0.0f;
 #pragma unroll
         for (int k = 0; k < kGnMaxPerLane / 4; ++k) {
@@ -599,8 +601,14 @@ cudaError_t prefill_mixer(const PfMixer& m, cudaStream_t s) {
         pf_ssd_out_mma_kernel<<<dim3(nch, m.G, kChunk / kSsdTi), 256, SL.total, s>>>(m.xc, m.xc16, m.dt, m.lam, m.sin16,
                                                                                      Lw.D, T, H, P, N, m.G, E, Cx, m.y);
     }
-    pf_gated_norm_kernel<<<T, 32 * m.NG, 0, s>>>(m.y, m.zx, zxw, Lw.gnorm, E, m.NG, m.eps, m.act, m.act_ld,
-                                                       m.f16);
+    // groups of 1280 columns (the backbone's) with aligned rows: the fixed-step instance, whose
+    // ten 16-byte loads per lane are all issued before the first is used
+    if (E / m.NG == 1280 && E % m.NG == 0 && zxw % 4 == 0 && m.act_ld % 4 == 0 && E % 4 == 0)
+        pf_gated_norm_kernel<10><<<T, 32 * m.NG, 0, s>>>(m.y, m.zx, zxw, Lw.gnorm, E, m.NG, m.eps, m.act, m.act_ld,
+                                                         m.f16);
+    else
+        pf_gated_norm_kernel<0><<<T, 32 * m.NG, 0, s>>>(m.y, m.zx, zxw, Lw.gnorm, E, m.NG, m.eps, m.act, m.act_ld,
+                                                        m.f16);
     return cudaGetLastError();
 }
 

@@ -59,13 +59,15 @@ def teacher_forced_check(run, x, ctx, hid, lg, zx):
                 assert np.array_equal(ring[b, int(ctx[b]) % W].astype(np.float64), zb[b, E:E + Cx]), (l, b)
             mi += 1
     run.ost.ctx_len[:B] += 1
-    # the appended K/V rows against the teacher-forced oracle's
+    # the appended K/V rows against the teacher-forced oracle's: both sides store bf16, so one
+    # rounding may go the other way (one bf16 ulp of the value) before the RMS bound applies
+    from tests.test_gpu_prefill import rel_stored
     k = run.st.k.float().cpu().numpy()
     v = run.st.v.float().cpu().numpy()
     for b in range(B):
         c = int(ctx[b])
-        assert rel(k[:, b, :, c], run.ost.k[:, b, :, c]) <= HID_TOL
-        assert rel(v[:, b, :, c], run.ost.v[:, b, :, c]) <= HID_TOL
+        assert rel_stored(k[:, b, :, c], run.ost.k[:, b, :, c]) <= HID_TOL, (b, rel(k[:, b, :, c], run.ost.k[:, b, :, c]))
+        assert rel_stored(v[:, b, :, c], run.ost.v[:, b, :, c]) <= HID_TOL, (b, rel(v[:, b, :, c], run.ost.v[:, b, :, c]))
     # heads from the GPU's final residual
     rh = run.om.heads(hid[cfg.n_layers].astype(np.float64), oracle.MIRROR)
     compared = 0
