@@ -20,7 +20,7 @@ _lib = C.CDLL(LIB_PATH)
 VC_OK, VC_ERR_INVALID_ARG, VC_ERR_UNSUPPORTED, VC_ERR_CUDA, VC_ERR_CAPACITY, VC_ERR_STATE = range(6)
 VC_DEV_CAPACITY, VC_DEV_NONFINITE, VC_DEV_TIMEOUT = 1, 2, 4
 W_BF16, W_INT8_SYM, W_INT4_ASYM, W_INT3_ASYM = 0, 1, 2, 3
-OPT_GRAPH, OPT_PDL, OPT_FRAME = 1, 2, 3
+OPT_GRAPH, OPT_PDL, OPT_FRAME, OPT_GEMV_SHAPE = 1, 2, 3, 4
 
 
 class VcConfig(C.Structure):

@@ -141,6 +141,7 @@ struct vc_backbone {
     Workspace ws;
     int num_sms = 148;
     int use_graph = 1, use_pdl = 1, use_frame = 0;
+    int gemv_shape = 0;   // VC_OPT_GEMV_SHAPE
     // the frame kernel's program as last uploaded, and the call signature it was built for
     std::unique_ptr<FrameProgram> host_prog;
     GraphKey prog_key;
@@ -363,6 +364,7 @@ extern "C" vc_status vc_set_option(vc_backbone* h, int option, int value) {
     if (option == VC_OPT_GRAPH) h->use_graph = value != 0;
     else if (option == VC_OPT_PDL) h->use_pdl = value != 0;
     else if (option == VC_OPT_FRAME) h->use_frame = value != 0;
+    else if (option == VC_OPT_GEMV_SHAPE && value >= 0 && value <= 2) h->gemv_shape = value;
     else return VC_ERR_INVALID_ARG;
     clear_graphs(h);
     h->prog_valid = false;
@@ -493,7 +495,7 @@ static cudaError_t record_step(vc_backbone* h, const void* x, int B, const int32
     base.status = st->status;
     base.slots = slots; base.ok = W.ok; base.ctx_len = st->ctx_len;
     GemvLaunch gl{};
-    gl.fmt = fmt; gl.group = grp; gl.num_sms = h->num_sms; gl.pdl = h->use_pdl;
+    gl.fmt = fmt; gl.group = grp; gl.num_sms = h->num_sms; gl.pdl = h->use_pdl; gl.shape = h->gemv_shape;
 
     auto resid_epi = [&](GemvArgs& a, int l) {
         a.resid = W.r; a.resid_ld = D.d;

@@ -73,6 +73,9 @@ struct GemvLaunch {
     int fmt, group, epi;
     int num_sms;
     int pdl;
+    // up to 8 rows: 0 = two CTAs per SM, each with half the ring budget; 1 = one CTA per SM with
+    // half the budget (the next launch's CTA fits beside it); 2 = one CTA per SM, whole budget
+    int shape;
 };
 
 // size in bytes of the scratch partial buffer and counters needed by any launch on num_sms SMs

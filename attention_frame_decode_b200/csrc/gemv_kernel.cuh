@@ -13,6 +13,8 @@
 //   * dequantization, tensor-core products and the fused epilogues are the shared per-warp
 //     building blocks of gemv_core.cuh.
 #pragma once
+#include <atomic>
+
 #include "gemv_core.cuh"
 #include "tc.cuh"
 
@@ -257,9 +259,15 @@ cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
         rg.act_off = wbytes;
         rg.slot_bytes = round_up(wbytes + (rg.act_smem ? 0 : L.bps * a.B * rg.act_row), 128);
     }
+    // CTAs per SM and the ring budget of each (GemvLaunch::shape, up to 8 rows): two CTAs with
+    // half the budget each; one CTA with half the budget, leaving room for a CTA of the next
+    // launch; one CTA with the whole budget
+    const int shape = NT == 1 ? Lh.shape : 0;
+    const int cps = shape ? 1 : ctas_per_sm(NT);
+    const int share = shape == 2 ? 1 : ctas_per_sm(NT);
     // as many 4 KB-class slots per warp as the budget allows: the bytes in flight per SM
     // (warps x (slots - 1) x slot) must cover HBM latency x per-SM bandwidth (~60-100 KB)
-    const int budget = kRingBudget / ctas_per_sm(NT) - 4096;   // two CTAs must fit one SM
+    const int budget = kRingBudget / share - 4096;   // `share` CTAs must fit one SM
     rg.slots = (budget - (rg.act_smem ? act_total : 0)) / (WARPS * rg.slot_bytes);
     if (rg.slots > kMaxSlots) rg.slots = kMaxSlots;
     if (rg.slots < 2) rg.slots = 2;
@@ -267,9 +275,17 @@ cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
     if (smem > kMaxDynSmem + 1024) return cudaErrorInvalidValue;
     auto kern = gemv_kernel<FMT, GRP, NT, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // shape 1: the largest shared-memory carveout, so that a CTA of the next launch can fit beside
+    // this one; the preference stays with the kernel, so once shape 1 has been used in the process
+    // the other shapes set it back to the driver's choice (untouched otherwise)
+    static std::atomic<bool> carveout_set{false};
+    if (shape == 1) carveout_set.store(true);
+    if (e == cudaSuccess && carveout_set.load())
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 shape == 1 ? 100 : (int)cudaSharedmemCarveoutDefault);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(Lh.num_sms * ctas_per_sm(NT));
+    cfg.gridDim = dim3(Lh.num_sms * cps);
     cfg.blockDim = dim3(WARPS * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;

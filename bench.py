@@ -424,6 +424,8 @@ def run_decode(args, cfg, world, rank, local, steps, e2e_steps, cpu_baseline):
         bb.set_option(vc.OPT_FRAME, 0)
     if args.frame:
         bb.set_option(vc.OPT_FRAME, 1)
+    if args.gemv_shape is not None:
+        bb.set_option(vc.OPT_GEMV_SHAPE, args.gemv_shape)
     frame = bb.uses_frame_kernel(B)
     st = dm.new_state(B, cap)
     if cfg.random_state:
@@ -545,7 +547,8 @@ def run_decode(args, cfg, world, rank, local, steps, e2e_steps, cpu_baseline):
                        [int(ctx0.min()), int(ctx0.max())], "layers": cfg.n_layers, "weights": synth.FMT_NAMES[cfg.wfmt],
                        "group": cfg.group_size, "heads": synth.FMT_NAMES[cfg.head_fmt],
                        "l2": f"no flush: {weight_total / 1e9:.2f} GB of weights per step >> 126 MB L2",
-                       "parallelism": f"replicas x{world}", "launch": launch},
+                       "parallelism": f"replicas x{world}", "launch": launch,
+                       **({"gemv_shape": args.gemv_shape} if args.gemv_shape is not None else {})},
             "achieved_step_gbs": step_gbs, "step_bytes_read": rbytes, "step_bytes_written": wbytes,
             "step_frac_of_peak": step_gbs / peak,
             "roofline": roofline, "gemv_kernel_alone": gemv_line,
@@ -581,6 +584,8 @@ def main():
                     help="run each frame as one kernel per operation")
     ap.add_argument("--frame", action="store_true",
                     help="run each frame as one launch of the frame kernel")
+    ap.add_argument("--gemv-shape", type=int, default=None, choices=[0, 1, 2],
+                    help="per-kernel path, up to 8 rows: SM occupancy of the streaming GEMV (VC_OPT_GEMV_SHAPE)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     cfg = synth.CONFIGS[args.config]

@@ -170,10 +170,18 @@ vc_status vc_backbone_create(const vc_config* cfg, const vc_weights* weights, vo
  * where it covers the backbone's formats and shapes; 0 = one kernel per operation, default),
  * VC_OPT_GRAPH (per-kernel path: 1 = capture and replay one CUDA graph per call signature,
  * default; 0 = launch the kernels directly), VC_OPT_PDL (per-kernel path: 1 = programmatic
- * dependent launch, default) */
+ * dependent launch, default), VC_OPT_GEMV_SHAPE (per-kernel path, projections of up to 8 rows:
+ * how the streaming GEMV occupies an SM; 0 = two 8-warp CTAs per SM, each with half of the ring
+ * budget (default); 1 = one 8-warp CTA per SM with half of the ring budget, so that a CTA of the
+ * next projection fits beside it and, under programmatic dependent launch, issues its first
+ * weight copies while this one runs; 2 = one 8-warp CTA per SM with the whole ring budget
+ * (deeper rings, no room beside it).  On a B200, 0 gives the fastest step (fewer resident warps
+ * per SM cost more than the prefetch or the deeper rings gain).  The results agree up to the order
+ * of fp32 sums; other values give VC_ERR_INVALID_ARG) */
 #define VC_OPT_GRAPH 1
 #define VC_OPT_PDL 2
 #define VC_OPT_FRAME 3
+#define VC_OPT_GEMV_SHAPE 4
 vc_status vc_set_option(vc_backbone* h, int option, int value);
 
 /* 1 if a vc_step of B rows on this backbone runs as one launch of the frame kernel (the option is

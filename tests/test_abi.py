@@ -36,6 +36,18 @@ def test_library_exports_every_declared_symbol():
     assert set(vc.EXPORTS) <= set(declared_functions())
 
 
+def test_option_numbers_match_the_header():
+    """every VC_OPT_* the header defines has the same number in the binding, and vc_set_option
+    refuses a NULL handle on the host"""
+    import attention_frame_decode_b200 as vc
+    src = open(os.path.join(ROOT, "include", "vc.h")).read()
+    opts = dict(re.findall(r"#define VC_(OPT_[A-Z_]+) (\d+)", src))
+    assert set(opts) == {"OPT_GRAPH", "OPT_PDL", "OPT_FRAME", "OPT_GEMV_SHAPE"}
+    for name, num in opts.items():
+        assert getattr(vc, name) == int(num), name
+    assert vc.lib().vc_set_option(None, vc.OPT_GEMV_SHAPE, 1) == vc.VC_ERR_INVALID_ARG
+
+
 def test_weight_bytes_and_workspace_host_only():
     import attention_frame_decode_b200 as vc
     import synth

@@ -191,6 +191,23 @@ def test_nano_layers_both_paths(cuda, frame, wfmt, group, B):
         assert rel(hid[layer], ro["hidden"][layer]) < HID_TOL, layer
 
 
+@pytest.mark.parametrize("shape", [1, 2])
+@pytest.mark.parametrize("wfmt,group,B", [(synth.FMT_W4, 64, 1), (synth.FMT_BF16, 64, 3), (synth.FMT_W3, 64, 8)])
+def test_nano_layers_gemv_shapes(cuda, shape, wfmt, group, B):
+    """one layer of each kind at the Nano widths with the streaming GEMV on one CTA per SM
+    (VC_OPT_GEMV_SHAPE 1 and 2), graph-captured, against the oracle over two frames"""
+    import attention_frame_decode_b200 as vc
+    cfg = nano_layer_cfg("M*-", wfmt, group)
+    ctx = synth.uniform_i32(9, 0, (B,), 10, 300)
+    run = Run(cfg, 5, B, 512, ctx_lens=ctx)
+    run.bb.set_option(vc.OPT_GEMV_SHAPE, shape)
+    run.bb.set_taps(run.hid, run.lg)
+    for t in range(2):
+        ro = run.step(t)
+        check_step(run, ro)
+    assert int(run.st.status.cpu()[0]) == 0
+
+
 # ------------------------------------------------------------------------------------------------
 # single layers at the Nano-9B-v2 widths
 # ------------------------------------------------------------------------------------------------
