@@ -34,12 +34,12 @@ static constexpr int kMaxSlots = 8;  // ring slots per warp (upper bound)
 // ------------------------------------------------------------------------------------------
 // With T (W + 1) < 2^32 (every shape of the backbone) the same integer quotients are taken in
 // 32-bit arithmetic, which costs a fraction of a 64-bit division.
-__device__ __forceinline__ long long part_begin(long long w, long long T, long long W, bool s32) {
+__host__ __device__ __forceinline__ long long part_begin(long long w, long long T, long long W, bool s32) {
     if (s32) return (long long)((uint32_t)w * (uint32_t)T / (uint32_t)W);
     return w * T / W;
 }
 // largest worker whose range starts at or before block f (always a non-empty range)
-__device__ __forceinline__ long long part_owner(long long f, long long T, long long W, bool s32) {
+__host__ __device__ __forceinline__ long long part_owner(long long f, long long T, long long W, bool s32) {
     if (s32) return (long long)(((uint32_t)(f + 1) * (uint32_t)W + (uint32_t)T - 1u) / (uint32_t)T) - 1;
     return ((f + 1) * W + T - 1) / T - 1;
 }
@@ -53,7 +53,7 @@ struct WarpRange {
     int f0, f1;            // block range [f0, f1)
 };
 
-__device__ __forceinline__ WarpRange warp_range(const GemvMat (&mat)[2], int nmat, long long wid, long long Wall) {
+__host__ __device__ __forceinline__ WarpRange warp_range(const GemvMat (&mat)[2], int nmat, long long wid, long long Wall) {
     WarpRange r;
     r.m = 0;
     r.Wm = Wall;
