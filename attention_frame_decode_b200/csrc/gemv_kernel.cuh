@@ -277,7 +277,7 @@ cudaError_t launch_t(const GemvLaunch& Lh, const GemvArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     // shape 1: the largest shared-memory carveout, so that a CTA of the next launch can fit beside
     // this one; the preference stays with the kernel, so once shape 1 has been used in the process
-    // the other shapes set it back to the driver's choice (untouched otherwise)
+    // the other shapes set it back to the default preference (untouched otherwise)
     static std::atomic<bool> carveout_set{false};
     if (shape == 1) carveout_set.store(true);
     if (e == cudaSuccess && carveout_set.load())

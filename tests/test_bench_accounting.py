@@ -64,7 +64,7 @@ def test_reference_arm_line_on_the_tiny_workload():
 
 
 def test_reference_arm_under_torchrun_prints_once():
-    """launched like the driver's N > 1 runs (torchrun, two local ranks on 127.0.0.1), only rank 0
+    """launched as N > 1 runs are (torchrun, two local ranks on 127.0.0.1), only rank 0
     runs the oracle and prints; the other rank exits 0 without work"""
     import json
     import os
