@@ -6,7 +6,9 @@ Default workload: the Nemotron-Nano-9B-v2-shaped backbone with W4 group-64 weigh
 batch 1, steady state decode at a context of 2000 frames (KV cache and SSM state pre-filled from
 N(0,1)), synthetic seeded weights N(0, 0.02) and inputs N(0, 1).  One "step" is one frame through
 all 56 layers and both vocabulary heads.  The same run then measures the bf16-weight backbone
-(nano_bf16) for up to 300 steps and reports it under "also" (--no-second skips it).  Other
+(nano_bf16) for up to 300 steps and reports it under "also"; on one GPU it then runs W3 at batch
+1, W8 g128 with 16 ragged sessions and the 4096-frame prefill, each as a short bench.py process of
+its own, and adds their numbers under "also" too (--no-second skips all of these).  Other
 workloads: --config nano_bf16 | nano_w3 | nano_w4_qheads | nano_w8_b16 | tiny_w8 (see
 synth.CONFIGS), and nano_prefill: one step is then one prefill of the 4096-frame opening context
 (tensor-core GEMMs, chunked SSD, causal attention).
@@ -562,6 +564,55 @@ def run_decode(args, cfg, world, rank, local, steps, e2e_steps, cpu_baseline):
     return line if rank == 0 else None
 
 
+# the other configurations of the metric, measured after the default workload in the same
+# single-GPU run: W3 at batch 1, W8 g128 with 16 ragged sessions, and the opening-context prefill
+EXTRA_CONFIGS = ("nano_w3", "nano_w8_b16", "nano_prefill")
+EXTRA_KEYS = ("value", "unit", "ms_per_step", "steps", "warmup", "achieved_step_gbs", "step_frac_of_peak",
+              "step_tflops", "e2e", "clocks", "device_status")
+
+
+def extra_command(name, steps, warmup):
+    """the bench.py command line of one further configuration (a short run of its own)"""
+    cfg = synth.CONFIGS[name]
+    n = 3 if cfg.prefill_T else max(1, min(steps, 300))
+    return [sys.executable, os.path.join(ROOT, "bench.py"), "--config", name, "--steps", str(n),
+            "--warmup", str(max(3, min(warmup, 10))), "--no-cpu-baseline", "--e2e-steps", "20"]
+
+
+def extra_summary(line):
+    """the numbers of a further configuration's JSON line that go under "also\" """
+    out = {k: line[k] for k in EXTRA_KEYS if k in line}
+    out["roofline_frac"] = line["roofline"]["frac"]
+    out["config"] = line["config"]
+    return out
+
+
+def run_extras(args, budget_s=420.0, run=subprocess.run):
+    """each further configuration as its own process on the same GPU (so that a failure there
+    leaves the default workload's line intact); a configuration that fails or would start after
+    `budget_s` seconds is recorded with the reason instead of numbers"""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "LOCAL_WORLD_SIZE",
+                                                              "MASTER_ADDR", "MASTER_PORT")}
+    out = {}
+    t0 = time.perf_counter()
+    for name in EXTRA_CONFIGS:
+        if time.perf_counter() - t0 > budget_s:
+            out[name] = {"skipped": f"time budget of {budget_s:.0f} s for the further configurations spent"}
+            continue
+        try:
+            r = run(extra_command(name, args.steps, args.warmup), capture_output=True, text=True, timeout=300,
+                    env=env, cwd=ROOT)
+            lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+            if r.returncode != 0 or not lines:
+                tail = (r.stderr or r.stdout).strip().splitlines()[-1:] or [""]
+                out[name] = {"error": f"exit {r.returncode}: {tail[0][:300]}"}
+            else:
+                out[name] = extra_summary(json.loads(lines[-1]))
+        except Exception as e:   # a timeout or an unreadable line: recorded, the default line stands
+            out[name] = {"error": f"{type(e).__name__}: {str(e)[:300]}"}
+    return out
+
+
 # ------------------------------------------------------------------------------------------------
 # GPU arm
 # ------------------------------------------------------------------------------------------------
@@ -622,6 +673,12 @@ def main():
                                                                   "e2e", "clocks")}}
             line["also"]["nano_bf16"]["roofline_frac"] = second["roofline"]["frac"]
             line["gpu_launches"] += second["gpu_launches"]
+        if world == 1:
+            # the further configurations, after this run's own timed regions (not counted in its
+            # gpu_launches)
+            del second
+            torch.cuda.empty_cache()
+            line["also"].update(run_extras(args))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -107,3 +107,40 @@ def test_decode_launch_count():
     the ncu launch lists of the step)"""
     assert bench.launches_per_step(synth.CONFIGS["nano_bf16"]) == 145
     assert bench.launches_per_step(synth.CONFIGS["tiny_w8"]) == 1 + 3 + 2 + 3 + 2 + 1
+
+
+def test_further_configurations_of_the_default_run():
+    """the default run measures W3, 16 sessions and the prefill as short runs of their own (one
+    process each): their command lines, the summary kept under "also", and that a failing or late
+    configuration is recorded without numbers while the others still report"""
+    import json
+    import subprocess
+    from types import SimpleNamespace
+
+    cmd = bench.extra_command("nano_w3", 20, 5)
+    assert cmd[cmd.index("--steps") + 1] == "20" and cmd[cmd.index("--warmup") + 1] == "5"
+    assert "--no-cpu-baseline" in cmd and cmd[cmd.index("--config") + 1] == "nano_w3"
+    cmd = bench.extra_command("nano_prefill", 1000, 20)
+    assert cmd[cmd.index("--steps") + 1] == "3" and cmd[cmd.index("--warmup") + 1] == "10"
+    assert bench.extra_command("nano_w8_b16", 1000, 1)[4:8] == ["--steps", "300", "--warmup", "3"]
+
+    calls = []
+
+    def fake_run(cmd, **kw):
+        name = cmd[cmd.index("--config") + 1]
+        calls.append((name, kw.get("env", {})))
+        if name == "nano_w8_b16":
+            return subprocess.CompletedProcess(cmd, 1, "", "Traceback ...\nRuntimeError: out of memory\n")
+        line = {"value": 12.5, "unit": "u", "ms_per_step": 3.0, "steps": 20, "roofline": {"frac": 0.25},
+                "config": {"workload": name}, "e2e": {"value": 12.0}, "clocks": {"sm_mhz": 1965.0}}
+        return subprocess.CompletedProcess(cmd, 0, "noise\n" + json.dumps(line) + "\n", "")
+
+    out = bench.run_extras(SimpleNamespace(steps=20, warmup=5), run=fake_run)
+    assert [c[0] for c in calls] == list(bench.EXTRA_CONFIGS)
+    assert all("RANK" not in env and "WORLD_SIZE" not in env for _, env in calls)
+    assert out["nano_w3"]["roofline_frac"] == 0.25 and out["nano_w3"]["value"] == 12.5
+    assert out["nano_w3"]["config"] == {"workload": "nano_w3"}
+    assert out["nano_w8_b16"] == {"error": "exit 1: RuntimeError: out of memory"}
+    assert out["nano_prefill"]["ms_per_step"] == 3.0
+    late = bench.run_extras(SimpleNamespace(steps=20, warmup=5), budget_s=-1.0, run=fake_run)
+    assert all("skipped" in late[n] for n in bench.EXTRA_CONFIGS)
