@@ -676,7 +676,9 @@ def main():
         if world == 1:
             # the further configurations, after this run's own timed regions (not counted in its
             # gpu_launches)
+            import gc
             del second
+            gc.collect()
             torch.cuda.empty_cache()
             line["also"].update(run_extras(args))
     if rank == 0:
