@@ -587,7 +587,7 @@ def extra_summary(line):
     return out
 
 
-def run_extras(args, budget_s=420.0, run=subprocess.run):
+def run_extras(args, budget_s=300.0, run=subprocess.run):
     """each further configuration as its own process on the same GPU (so that a failure there
     leaves the default workload's line intact); a configuration that fails or would start after
     `budget_s` seconds is recorded with the reason instead of numbers"""
@@ -600,7 +600,7 @@ def run_extras(args, budget_s=420.0, run=subprocess.run):
             out[name] = {"skipped": f"time budget of {budget_s:.0f} s for the further configurations spent"}
             continue
         try:
-            r = run(extra_command(name, args.steps, args.warmup), capture_output=True, text=True, timeout=300,
+            r = run(extra_command(name, args.steps, args.warmup), capture_output=True, text=True, timeout=240,
                     env=env, cwd=ROOT)
             lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
             if r.returncode != 0 or not lines:
