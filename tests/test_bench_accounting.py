@@ -144,3 +144,34 @@ def test_further_configurations_of_the_default_run():
     assert out["nano_prefill"]["ms_per_step"] == 3.0
     late = bench.run_extras(SimpleNamespace(steps=20, warmup=5), budget_s=-1.0, run=fake_run)
     assert all("skipped" in late[n] for n in bench.EXTRA_CONFIGS)
+
+
+def test_default_run_assembles_one_line(monkeypatch, capsys):
+    """main() of the default run on one GPU, with the measurements faked on the host: one JSON line
+    whose "also" holds the bf16 backbone and the further configurations, and whose gpu_launches
+    counts the two timed decode runs only"""
+    import json
+    import sys
+    import torch
+
+    def fake_decode(args, cfg, world, rank, local, steps, e2e_steps, cpu_baseline):
+        return {"metric": bench.METRIC, "value": 1.0 if cfg.name == bench.DEFAULT_CONFIG else 2.0,
+                "unit": "frame-steps/s", "ms_per_step": 3.0, "steps": steps, "achieved_step_gbs": 1.0,
+                "step_frac_of_peak": 0.5, "e2e": {"value": 1.0}, "clocks": {}, "roofline": {"frac": 0.4},
+                "gpu_launches": 100 if cfg.name == bench.DEFAULT_CONFIG else 7, "config": {"workload": cfg.name}}
+
+    monkeypatch.setattr(bench, "run_decode", fake_decode)
+    monkeypatch.setattr(bench, "run_extras", lambda args: {n: {"value": 3.0} for n in bench.EXTRA_CONFIGS})
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a: None)
+    monkeypatch.setattr(torch.cuda, "empty_cache", lambda *a: None)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "20", "--warmup", "5"])
+    bench.main()
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["config"]["workload"] == bench.DEFAULT_CONFIG and line["value"] == 1.0
+    assert set(line["also"]) == {"nano_bf16", *bench.EXTRA_CONFIGS}
+    assert line["also"]["nano_bf16"]["value"] == 2.0 and line["also"]["nano_bf16"]["roofline_frac"] == 0.4
+    assert line["gpu_launches"] == 107
