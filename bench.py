@@ -115,6 +115,15 @@ def replica_rate(units_per_rank: float, world: int, seconds: float) -> float:
     return world * units_per_rank / seconds
 
 
+def latency_ms(durations_s):
+    """mean, median and 95th percentile (ms) of per-step wall times in seconds, as the pages report a
+    frame's latency (mean and p95)"""
+    d = np.asarray(durations_s, np.float64) * 1000.0
+    if d.size == 0:
+        return {"mean_ms": None, "p50_ms": None, "p95_ms": None}
+    return {"mean_ms": float(d.mean()), "p50_ms": float(np.percentile(d, 50)), "p95_ms": float(np.percentile(d, 95))}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -361,11 +370,14 @@ def run_prefill_bench(args, cfg, world, rank, local):
     ne = max(2, min(args.steps, 10))
     torch.cuda.synchronize()
     t0 = time.perf_counter()
+    lat = []
     for _ in range(ne):
+        t1 = time.perf_counter()
         xd.copy_(xh, non_blocking=True)
         bb.prefill(xd, 0, st)
         ch.copy_(st.ctx_len[:1], non_blocking=True)
         stream.synchronize()
+        lat.append(time.perf_counter() - t1)
     e2e_s = time.perf_counter() - t0
     assert int(ch[0]) == T
     e2e_value = world * T * ne / e2e_s
@@ -394,7 +406,7 @@ def run_prefill_bench(args, cfg, world, rank, local):
                          "flops_per_launch": 2.0 * M * N * K},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "frames/s", "h2d_bytes_per_step": T * cfg.d_model * 2,
-                    "d2h_bytes_per_step": 4, "steps": ne},
+                    "d2h_bytes_per_step": 4, "steps": ne, "prefill_latency": latency_ms(lat)},
             "gpu_launches": n_launch * args.steps, "clocks": clk, "device_status": int(st.status.cpu()[0]),
         }
         print(json.dumps(line), flush=True)
@@ -507,9 +519,12 @@ def run_decode(args, cfg, world, rank, local, steps, e2e_steps, cpu_baseline):
     if world > 1:
         dist.barrier()
     t0 = time.perf_counter()
+    lat = []
     for s in range(1, ne):
+        t1 = time.perf_counter()
         bb.step_host(xh[s], st, th, fh)
         stream.synchronize()   # the frame's tokens are on the host before the next frame
+        lat.append(time.perf_counter() - t1)
     e2e_s = time.perf_counter() - t0
     e2e_s = max_over_ranks(e2e_s, world)
     e2e_value = world * B * (ne - 1) / e2e_s
@@ -556,7 +571,7 @@ def run_decode(args, cfg, world, rank, local, steps, e2e_steps, cpu_baseline):
             "roofline": roofline, "gemv_kernel_alone": gemv_line,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "frame-steps/s", "h2d_bytes_per_step": B * cfg.d_model * 2,
-                    "d2h_bytes_per_step": 2 * B * 4, "steps": ne - 1},
+                    "d2h_bytes_per_step": 2 * B * 4, "steps": ne - 1, "frame_latency": latency_ms(lat)},
             "gpu_launches": n_launches,
             "clocks": clk, "device_status": status,
         }

@@ -175,3 +175,14 @@ def test_default_run_assembles_one_line(monkeypatch, capsys):
     assert set(line["also"]) == {"nano_bf16", *bench.EXTRA_CONFIGS}
     assert line["also"]["nano_bf16"]["value"] == 2.0 and line["also"]["nano_bf16"]["roofline_frac"] == 0.4
     assert line["gpu_launches"] == 107
+
+
+def test_latency_summary():
+    """per-step wall times (s) -> mean, median and 95th percentile in ms (linear interpolation
+    between order statistics, numpy's default)"""
+    d = [0.001 * i for i in range(1, 101)]          # 1 .. 100 ms
+    r = bench.latency_ms(d)
+    assert abs(r["mean_ms"] - 50.5) < 1e-9
+    assert abs(r["p50_ms"] - 50.5) < 1e-9
+    assert abs(r["p95_ms"] - 95.05) < 1e-9
+    assert bench.latency_ms([]) == {"mean_ms": None, "p50_ms": None, "p95_ms": None}
