@@ -3,6 +3,7 @@
     python -m attention_frame_decode_b200.kernel_cases gemv --fmt w4 --n 15680 --k 4480
     python -m attention_frame_decode_b200.kernel_cases gemm --m 4096 --n 15680 --k 4480
     python -m attention_frame_decode_b200.kernel_cases ssd --frames 1024
+    python -m attention_frame_decode_b200.kernel_cases attn --batch 16
 
 Each case builds its inputs on the device from the seeded generators, runs the kernel a few
 times, and prints the mean time of `--reps` further launches measured with CUDA events.  The
@@ -118,6 +119,38 @@ def case_mamba(a):
     bb.close()
 
 
+def case_attn(a):
+    """decode frames of one Nano attention layer (W8 g128 projections) for `batch` sessions whose
+    K/V caches hold contexts drawn U(500, 6000) (a fixed 2000 for one session), launched kernel by
+    kernel: its split-K decode attention is the kernel of interest"""
+    import numpy as np
+    import torch
+    import attention_frame_decode_b200 as vc
+    import synth
+    from attention_frame_decode_b200.synthetic import build_model, fill_state
+    B = a.batch
+    cfg = synth.nano_config(name="nano_attn_layer", pattern="*", wfmt=synth.FMT_W8, group_size=128,
+                            vocab_text=4096, vocab_func=2048, batch=B,
+                            ctx_range=None if B == 1 else (500, 6000), kv_capacity=7000)
+    ctx = synth.context_lengths(cfg, 0, B)
+    cap = int(ctx.max()) + a.warmup + a.reps + 8
+    dm = build_model(cfg, 0)
+    bb = dm.backbone(B, cap, B)
+    bb.set_option(vc.OPT_GRAPH, 0)
+    st = dm.new_state(B, cap)
+    fill_state(st, cfg, 0, ctx, cap)
+    tt = torch.zeros((B,), dtype=torch.int32, device="cuda")
+    tf = torch.zeros_like(tt)
+    x = torch.from_numpy(synth.frame_inputs(cfg, 0, 0, B)).cuda().view(torch.bfloat16)
+    run = lambda: bb.step(x, st, tt, tf)
+    for _ in range(a.warmup):
+        run()
+    us = _time(run, a.reps)
+    print(f"one Nano attention layer + heads, {B} sessions, contexts {int(ctx.min())}..{int(ctx.max())}: "
+          f"{us:.1f} us/step, status {int(st.status.cpu()[0])}")
+    bb.close()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     sub = ap.add_subparsers(dest="case", required=True)
@@ -135,11 +168,13 @@ def main(argv=None):
     s.add_argument("--frames", type=int, default=1024)
     mb = sub.add_parser("mamba")
     mb.add_argument("--batch", type=int, default=16)
-    for p in (g, m, s, mb):
+    at = sub.add_parser("attn")
+    at.add_argument("--batch", type=int, default=16)
+    for p in (g, m, s, mb, at):
         p.add_argument("--warmup", type=int, default=3)
         p.add_argument("--reps", type=int, default=20)
     a = ap.parse_args(argv)
-    {"gemv": case_gemv, "gemm": case_gemm, "ssd": case_ssd, "mamba": case_mamba}[a.case](a)
+    {"gemv": case_gemv, "gemm": case_gemm, "ssd": case_ssd, "mamba": case_mamba, "attn": case_attn}[a.case](a)
 
 
 if __name__ == "__main__":
